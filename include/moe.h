@@ -1,0 +1,173 @@
+/*
+ * moe.h -- C ABI of libmoe: forward pass of one DeepSeek-V3-style
+ * mixture-of-experts feed-forward layer on one NVIDIA B200 (sm_100a).
+ *
+ * What the layer computes (sources are the web pages this library follows):
+ *   logits = x Wg^T                       gate, a linear layer without bias
+ *       ("DeepSeek-V3's mixture-of-experts architecture explained", n4n.ai,
+ *        section "The architecture in one diagram", simplified block code)
+ *   idx, w = route(logits)                top-k then softmax over the k
+ *       (same section), or the sigmoid group-limited rule with selection
+ *       bias (MOE_ROUTE_SIGMOID_GROUP, below)
+ *   expert(x) = W2^T (silu(x W1) * (x W3))   SwiGLU, "All 5 steps" of
+ *       "DeepSeek-V3.2-Exp / Mixture of experts / Shared expert" (atlas page)
+ *   y[t] = sum_j w[t,j] expert_{idx[t,j]}(x[t]) + shared(x[t])
+ *       (atlas page, MoE forward excerpt model.py 790-803: per-expert token
+ *        lists from bincount/where, an fp32 accumulator, then the shared
+ *        expert added to every token)
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller, contiguous
+ *    row-major, 16-byte aligned (the tensor-memory-accelerator copies require
+ *    it).  The library never allocates, frees or keeps a pointer after a call
+ *    returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default
+ *    stream) and never synchronise the host, except moe_check_device_status.
+ *  - Arguments are validated on the host before any launch; an invalid call
+ *    returns an error and launches nothing.  T == 0 is valid and does nothing.
+ *  - Dtypes: x, Wg, the shared expert and bf16 routed weights are bfloat16.
+ *    FP8 routed weights are OCP e4m3 codes (one byte) with one fp32 scale per
+ *    128 x 128 block.  Logits, routing weights and the combine accumulate in
+ *    fp32; all tensor-core contractions accumulate in fp32.
+ *  - `ws` is a caller-allocated device workspace of at least
+ *    moe_workspace_size(shape) bytes (256-byte aligned).  Its first 4 bytes
+ *    are the device status word (see moe_check_device_status); the rest is
+ *    scratch whose contents do not survive between calls.  Calls that overlap
+ *    on the device must use different workspaces.
+ *  - Identical inputs give bit-identical outputs (no floating-point atomics).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,    /* null required pointer, misaligned pointer, bad size */
+  MOE_ERR_UNSUPPORTED = 2,    /* shape/dtype combination this library does not implement */
+  MOE_ERR_WORKSPACE = 3,      /* ws null or smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 4,           /* a CUDA runtime/driver call or a launch failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait gave up (reported by moe_check_device_status) */
+  MOE_ERR_DEVICE_BOUNDS = 6   /* an expert index outside [0, E) was seen and skipped */
+} moe_status;
+
+typedef enum { MOE_BF16 = 0, MOE_E4M3 = 1, MOE_F32 = 2 } moe_dtype;
+
+typedef enum {
+  /* top-k of the logits (descending, lowest index first on ties), softmax
+   * over the k selected logits (n4n.ai page, "The architecture in one
+   * diagram"). */
+  MOE_ROUTE_TOPK_SOFTMAX = 0,
+  /* s = sigmoid(logit), sel = s + bias; experts form n_group contiguous
+   * groups of E/n_group; a group's score is the sum of its group_topn best
+   * sel; the topk_group best groups are kept; the k best sel among their
+   * experts are chosen; w = route_scale * s / sum(s) over the chosen
+   * (DeepSeek-V3 group-limited routing; the pages only outline it: Baidu
+   * page "Hierarchical Dynamic Routing", freedom251 page "How V3 balances
+   * expert traffic"). */
+  MOE_ROUTE_SIGMOID_GROUP = 1
+} moe_route;
+
+typedef struct {
+  int64_t T;            /* tokens (rows of x); 0 <= T, T*k < 2^31 */
+  int32_t d;            /* model width (7168); multiple of 128 */
+  int32_t E;            /* routed experts (256); multiple of 32, <= 1024 */
+  int32_t k;            /* experts per token (8); 1 <= k <= min(E, 32) */
+  int32_t inter;        /* routed expert width (moe_inter_dim, 2048); multiple of 128 */
+  int32_t shared_inter; /* shared expert width (n_shared x moe_inter = 2048); 0 = none; multiple of 128 */
+  int32_t route;        /* moe_route */
+  int32_t n_group;      /* group mode: groups (8); divides E; E/n_group <= 64; n_group <= 32 */
+  int32_t topk_group;   /* group mode: kept groups (4); topk_group*E/n_group >= k */
+  int32_t group_topn;   /* group mode: experts summed per group score (2) */
+  float route_scale;    /* group mode: weight scale (2.5); ignored in top-k/softmax mode */
+  int32_t w_dtype;      /* routed expert weights: MOE_BF16 or MOE_E4M3 */
+  int32_t y_dtype;      /* output y: MOE_F32 (the pages' fp32 accumulator) or MOE_BF16 */
+} moe_shape;
+
+/* Bytes of workspace every entry point below needs for `shape` (the maximum
+ * over them).  Returns 0 when the shape is invalid or unsupported. */
+size_t moe_workspace_size(const moe_shape* shape);
+
+/* Router: logits = x Wg^T in fp32 (tensor cores; each 64-term partial sum is
+ * accumulated in fp64), then the k experts per token and their weights.
+ *   x        [T, d] bf16            Wg [E, d] bf16
+ *   bias     [E] fp32 selection bias, group mode only (may be NULL = zeros)
+ *   topk_idx [T, k] int32 out, slots in descending score order
+ *   topk_w   [T, k] fp32 out
+ *   logits   [T, E] fp32 out, optional (NULL: kept in the workspace)
+ * Source: n4n.ai page "The architecture in one diagram" (gate, topk, softmax). */
+moe_status moe_router_topk(const moe_shape* shape, const void* x, const void* Wg, const float* bias,
+                           int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Dispatch: counts = bincount(topk_idx, minlength=E); offsets = exclusive
+ * prefix sum (E+1 entries); the permuted order lists experts ascending and,
+ * within an expert, its (token, slot) entries ascending -- the order of the
+ * atlas page's torch.where(indices == i) (model.py 790-803 excerpt).
+ *   perm_token [T*k] int32 out: token at permuted position r
+ *   row_of     [T*k] int32 out: permuted position of entry (t, j) at t*k + j
+ *   x, x_perm  optional pair: when both are non-NULL, x_perm [T*k, d] bf16
+ *              receives x[perm_token[r]] at row r.
+ * An index outside [0, E) is skipped (its row_of is -1) and raises
+ * MOE_ERR_DEVICE_BOUNDS in the workspace status word. */
+moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                       int32_t* perm_token, int32_t* row_of, const void* x, void* x_perm, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Grouped SwiGLU experts over the permuted rows plus the shared expert:
+ *   for each expert e and each permuted row r in [offsets[e], offsets[e+1]):
+ *     Y_perm[r] = bf16( (bf16(silu(x_perm[r] W1[e]) * (x_perm[r] W3[e]))) W2[e] )
+ *   for each token t (shared expert, when shape->shared_inter > 0):
+ *     Y_shared[t] = (bf16(silu(x[t] W1s) * (x[t] W3s))) W2s   in fp32
+ *   x [T, d] bf16; x_perm [T*k, d] bf16 (from moe_permute); offsets [E+1]
+ *   W1, W3 [E, d, inter], W2 [E, inter, d]: bf16, or e4m3 codes when
+ *     w_dtype == MOE_E4M3 with fp32 block scales s1, s3 [E, d/128, inter/128]
+ *     and s2 [E, inter/128, d/128] (dequantised value = code * scale)
+ *   W1s, W3s [d, shared_inter], W2s [shared_inter, d] bf16 (NULL when none)
+ *   Y_perm [T*k, d] bf16 out; Y_shared [T, d] fp32 out (NULL when none)
+ * Source: atlas page "All 5 steps" and the model.py 643 excerpt (silu and
+ * product in fp32, h cast to the activation dtype before W2). */
+moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const void* x_perm, const int32_t* offsets,
+                              const void* W1, const void* W3, const void* W2, const float* s1, const float* s3,
+                              const float* s2, const void* W1s, const void* W3s, const void* W2s, void* Y_perm,
+                              float* Y_shared, void* ws, size_t ws_bytes, void* stream);
+
+/* Combine: y[t] = Y_shared[t] + sum_j topk_w[t,j] * Y_perm[row_of[t*k+j]],
+ * summed in fp32 in slot order, written as shape->y_dtype.  Y_shared may be
+ * NULL (no shared expert).  Source: atlas page model.py 790-803 excerpt. */
+moe_status moe_combine(const moe_shape* shape, const void* Y_perm, const float* Y_shared, const int32_t* row_of,
+                       const float* topk_w, void* y, void* stream);
+
+/* The whole layer: router, dispatch, grouped experts, shared expert and
+ * combine, with no host synchronisation.
+ *   y [T, d] out (fp32 or bf16 per shape->y_dtype)
+ *   topk_idx_out [T, k], topk_w_out [T, k], counts_out [E]: optional copies
+ *   of the routing (NULL = not returned). */
+moe_status moe_forward(const moe_shape* shape, const void* x, const void* Wg, const float* bias, const void* W1,
+                       const void* W3, const void* W2, const float* s1, const float* s3, const float* s2,
+                       const void* W1s, const void* W3s, const void* W2s, void* y, int32_t* topk_idx_out,
+                       float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, reads the status word of `ws` written by the last
+ * call that used this workspace and returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT or
+ * MOE_ERR_DEVICE_BOUNDS (timeout wins when both are set); `raw` (optional)
+ * receives the raw bits.  Returns MOE_ERR_CUDA when the stream itself reports
+ * an error. */
+moe_status moe_check_device_status(const void* ws, void* stream, uint32_t* raw);
+
+/* Static description of a status code. */
+const char* moe_status_string(moe_status status);
+
+/* Library version string. */
+const char* moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

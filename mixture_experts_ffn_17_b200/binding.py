@@ -1,0 +1,157 @@
+"""ctypes binding of libmoe (include/moe.h): argument marshalling only.
+
+Every function takes torch CUDA tensors, passes their data pointers and the
+current CUDA stream to the C entry point of the same name, and raises
+MoeError on a non-OK status.  All computation happens in the library's
+kernels; nothing here computes on the host.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, \
+    MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS = range(7)
+MOE_BF16, MOE_E4M3, MOE_F32 = 0, 1, 2
+MOE_ROUTE_TOPK_SOFTMAX, MOE_ROUTE_SIGMOID_GROUP = 0, 1
+
+EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
+            "moe_forward", "moe_check_device_status", "moe_status_string", "moe_version")
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class MoeShape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("inter", ctypes.c_int32), ("shared_inter", ctypes.c_int32), ("route", ctypes.c_int32),
+                ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32), ("group_topn", ctypes.c_int32),
+                ("route_scale", ctypes.c_float), ("w_dtype", ctypes.c_int32), ("y_dtype", ctypes.c_int32)]
+
+
+def make_shape(T, d, E, k, inter, shared_inter, route=0, n_group=1, topk_group=1, group_topn=2,
+               route_scale=1.0, w_dtype=MOE_BF16, y_dtype=MOE_F32) -> MoeShape:
+    return MoeShape(int(T), int(d), int(E), int(k), int(inter), int(shared_inter), int(route), int(n_group),
+                    int(topk_group), int(group_topn), float(route_scale), int(w_dtype), int(y_dtype))
+
+
+def shape_of(cfg, y_dtype=MOE_F32) -> MoeShape:
+    """MoeShape of a workloads.Config."""
+    return make_shape(cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter, cfg.shared_inter, cfg.route, cfg.n_group,
+                      cfg.topk_group, cfg.group_topn, cfg.route_scale, MOE_E4M3 if cfg.fp8 else MOE_BF16, y_dtype)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so; raises when it is missing (there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmoe.so not built ({LIB_PATH}); run `python -m mixture_experts_ffn_17_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S, sz = ctypes.c_void_p, ctypes.POINTER(MoeShape), ctypes.c_size_t
+        L.moe_workspace_size.argtypes = [S]
+        L.moe_workspace_size.restype = sz
+        L.moe_router_topk.argtypes = [S, P, P, P, P, P, P, P, sz, P]
+        L.moe_permute.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_grouped_swiglu.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_combine.argtypes = [S, P, P, P, P, P, P]
+        L.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+        for fn in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward",
+                   "moe_check_device_status"):
+            getattr(L, fn).restype = ctypes.c_int
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_status_string.restype = ctypes.c_char_p
+        L.moe_version.argtypes = []
+        L.moe_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmoe must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != MOE_OK:
+        raise MoeError(rc, where)
+
+
+def workspace_size(shape: MoeShape) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(shape)))
+
+
+def alloc_workspace(shape: MoeShape, device="cuda") -> torch.Tensor:
+    n = workspace_size(shape)
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def router_topk(shape, x, Wg, bias, topk_idx, topk_w, logits, ws, stream=None):
+    _check(lib().moe_router_topk(ctypes.byref(shape), _ptr(x), _ptr(Wg), _ptr(bias), _ptr(topk_idx), _ptr(topk_w),
+                                 _ptr(logits), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
+           "moe_router_topk")
+
+
+def permute(shape, topk_idx, counts, offsets, perm_token, row_of, x, x_perm, ws, stream=None):
+    _check(lib().moe_permute(ctypes.byref(shape), _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(perm_token),
+                             _ptr(row_of), _ptr(x), _ptr(x_perm), _ptr(ws), ws.numel() if ws is not None else 0,
+                             _stream(stream)), "moe_permute")
+
+
+def grouped_swiglu(shape, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared, ws,
+                   stream=None):
+    _check(lib().moe_grouped_swiglu(ctypes.byref(shape), _ptr(x), _ptr(x_perm), _ptr(offsets), _ptr(W1), _ptr(W3),
+                                    _ptr(W2), _ptr(s1), _ptr(s3), _ptr(s2), _ptr(W1s), _ptr(W3s), _ptr(W2s),
+                                    _ptr(Y_perm), _ptr(Y_shared), _ptr(ws), ws.numel() if ws is not None else 0,
+                                    _stream(stream)), "moe_grouped_swiglu")
+
+
+def combine(shape, Y_perm, Y_shared, row_of, topk_w, y, stream=None):
+    _check(lib().moe_combine(ctypes.byref(shape), _ptr(Y_perm), _ptr(Y_shared), _ptr(row_of), _ptr(topk_w), _ptr(y),
+                             _stream(stream)), "moe_combine")
+
+
+def forward(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, ws, topk_idx=None, topk_w=None,
+            counts=None, stream=None):
+    _check(lib().moe_forward(ctypes.byref(shape), _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2),
+                             _ptr(s1), _ptr(s3), _ptr(s2), _ptr(W1s), _ptr(W3s), _ptr(W2s), _ptr(y), _ptr(topk_idx),
+                             _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel() if ws is not None else 0,
+                             _stream(stream)), "moe_forward")
+
+
+def check_device_status(ws, stream=None) -> tuple[int, int]:
+    raw = ctypes.c_uint32(0)
+    rc = lib().moe_check_device_status(_ptr(ws), _stream(stream), ctypes.byref(raw))
+    return rc, raw.value
+
+
+def version() -> str:
+    return lib().moe_version().decode()

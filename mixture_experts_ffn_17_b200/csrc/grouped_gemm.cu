@@ -1,0 +1,346 @@
+// grouped_gemm.cu -- the expert contractions on the 5th-generation tensor cores.
+//
+// SwiGLU expert ("DeepSeek-V3.2-Exp / Mixture of experts / Shared expert",
+// "All 5 steps"): g = x W1, u = x W3, a = g sigmoid(g), h = a * u, y = h W2.
+// The page's code applies silu and the product in fp32 and casts h to the
+// activation dtype before W2 (model.py 643 excerpt); here h is stored bf16.
+//
+// Both kernels are persistent (one CTA per SM) and walk a device-side tile
+// list: one entry per 128-row slice of an expert's segment of permuted rows,
+// plus the shared expert (group E) over all T tokens.  Tile t -> (row tile
+// t / n_nb, column block t % n_nb).  Warp roles:
+//   warp 0    TMA producer: A tile [128 rows x 64 K] (K-major, 128B swizzle)
+//             and B tiles [64 K x 64 N] boxes (N-major, the weights' natural
+//             [K, N] row-major layout) into a 4-stage ring;
+//   warp 1    single-thread tcgen05.mma issuer, M=128, K=16 per instruction,
+//             fp32 accumulators in TMEM, two accumulator buffers so the
+//             epilogue of one tile overlaps the main loop of the next;
+//   warps 2-5 epilogue: tcgen05.ld the accumulator rows (one row per
+//             thread), apply silu(g)*u (SwiGLU kernel) and store.
+//
+// Kernel A (SwiGLU):  N = 128 columns of W1 and the same 128 of W3 per tile
+//                     (two MMAs per K step into two 128-column accumulators),
+//                     H[row, n0:n0+128] = bf16(silu(g) * u).
+// Kernel B (down):    N = 256 columns of W2 per tile; routed rows are stored
+//                     bf16 into Y_perm, shared-expert rows fp32 into Y_shared.
+#include <algorithm>
+#include <cstdint>
+
+#include "common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr uint32_t kABytes = kTileM * kBK * 2;  // 16 KB
+constexpr uint32_t kBoxBytes = 64 * kBK * 2;    // one [64 K x 64 N] bf16 box, 8 KB
+constexpr uint32_t kTmemCols = 512;             // 2 accumulator buffers x 256 columns
+
+enum class Mode { kSwiGLU, kDown };
+
+template <Mode M>
+struct Cfg;
+template <>
+struct Cfg<Mode::kSwiGLU> {
+  static constexpr int BN = 128;                    // per weight matrix
+  static constexpr uint32_t kBBytes = 2 * kBoxBytes;  // W1 part (W3 part follows)
+  static constexpr uint32_t kStageBytes = kABytes + 2 * kBBytes;
+};
+template <>
+struct Cfg<Mode::kDown> {
+  static constexpr int BN = 256;
+  static constexpr uint32_t kBBytes = 4 * kBoxBytes;
+  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+};
+
+template <Mode M>
+constexpr size_t smem_bytes() {
+  return 1024 + kStages * Cfg<M>::kStageBytes + 256;
+}
+
+struct TileInfo {
+  int group, row0, rows, nb;
+  bool shared;
+};
+
+__device__ __forceinline__ bool tile_at(const GemmParams& p, int tile, int BN, TileInfo& ti) {
+  const int mt = tile / p.n_nb;
+  ti.nb = tile - mt * p.n_nb;
+  const int4 e = p.tiles[mt];
+  ti.group = e.x;
+  ti.row0 = e.y;
+  ti.rows = e.z;
+  ti.shared = (e.x == p.E);
+  const int N = ti.shared ? p.N_shared : p.N_routed;
+  return ti.nb * BN < N;  // false: this column block does not exist for the group
+}
+
+template <Mode M>
+__global__ void __launch_bounds__(192, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
+                        const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
+                        const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s,
+                        const GemmParams p) {
+  using C = Cfg<M>;
+  constexpr int S = kStages;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* stage0 = align_1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage0 + S * C::kStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  __shared__ uint32_t never;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&tfull[b], 1);
+      ptx::mbar_init(&tempty[b], 128);
+    }
+    ptx::mbar_init(done, 1);
+    *abort_flag = 0u;
+    never = 0u;
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int total = min(p.ntiles[0], p.max_mtiles) * p.n_nb;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmA_r);
+      ptx::prefetch_tmap(&tmA_s);
+      ptx::prefetch_tmap(&tmB_r);
+      ptx::prefetch_tmap(&tmB_s);
+      if (M == Mode::kSwiGLU) {
+        ptx::prefetch_tmap(&tmC_r);
+        ptx::prefetch_tmap(&tmC_s);
+      }
+      const uint64_t pol_a = ptx::policy_evict_last();   // A rows are reused by every column block
+      const uint64_t pol_w = ptx::policy_evict_first();  // weights stream through once
+      int kg = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        TileInfo ti;
+        if (!tile_at(p, tile, BN, ti)) continue;
+        const CUtensorMap* mA = ti.shared ? &tmA_s : &tmA_r;
+        const CUtensorMap* mB = ti.shared ? &tmB_s : &tmB_r;
+        const CUtensorMap* mC = ti.shared ? &tmC_s : &tmC_r;
+        const int arow = ti.row0 + (ti.shared ? p.a_shared_row_offset : 0);
+        const int e3 = ti.shared ? 0 : ti.group;
+        const int nk = (ti.shared ? p.K_shared : p.K_routed) / kBK;
+        const int n0 = ti.nb * BN;
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % S;
+          const uint32_t ph = (kg / S) & 1;
+          if (!ptx::wait_bounded(&empty[s], ph ^ 1, abort_flag)) {
+            raise_status(p.status, abort_flag, kStatusTimeout);
+            ok = false;
+            break;
+          }
+          uint8_t* st = stage0 + s * C::kStageBytes;
+          ptx::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          ptx::tma_load_2d(st, mA, &full[s], kb * kBK, arow, pol_a);
+          uint8_t* sb = st + kABytes;
+#pragma unroll
+          for (int h = 0; h < BN / 64; ++h)
+            ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
+          if (M == Mode::kSwiGLU) {
+            uint8_t* sc = sb + C::kBBytes;
+#pragma unroll
+            for (int h = 0; h < BN / 64; ++h)
+              ptx::tma_load_3d(sc + h * kBoxBytes, mC, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
+          }
+        }
+      }
+      // every issued copy must land before the CTA may exit
+      for (int j = (kg > S ? kg - S : 0); j < kg; ++j)
+        if (!ptx::wait_bounded(&full[j % S], (j / S) & 1, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_bf16(kTileM, BN, false, true);
+      int kg = 0, it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        TileInfo ti;
+        if (!tile_at(p, tile, BN, ti)) continue;
+        const int nk = (ti.shared ? p.K_shared : p.K_routed) / kBK;
+        const int b = it & 1;
+        const uint32_t use = (uint32_t)it >> 1;
+        if (!ptx::wait_bounded(&tempty[b], (use & 1) ^ 1, abort_flag)) {
+          raise_status(p.status, abort_flag, kStatusTimeout);
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d0 = tmem + b * 256;
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % S;
+          const uint32_t ph = (kg / S) & 1;
+          if (!ptx::wait_bounded(&full[s], ph, abort_flag)) {
+            raise_status(p.status, abort_flag, kStatusTimeout);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = ptx::smem_u32(stage0 + s * C::kStageBytes);
+          const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = ptx::sdesc_sw128(a0 + kk * 32, 16, 1024);
+            const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
+            ptx::mma_bf16(d0, ad, ptx::sdesc_sw128(b0 + kk * 2048, kBoxBytes, 1024), idesc, acc);
+            if (M == Mode::kSwiGLU)
+              ptx::mma_bf16(d0 + 128, ad, ptx::sdesc_sw128(b0 + C::kBBytes + kk * 2048, kBoxBytes, 1024), idesc,
+                            acc);
+          }
+          ptx::mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        ptx::mma_commit(&tfull[b]);
+        ++it;
+      }
+      ptx::mma_commit(done);
+      if (!ptx::wait_bounded(done, 0, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      TileInfo ti;
+      if (!tile_at(p, tile, BN, ti)) continue;
+      const int b = it & 1;
+      const uint32_t use = (uint32_t)it >> 1;
+      if (!ptx::wait_bounded(&tfull[b], use & 1, abort_flag)) {
+        raise_status(p.status, abort_flag, kStatusTimeout);
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + b * 256;
+      const bool valid = row < ti.rows;
+      const int n0 = ti.nb * BN;
+      if (M == Mode::kSwiGLU) {
+        const int64_t hrow = (int64_t)ti.row0 + row + (ti.shared ? p.out_shared_row_offset : 0);
+        uint16_t* base = static_cast<uint16_t*>(ti.shared ? p.out_shared : p.out_routed);
+        uint4* out = reinterpret_cast<uint4*>(base + hrow * p.ld_out + n0);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t g[32], u[32];
+          ptx::tmem_ld32(tbase + c * 32, g);
+          ptx::tmem_ld32(tbase + 128 + c * 32, u);
+          ptx::tmem_ld_wait2(g, u);
+          if (c == BN / 32 - 1) {
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&tempty[b]);
+          }
+          if (valid) {
+            uint32_t hp[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+              const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+              const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+              hp[i] = ptx::pack_bf16x2(h0, h1);
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              out[c * 4 + v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
+          }
+        }
+      } else {
+        const int64_t orow = (int64_t)ti.row0 + row + (ti.shared ? p.out_shared_row_offset : 0);
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          ptx::tmem_ld32(tbase + c * 32, r);
+          ptx::tmem_ld_wait(r);
+          if (c == BN / 32 - 1) {
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&tempty[b]);
+          }
+          if (valid && n0 + c * 32 < (ti.shared ? p.N_shared : p.N_routed)) {
+            if (ti.shared) {
+              float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.out_shared) + orow * p.ld_out + n0 + c * 32);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                out[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            } else {
+              uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out_routed) + orow * p.ld_out + n0 + c * 32);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                out[v] = make_uint4(
+                    ptx::pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
+                    ptx::pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                    ptx::pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                    ptx::pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+            }
+          }
+        }
+      }
+      ++it;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <Mode M>
+cudaError_t launch(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtensorMap& b_r, const CUtensorMap& b_s,
+                   const CUtensorMap& c_r, const CUtensorMap& c_s, const GemmParams& p, int grid,
+                   cudaStream_t stream) {
+  const size_t smem = smem_bytes<M>();
+  cudaError_t err =
+      cudaFuncSetAttribute(grouped_gemm_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  if (grid <= 0) return cudaSuccess;
+  grouped_gemm_kernel<M><<<grid, 192, smem, stream>>>(a_r, a_s, b_r, b_s, c_r, c_s, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int gemm_block_n_swiglu() { return Cfg<Mode::kSwiGLU>::BN; }
+int gemm_block_n_down() { return Cfg<Mode::kDown>::BN; }
+
+cudaError_t launch_grouped_swiglu(const CUtensorMap& tmA_r, const CUtensorMap& tmA_s, const CUtensorMap& tmW1_r,
+                                  const CUtensorMap& tmW1_s, const CUtensorMap& tmW3_r, const CUtensorMap& tmW3_s,
+                                  const GemmParams& p, int grid, cudaStream_t stream) {
+  return launch<Mode::kSwiGLU>(tmA_r, tmA_s, tmW1_r, tmW1_s, tmW3_r, tmW3_s, p, grid, stream);
+}
+
+cudaError_t launch_grouped_down(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
+                                const GemmParams& p, int grid, cudaStream_t stream) {
+  return launch<Mode::kDown>(tmA, tmA, tmW2_r, tmW2_s, tmW2_r, tmW2_s, p, grid, stream);
+}
+
+}  // namespace moe

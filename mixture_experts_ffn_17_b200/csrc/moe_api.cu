@@ -1,0 +1,400 @@
+// moe_api.cu -- host side of the C ABI declared in include/moe.h: argument
+// validation, workspace layout, TMA tensor maps and the launch sequences.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "moe.h"
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status validate_shape(const moe_shape* s) {
+  if (!s) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->d <= 0 || s->E <= 0 || s->k <= 0 || s->inter <= 0 || s->shared_inter < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (s->k > s->E) return MOE_ERR_INVALID_ARG;
+  if (s->route != MOE_ROUTE_TOPK_SOFTMAX && s->route != MOE_ROUTE_SIGMOID_GROUP) return MOE_ERR_INVALID_ARG;
+  if (s->w_dtype != MOE_BF16 && s->w_dtype != MOE_E4M3) return MOE_ERR_INVALID_ARG;
+  if (s->y_dtype != MOE_F32 && s->y_dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (s->route == MOE_ROUTE_SIGMOID_GROUP) {
+    if (s->n_group <= 0 || s->E % s->n_group != 0) return MOE_ERR_INVALID_ARG;
+    const int gsize = s->E / s->n_group;
+    if (s->topk_group <= 0 || s->topk_group > s->n_group) return MOE_ERR_INVALID_ARG;
+    if (s->group_topn <= 0 || s->group_topn > gsize) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)s->topk_group * gsize < s->k) return MOE_ERR_INVALID_ARG;
+    if (s->n_group > 32 || gsize > 64) return MOE_ERR_UNSUPPORTED;
+  }
+  if (s->d % 128 != 0 || s->inter % 128 != 0 || s->shared_inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (s->E % 32 != 0 || s->E > 1024 || s->k > 32) return MOE_ERR_UNSUPPORTED;
+  if (s->T * (int64_t)s->k + s->T >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+  if (s->d > (1 << 20) || s->inter > (1 << 20) || s->shared_inter > (1 << 20)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+struct Layout {
+  size_t status, logits, idx, w, hist, base, counts, offsets, perm, row_of, tiles, ntiles, x_perm, H, Y_perm,
+      Y_shared, total;
+  int nb, max_mtiles, Hld;
+  int64_t Hrows;
+};
+
+Layout make_layout(const moe_shape& s) {
+  Layout L{};
+  const int64_t T = s.T, Tk = s.T * s.k;
+  const bool sh = s.shared_inter > 0;
+  L.nb = permute_blocks(T);
+  L.max_mtiles = (int)((Tk + kTileM - 1) / kTileM + s.E + (sh ? (T + kTileM - 1) / kTileM : 0));
+  L.Hld = std::max(s.inter, s.shared_inter);
+  L.Hrows = Tk + (sh ? T : 0);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off += align_up(std::max<size_t>(bytes, 1));
+    return at;
+  };
+  L.status = take(64);
+  L.logits = take((size_t)T * s.E * 4);
+  L.idx = take((size_t)Tk * 4);
+  L.w = take((size_t)Tk * 4);
+  L.hist = take((size_t)L.nb * s.E * 4);
+  L.base = take((size_t)L.nb * s.E * 4);
+  L.counts = take((size_t)s.E * 4);
+  L.offsets = take((size_t)(s.E + 1) * 4);
+  L.perm = take((size_t)Tk * 4);
+  L.row_of = take((size_t)Tk * 4);
+  L.tiles = take((size_t)L.max_mtiles * 16);
+  L.ntiles = take(4);
+  L.x_perm = take((size_t)Tk * s.d * 2);
+  L.H = take((size_t)L.Hrows * L.Hld * 2);
+  L.Y_perm = take((size_t)Tk * s.d * 2);
+  L.Y_shared = take(sh ? (size_t)T * s.d * 4 : 0);
+  L.total = off;
+  return L;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// bf16 row-major [outer, inner]; box [box_outer rows x box_inner elements];
+// 128-byte swizzle (box_inner * 2 must be 128 bytes).
+bool map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+            uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// bf16 row-major [outer, mid, inner]; box [1 x 64 x 64], 128-byte swizzle.
+bool map_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+#define MOE_CUDA(call)                          \
+  do {                                          \
+    if ((call) != cudaSuccess) return MOE_ERR_CUDA; \
+  } while (0)
+
+// ------------------------------------------------------------ stages
+moe_status run_router(const moe_shape& s, const void* x, const void* Wg, const float* bias, int32_t* idx, float* w,
+                      float* logits, uint32_t* status, cudaStream_t st) {
+  CUtensorMap tm_x, tm_wg;
+  const int eb = router_expert_block(s.E);
+  if (!map_2d(&tm_x, x, s.d, s.T, 64, 128) || !map_2d(&tm_wg, Wg, s.d, s.E, 64, eb)) return MOE_ERR_CUDA;
+  MOE_CUDA(launch_router_logits(tm_x, tm_wg, (int)s.T, s.d, s.E, logits, status, st));
+  RouteParams rp{s.route, s.n_group, s.topk_group, s.group_topn, s.route_scale};
+  MOE_CUDA(launch_router_topk(logits, s.route == MOE_ROUTE_SIGMOID_GROUP ? bias : nullptr, rp, (int)s.T, s.E, s.k,
+                              idx, w, st));
+  return MOE_OK;
+}
+
+moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void* x, const void* x_perm,
+                       const int32_t* offsets, const void* W1, const void* W3, const void* W2, const void* W1s,
+                       const void* W3s, const void* W2s, void* Y_perm, float* Y_shared, uint32_t* status,
+                       cudaStream_t st) {
+  const bool sh = s.shared_inter > 0;
+  const int64_t Tk = s.T * s.k;
+  int4* tiles = at<int4>(ws, L.tiles);
+  int32_t* ntiles = at<int32_t>(ws, L.ntiles);
+  uint16_t* H = at<uint16_t>(ws, L.H);
+  MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, sh, tiles, ntiles, st));
+
+  const int sms = num_sms();
+  // SwiGLU: A = gathered rows (routed) or x (shared); B = W1 | W3 column blocks
+  CUtensorMap a_r, a_s, w1_r, w1_s, w3_r, w3_s;
+  if (!map_2d(&a_r, x_perm, s.d, Tk, 64, kTileM) || !map_2d(&a_s, x, s.d, s.T, 64, kTileM) ||
+      !map_3d(&w1_r, W1, s.inter, s.d, s.E) || !map_3d(&w3_r, W3, s.inter, s.d, s.E))
+    return MOE_ERR_CUDA;
+  if (sh) {
+    if (!map_3d(&w1_s, W1s, s.shared_inter, s.d, 1) || !map_3d(&w3_s, W3s, s.shared_inter, s.d, 1))
+      return MOE_ERR_CUDA;
+  } else {
+    w1_s = w1_r;
+    w3_s = w3_r;
+  }
+  GemmParams p1{};
+  p1.tiles = tiles;
+  p1.ntiles = ntiles;
+  p1.max_mtiles = L.max_mtiles;
+  p1.E = s.E;
+  const int bn1 = gemm_block_n_swiglu();
+  p1.n_nb = (L.Hld + bn1 - 1) / bn1;
+  p1.K_routed = s.d;
+  p1.K_shared = s.d;
+  p1.N_routed = s.inter;
+  p1.N_shared = s.shared_inter;
+  p1.a_shared_row_offset = 0;
+  p1.out_routed = H;
+  p1.out_shared = H;
+  p1.out_shared_row_offset = Tk;
+  p1.ld_out = L.Hld;
+  p1.status = status;
+  const int grid1 = (int)std::min<int64_t>(sms, (int64_t)L.max_mtiles * p1.n_nb);
+  MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, p1, grid1, st));
+
+  // down projection: A = H (routed rows, then shared rows); B = W2 column blocks
+  CUtensorMap h_map, w2_r, w2_s;
+  if (!map_2d(&h_map, H, L.Hld, L.Hrows, 64, kTileM) || !map_3d(&w2_r, W2, s.d, s.inter, s.E)) return MOE_ERR_CUDA;
+  if (sh) {
+    if (!map_3d(&w2_s, W2s, s.d, s.shared_inter, 1)) return MOE_ERR_CUDA;
+  } else {
+    w2_s = w2_r;
+  }
+  GemmParams p2 = p1;
+  const int bn2 = gemm_block_n_down();
+  p2.n_nb = (s.d + bn2 - 1) / bn2;
+  p2.K_routed = s.inter;
+  p2.K_shared = s.shared_inter;
+  p2.N_routed = s.d;
+  p2.N_shared = s.d;
+  p2.a_shared_row_offset = (int)Tk;
+  p2.out_routed = Y_perm;
+  p2.out_shared = Y_shared;
+  p2.out_shared_row_offset = 0;
+  p2.ld_out = s.d;
+  const int grid2 = (int)std::min<int64_t>(sms, (int64_t)L.max_mtiles * p2.n_nb);
+  MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, p2, grid2, st));
+  return MOE_OK;
+}
+
+bool ws_ok(const void* ws, size_t ws_bytes, size_t need) {
+  return ws && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_shape* shape) {
+  if (validate_shape(shape) != MOE_OK) return 0;
+  return make_layout(*shape).total;
+}
+
+moe_status moe_router_topk(const moe_shape* shape, const void* x, const void* Wg, const float* bias,
+                           int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t ws_bytes,
+                           void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  if (!x || !Wg || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wg) || !aligned16(topk_idx) || !aligned16(topk_w) ||
+      (logits && !aligned16(logits)) || (bias && !aligned16(bias)))
+    return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(s);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  if (s.T == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
+  return run_router(s, x, Wg, bias, topk_idx, topk_w, logits ? logits : at<float>(ws, L.logits), status, st);
+}
+
+moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                       int32_t* perm_token, int32_t* row_of, const void* x, void* x_perm, void* ws,
+                       size_t ws_bytes, void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  if (!topk_idx || !counts || !offsets || !perm_token || !row_of) return MOE_ERR_INVALID_ARG;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(topk_idx) || !aligned16(counts) || !aligned16(offsets) || !aligned16(perm_token) ||
+      !aligned16(row_of) || (x && !aligned16(x)) || (x_perm && !aligned16(x_perm)))
+    return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(s);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
+  if (s.T == 0) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, (size_t)s.E * 4, st));
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, (size_t)(s.E + 1) * 4, st));
+    return MOE_OK;
+  }
+  MOE_CUDA(launch_permute(topk_idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
+                          perm_token, row_of, status, st));
+  if (x) MOE_CUDA(launch_gather_rows(x, perm_token, s.T * s.k, s.d, x_perm, num_sms(), st));
+  return MOE_OK;
+}
+
+moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const void* x_perm, const int32_t* offsets,
+                              const void* W1, const void* W3, const void* W2, const float* s1, const float* s3,
+                              const float* s2, const void* W1s, const void* W3s, const void* W2s, void* Y_perm,
+                              float* Y_shared, void* ws, size_t ws_bytes, void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  const bool sh = s.shared_inter > 0;
+  if (!x || !x_perm || !offsets || !W1 || !W3 || !W2 || !Y_perm) return MOE_ERR_INVALID_ARG;
+  if (sh && (!W1s || !W3s || !W2s || !Y_shared)) return MOE_ERR_INVALID_ARG;
+  if (s.w_dtype == MOE_E4M3 && (!s1 || !s3 || !s2)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (s.w_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  const Layout L = make_layout(s);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
+  if (s.T == 0) return MOE_OK;
+  return run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, W1s, W3s, W2s, Y_perm, sh ? Y_shared : nullptr,
+                     status, st);
+}
+
+moe_status moe_combine(const moe_shape* shape, const void* Y_perm, const float* Y_shared, const int32_t* row_of,
+                       const float* topk_w, void* y, void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  if (!Y_perm || !row_of || !topk_w || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(Y_perm) || !aligned16(row_of) || !aligned16(topk_w) || !aligned16(y) ||
+      (Y_shared && !aligned16(Y_shared)))
+    return MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, topk_w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16,
+                          static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_shape* shape, const void* x, const void* Wg, const float* bias, const void* W1,
+                       const void* W3, const void* W2, const float* s1, const float* s3, const float* s2,
+                       const void* W1s, const void* W3s, const void* W2s, void* y, int32_t* topk_idx_out,
+                       float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes, void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  const bool sh = s.shared_inter > 0;
+  if (!x || !Wg || !W1 || !W3 || !W2 || !y) return MOE_ERR_INVALID_ARG;
+  if (sh && (!W1s || !W3s || !W2s)) return MOE_ERR_INVALID_ARG;
+  if (s.w_dtype == MOE_E4M3 && (!s1 || !s3 || !s2)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out, counts_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (s.w_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  const Layout L = make_layout(s);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  if (s.T == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
+
+  int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+  float* w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
+  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  void* x_perm = at<void>(ws, L.x_perm);
+  void* Y_perm = at<void>(ws, L.Y_perm);
+  float* Y_shared = sh ? at<float>(ws, L.Y_shared) : nullptr;
+
+  moe_status r = run_router(s, x, Wg, bias, idx, w, at<float>(ws, L.logits), status, st);
+  if (r != MOE_OK) return r;
+  MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
+                          perm, row_of, status, st));
+  MOE_CUDA(launch_gather_rows(x, perm, s.T * s.k, s.d, x_perm, num_sms(), st));
+  r = run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, W1s, W3s, W2s, Y_perm, Y_shared, status, st);
+  if (r != MOE_OK) return r;
+  MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16, st));
+  return MOE_OK;
+}
+
+moe_status moe_check_device_status(const void* ws, void* stream, uint32_t* raw) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (raw) *raw = v;
+  if (v & kStatusTimeout) return MOE_ERR_DEVICE_TIMEOUT;
+  if (v & kStatusBounds) return MOE_ERR_DEVICE_BOUNDS;
+  return MOE_OK;
+}
+
+const char* moe_status_string(moe_status status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA call or kernel launch failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait timed out";
+    case MOE_ERR_DEVICE_BOUNDS: return "expert index out of range (skipped)";
+  }
+  return "unknown status";
+}
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// moe_internal.h -- host-side declarations shared by the library's .cu files.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+constexpr int kTileM = 128;  // rows per grouped-GEMM tile (tcgen05 M)
+
+// Device status bits OR-ed into the status word at the head of the workspace.
+enum : uint32_t {
+  kStatusTimeout = 1u,  // a bounded wait gave up
+  kStatusBounds = 2u,   // an index outside its range was seen and skipped
+};
+
+// A wait longer than this is a fault (a wait in a healthy launch lasts
+// microseconds).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+struct RouteParams {
+  int route;        // 0: top-k then softmax; 1: sigmoid group-limited
+  int n_group;
+  int topk_group;
+  int group_topn;
+  float route_scale;
+};
+
+// router.cu
+int router_expert_block(int E);
+cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E,
+                                 float* logits, uint32_t* status, cudaStream_t stream);
+cudaError_t launch_router_topk(const float* logits, const float* bias, const RouteParams& rp, int T, int E, int k,
+                               int32_t* idx, float* w, cudaStream_t stream);
+
+// permute.cu
+int permute_blocks(int64_t T);
+cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int32_t* hist, int32_t* base,
+                           int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* row_of,
+                           uint32_t* status, cudaStream_t stream);
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t rows, int d, void* x_perm,
+                               int num_sms, cudaStream_t stream);
+cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, bool with_shared, int4* tiles,
+                               int32_t* ntiles, cudaStream_t stream);
+
+// grouped_gemm.cu
+struct GemmParams {
+  const int4* tiles;
+  const int32_t* ntiles;
+  int max_mtiles;        // capacity of the tile list (clamps the device count)
+  int E;                 // group index E = shared expert
+  int n_nb;              // N blocks per tile row (max over routed / shared)
+  int K_routed, K_shared;
+  int N_routed, N_shared;
+  int a_shared_row_offset;  // row of the shared expert's first A row in its map
+  void* out_routed;      // bf16 rows
+  void* out_shared;      // SwiGLU: bf16 rows; down: fp32 rows
+  int64_t out_shared_row_offset;  // rows to skip in out_shared
+  int ld_out;            // output row stride (elements)
+  uint32_t* status;
+};
+
+int gemm_block_n_swiglu();
+int gemm_block_n_down();
+cudaError_t launch_grouped_swiglu(const CUtensorMap& tmA_r, const CUtensorMap& tmA_s, const CUtensorMap& tmW1_r,
+                                  const CUtensorMap& tmW1_s, const CUtensorMap& tmW3_r, const CUtensorMap& tmW3_s,
+                                  const GemmParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_grouped_down(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
+                                const GemmParams& p, int grid, cudaStream_t stream);
+
+// combine.cu
+cudaError_t launch_combine(const void* Y_perm, const float* Y_shared, const int32_t* row_of, const float* topk_w,
+                           int64_t T, int k, int d, void* y, bool y_bf16, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,263 @@
+// permute.cu -- token-to-expert dispatch without a host round trip.
+//
+// The atlas page's MoE forward ("DeepSeek-V3.2-Exp / Mixture of experts",
+// model.py 790-803 excerpt) counts assignments with bincount(indices,
+// minlength=E), copies the counts to the host and, for each expert, gathers
+// the tokens that chose it with torch.where(indices == e), i.e. in ascending
+// (token, slot) order.  Here the same order is built on the device as a stable
+// counting sort in three launches:
+//   1. hist    : per block of 256 tokens, a shared-memory histogram over E;
+//   2. scan    : one CTA; per expert the running sum over blocks (each block's
+//                base), counts[e], and the exclusive prefix sum offsets[E+1];
+//   3. scatter : each warp ranks its 32 tokens' k entries per expert with
+//                __match_any_sync, warps are ordered by a per-warp histogram,
+//                and entry (t, j) lands at offsets-based position r:
+//                perm_token[r] = t, row_of[t*k + j] = r.
+// A separate gather copies x rows into permuted order (x_perm), and the tile
+// builder lists the 128-row tiles of every expert segment (plus the shared
+// expert's tiles over all T tokens) for the grouped GEMMs.
+#include <algorithm>
+#include <cstdint>
+
+#include "common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kPermTokens = 256;  // tokens per block in hist / scatter
+constexpr int kPermThreads = 256;
+
+__global__ void __launch_bounds__(kPermThreads)
+    hist_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int32_t* __restrict__ hist,
+                uint32_t* __restrict__ status) {
+  extern __shared__ int32_t h[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+  __syncthreads();
+  const int64_t begin = (int64_t)blockIdx.x * kPermTokens * k;
+  const int64_t end = ::min((long long)T * k, (long long)(begin + (int64_t)kPermTokens * k));
+  for (int64_t i = begin + threadIdx.x; i < end; i += blockDim.x) {
+    const int e = idx[i];
+    if (e < 0 || e >= E) {
+      atomicOr(status, kStatusBounds);
+      continue;
+    }
+    atomicAdd(&h[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)blockIdx.x * E + e] = h[e];
+}
+
+// One CTA of >= E threads (a multiple of 32, <= 1024).
+__global__ void scan_kernel(const int32_t* __restrict__ hist, int nb, int E, int32_t* __restrict__ base,
+                            int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  __shared__ int32_t warp_sums[32];
+  const int e = threadIdx.x;
+  int32_t run = 0;
+  if (e < E)
+    for (int b = 0; b < nb; ++b) {
+      const int32_t v = hist[(size_t)b * E + e];
+      base[(size_t)b * E + e] = run;
+      run += v;
+    }
+  const int32_t c = (e < E) ? run : 0;
+  // block exclusive scan of c
+  const int lane = e & 31, warp = e >> 5;
+  int32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int32_t v = (lane < nw) ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane < nw) warp_sums[lane] = v - ((lane < nw) ? warp_sums[lane] : 0);  // exclusive per warp
+  }
+  __syncthreads();
+  const int32_t excl = warp_sums[warp] + incl - c;
+  if (e < E) {
+    counts[e] = c;
+    offsets[e] = excl;
+    if (e == E - 1) offsets[E] = excl + c;
+    for (int b = 0; b < nb; ++b) base[(size_t)b * E + e] += excl;
+  }
+}
+
+// Stable scatter.  Block = 8 warps x 32 tokens; a warp walks its tokens' k*32
+// entries in (token, slot) order, 32 entries per step.
+__global__ void __launch_bounds__(kPermThreads)
+    scatter_kernel(const int32_t* __restrict__ idx, int T, int k, int E, const int32_t* __restrict__ base,
+                   int32_t* __restrict__ perm_token, int32_t* __restrict__ row_of) {
+  extern __shared__ int32_t wh[];  // [8][E] per-warp counts, then exclusive per-warp bases
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = kPermThreads / 32;
+  for (int i = threadIdx.x; i < nwarps * E; i += blockDim.x) wh[i] = 0;
+  __syncthreads();
+
+  const int64_t tok0 = (int64_t)blockIdx.x * kPermTokens + warp * 32;
+  const int64_t ent0 = tok0 * k;
+  const int64_t ent_end = ::min((long long)T * k, (long long)(ent0 + 32LL * k));
+  int32_t* my = wh + warp * E;
+  // pass 1: per-warp counts (entries in order, so ranks within the warp are
+  // the running count before each entry)
+  for (int64_t i0 = ent0; i0 < ent_end; i0 += 32) {
+    const int64_t i = i0 + lane;
+    const bool valid = i < ent_end;
+    const int e = valid ? idx[i] : -1;
+    const bool inrange = valid && e >= 0 && e < E;
+    const uint32_t peers = __match_any_sync(0xffffffffu, inrange ? e : -1);
+    if (inrange) {
+      const int leader = __ffs(peers) - 1;
+      if (lane == leader) my[e] += __popc(peers);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  // exclusive scan over warps per expert
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      const int32_t v = wh[w * E + e];
+      wh[w * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // pass 2: positions
+  const int32_t* bb = base + (size_t)blockIdx.x * E;
+  for (int64_t i0 = ent0; i0 < ent_end; i0 += 32) {
+    const int64_t i = i0 + lane;
+    const bool valid = i < ent_end;
+    const int e = valid ? idx[i] : -1;
+    const bool inrange = valid && e >= 0 && e < E;
+    const uint32_t peers = __match_any_sync(0xffffffffu, inrange ? e : -1);
+    if (inrange) {
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int32_t r = bb[e] + my[e] + rank;
+      perm_token[r] = (int32_t)(i / k);
+      row_of[i] = r;
+    } else if (valid) {
+      row_of[i] = -1;
+    }
+    __syncwarp();
+    if (inrange) {
+      const int leader = __ffs(peers) - 1;
+      if (lane == leader) my[e] += __popc(peers);
+    }
+    __syncwarp();
+  }
+}
+
+// x_perm[r, :] = x[perm_token[r], :]; rows of d bf16 (d % 8 == 0), 16-byte
+// vectors, one CTA per row at a time.
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_token, int64_t rows,
+                       int vec_per_row, uint4* __restrict__ x_perm) {
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int32_t t = perm_token[r];
+    const uint4* src = x + (size_t)t * vec_per_row;
+    uint4* dst = x_perm + (size_t)r * vec_per_row;
+    for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) dst[v] = __ldg(src + v);
+  }
+}
+
+// Tile list for the grouped GEMMs: one int4 {group, row_start, rows, 0} per
+// 128-row tile of each expert segment (group e, rows in permuted order), then
+// the shared expert's tiles (group E, rows in token order).  ntiles[0] = count.
+__global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, int T, int with_shared,
+                                   int4* __restrict__ tiles, int32_t* __restrict__ ntiles) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t total;
+  const int e = threadIdx.x;
+  const int lane = e & 31, warp = e >> 5;
+  int32_t start = 0, cnt = 0, mt = 0;
+  if (e < E) {
+    start = offsets[e];
+    cnt = offsets[e + 1] - start;
+    mt = (cnt + kTileM - 1) / kTileM;
+  }
+  int32_t incl = mt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    const int32_t mine = (lane < nw) ? warp_sums[lane] : 0;
+    int32_t v = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane < nw) warp_sums[lane] = v - mine;
+    if (lane == nw - 1) total = v;
+  }
+  __syncthreads();
+  const int32_t first = warp_sums[warp] + incl - mt;
+  for (int m = 0; m < mt; ++m) {
+    const int32_t r0 = m * kTileM;
+    tiles[first + m] = make_int4(e, start + r0, min(kTileM, cnt - r0), 0);
+  }
+  const int32_t routed = total;
+  const int32_t shared_tiles = with_shared ? (T + kTileM - 1) / kTileM : 0;
+  for (int m = threadIdx.x; m < shared_tiles; m += blockDim.x) {
+    const int32_t r0 = m * kTileM;
+    tiles[routed + m] = make_int4(E, r0, min(kTileM, T - r0), 0);
+  }
+  if (threadIdx.x == 0) ntiles[0] = routed + shared_tiles;
+}
+
+}  // namespace
+
+int permute_blocks(int64_t T) { return (int)((T + kPermTokens - 1) / kPermTokens); }
+
+cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int32_t* hist, int32_t* base,
+                           int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* row_of,
+                           uint32_t* status, cudaStream_t stream) {
+  const int nb = permute_blocks(T);
+  hist_kernel<<<nb, kPermThreads, E * sizeof(int32_t), stream>>>(idx, (int)T, k, E, hist, status);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int st = ((E + 31) / 32) * 32;
+  scan_kernel<<<1, st, 0, stream>>>(hist, nb, E, base, counts, offsets);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const size_t sm = (size_t)(kPermThreads / 32) * E * sizeof(int32_t);
+  if (sm > 48 * 1024) {
+    err = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (err != cudaSuccess) return err;
+  }
+  scatter_kernel<<<nb, kPermThreads, sm, stream>>>(idx, (int)T, k, E, base, perm_token, row_of);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t rows, int d, void* x_perm,
+                               int num_sms, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  const int64_t g = std::min<int64_t>(rows, (int64_t)num_sms * 16);
+  gather_rows_kernel<<<(unsigned)g, 256, 0, stream>>>(static_cast<const uint4*>(x), perm_token, rows, d / 8,
+                                                      static_cast<uint4*>(x_perm));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, bool with_shared, int4* tiles,
+                               int32_t* ntiles, cudaStream_t stream) {
+  const int threads = ((E + 31) / 32) * 32;
+  build_tiles_kernel<<<1, threads < 32 ? 32 : threads, 0, stream>>>(offsets, E, (int)T, with_shared ? 1 : 0,
+                                                                    tiles, ntiles);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

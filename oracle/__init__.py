@@ -62,6 +62,7 @@ def lib():
             "oracle_weights_sigmoid": [i64, i32, i32, f64, P, P, P],
             "oracle_dispatch": [i64, i32, i32, P, P, P, P, P],
             "oracle_swiglu_rows": [i64, i64, i64, P, P, P, P, P],
+            "oracle_combine": [i64, i32, i64, P, P, P, P, P],
             "oracle_moe_forward": [i64, i64, i32, i32, i64, i64, i32, i32, i32, i32, f64,
                                    P, P, P, P, P, P, P, P, P, P, P, P, P, P],
         }
@@ -204,6 +205,19 @@ def swiglu_rows(x: np.ndarray, W1: np.ndarray, W3: np.ndarray, W2: np.ndarray) -
     out = np.empty((n, d), dtype=np.float64)
     lib().oracle_swiglu_rows(n, d, I, _p(x), _p(W1), _p(W3), _p(W2), _p(out))
     return out
+
+
+def combine(Yp: np.ndarray, Ys, row_of: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """y[t] = sum_j w[t,j] Yp[row_of[t,j]] + Ys[t] in fp64 (Ys may be None)."""
+    Yp = _c(Yp, np.float64)
+    Ys = None if Ys is None else _c(Ys, np.float64)
+    row_of = _c(row_of, np.int32)
+    w = _c(w, np.float64)
+    T, k = w.shape
+    d = Yp.shape[1]
+    y = np.empty((T, d), dtype=np.float64)
+    lib().oracle_combine(T, k, d, _p(Yp), _p(Ys), _p(row_of), _p(w), _p(y))
+    return y
 
 
 def moe_forward(x, Wg, W1, W3, W2, W1s=None, W3s=None, W2s=None, *, k: int, route: int = 0,

@@ -405,3 +405,26 @@ ORACLE_EXPORT int oracle_moe_forward(int64_t T, int64_t d, int E, int k, int64_t
     free(logits); free(idx); free(w);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Combine step alone: y[t] = sum_j w[t,j] * Yp[row_of[t*k+j]] + Ys[t]        */
+/* (the y[idx] += expert_out * weight accumulation of the atlas page's       */
+/* model.py 790-803 excerpt, then y += shared).  Ys may be NULL.  Rows with   */
+/* row_of < 0 are skipped.                                                    */
+/* ------------------------------------------------------------------------ */
+ORACLE_EXPORT void oracle_combine(int64_t T, int k, int64_t d, const double *Yp, const double *Ys,
+                                  const int32_t *row_of, const double *w, double *y)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double *yt = y + t * d;
+        for (int64_t c = 0; c < d; ++c) yt[c] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int32_t r = row_of[t * k + j];
+            if (r < 0) continue;
+            for (int64_t c = 0; c < d; ++c) yt[c] += w[t * k + j] * Yp[(int64_t)r * d + c];
+        }
+        if (Ys)
+            for (int64_t c = 0; c < d; ++c) yt[c] += Ys[t * d + c];
+    }
+}

@@ -1,0 +1,265 @@
+"""CUDA path vs the fp64 oracle at sizes the oracle finishes in seconds: every
+entry point of the C ABI, several tiles and ragged tails, and the degenerate
+cases of the layer (empty experts, one oversize expert, T=1, k=1, k=E, no
+shared expert, zero weights)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_ffn_17_b200 import binding as B
+from mixture_experts_ffn_17_b200 import build as libbuild
+from mixture_experts_ffn_17_b200 import workloads
+
+from gpu_util import oracle_full, route_with_exemptions, run_forward, to_device
+from parity import TOL_BF16, dec, max_rel_err, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    libbuild.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+
+
+def _tiny():
+    return to_device(workloads.make("tiny"))
+
+
+def _medium(**kw):
+    # several tiles per expert, ragged tails, inter != shared_inter
+    shape = dict(T=1000, d=1024, E=64, k=6, inter=512, shared_inter=384)
+    shape.update(kw)
+    return to_device(workloads.make_small("prefill", **shape))
+
+
+# --------------------------------------------------------------- router
+@pytest.mark.parametrize("make", [_tiny, _medium])
+def test_router_matches_oracle(make):
+    w = make()
+    cfg = w.cfg
+    shape = B.shape_of(cfg)
+    ws = B.alloc_workspace(shape)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    lg_dev = torch.empty(cfg.T, cfg.E, dtype=torch.float32, device="cuda")
+    B.router_topk(shape, w.x, w.Wg, w.bias, idx, tw, lg_dev, ws)
+    torch.cuda.synchronize()
+    lg = oracle.logits(dec(w.x), dec(w.Wg))
+    err = np.abs(to_np(lg_dev).astype(np.float64) - lg)
+    assert err.max() <= 1e-6 * (1 + np.abs(lg).max()), err.max()
+    idx_o, w_o, merged, report = route_with_exemptions(w, lg, to_np(idx))
+    assert len(report) <= max(1, cfg.T // 100)
+    ok = np.all(to_np(idx) == merged, axis=1)
+    assert np.allclose(to_np(tw)[ok], w_o[ok], rtol=0, atol=2e-6)
+
+
+def test_router_group_mode_matches_oracle():
+    w = to_device(workloads.make_small("fp8", T=700, d=512, E=64, k=6, inter=256, shared_inter=256, n_group=8,
+                                       topk_group=3, fp8=False))
+    cfg = w.cfg
+    shape = B.shape_of(cfg)
+    ws = B.alloc_workspace(shape)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    B.router_topk(shape, w.x, w.Wg, w.bias, idx, tw, None, ws)
+    torch.cuda.synchronize()
+    lg = oracle.logits(dec(w.x), dec(w.Wg))
+    idx_o, w_o, merged, report = route_with_exemptions(w, lg, to_np(idx))
+    ok = np.all(to_np(idx) == merged, axis=1)
+    assert np.allclose(to_np(tw)[ok], w_o[ok], rtol=0, atol=1e-5)
+    assert np.allclose(to_np(tw).sum(1), 2.5, atol=1e-5)
+
+
+# --------------------------------------------------------------- permute
+def _permute_case(idx_np, E, d=256, x=None):
+    T, k = idx_np.shape
+    shape = B.make_shape(T=T, d=d, E=E, k=k, inter=128, shared_inter=0)
+    ws = B.alloc_workspace(shape)
+    dev = lambda a: torch.as_tensor(a, device="cuda")
+    idx = dev(np.ascontiguousarray(idx_np, dtype=np.int32))
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    if x is None:
+        g = torch.Generator(device="cuda").manual_seed(5)
+        x = torch.randn(T, d, generator=g, device="cuda").to(torch.bfloat16)
+    x_perm = torch.empty(T * k, d, dtype=torch.bfloat16, device="cuda")
+    B.permute(shape, idx, counts, offsets, perm, row_of, x, x_perm, ws)
+    rc, raw = B.check_device_status(ws)
+    c, o, p, r = oracle.dispatch(idx_np, E)
+    assert np.array_equal(to_np(counts), c)
+    assert np.array_equal(to_np(offsets), o)
+    assert np.array_equal(to_np(perm), p)
+    assert np.array_equal(to_np(row_of), r)
+    assert torch.equal(x_perm, x[torch.as_tensor(p, device="cuda").long()])
+    assert rc == B.MOE_OK, raw
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 32, 1), (255, 32, 4), (257, 64, 8), (1000, 256, 8), (16384, 256, 8)])
+def test_permute_random_routing(T, E, k):
+    rng = np.random.default_rng(T + E + k)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    _permute_case(idx, E)
+
+
+def test_permute_one_expert_takes_everything():
+    T, E, k = 700, 64, 2
+    idx = np.zeros((T, k), dtype=np.int32)
+    idx[:, 0] = 13
+    idx[:, 1] = 40 + (np.arange(T) % 3)      # three busy experts, 60 empty ones
+    _permute_case(idx, E)
+
+
+def test_permute_duplicate_slots():
+    # caller-supplied indices may repeat an expert within a token; each entry
+    # still gets its own row, in (token, slot) order
+    rng = np.random.default_rng(9)
+    idx = rng.integers(0, 32, size=(300, 4)).astype(np.int32)
+    idx[:, 1] = idx[:, 0]
+    _permute_case(idx, 32)
+
+
+def test_permute_reports_out_of_range_index():
+    T, E, k = 64, 32, 2
+    shape = B.make_shape(T=T, d=256, E=E, k=k, inter=128, shared_inter=0)
+    ws = B.alloc_workspace(shape)
+    idx = torch.randint(0, E, (T, k), dtype=torch.int32, device="cuda")
+    idx[5, 1] = E + 3
+    idx[9, 0] = -1
+    out = [torch.empty(n, dtype=torch.int32, device="cuda") for n in (E, E + 1, T * k, T * k)]
+    B.permute(shape, idx, *out, None, None, ws)
+    rc, raw = B.check_device_status(ws)
+    assert rc == B.MOE_ERR_DEVICE_BOUNDS and raw & 2
+    row_of = to_np(out[3]).reshape(T, k)
+    assert row_of[5, 1] == -1 and row_of[9, 0] == -1
+    assert to_np(out[0]).sum() == T * k - 2
+
+
+# --------------------------------------------------------------- experts
+def _experts_case(w, idx_np):
+    cfg = w.cfg
+    T, k = idx_np.shape
+    shape = B.shape_of(cfg)
+    ws = B.alloc_workspace(shape)
+    c, o, p, r = oracle.dispatch(idx_np, cfg.E)
+    x_perm = w.x[torch.as_tensor(p, device="cuda").long()].contiguous()
+    offsets = torch.as_tensor(o, device="cuda")
+    Y_perm = torch.empty(T * k, cfg.d, dtype=torch.bfloat16, device="cuda")
+    Y_sh = torch.empty(T, cfg.d, dtype=torch.float32, device="cuda") if cfg.shared_inter else None
+    B.grouped_swiglu(shape, w.x, x_perm, offsets, w.W1, w.W3, w.W2, None, None, None, w.W1s, w.W3s, w.W2s, Y_perm,
+                     Y_sh, ws)
+    rc, raw = B.check_device_status(ws)
+    assert rc == B.MOE_OK, raw
+    x = dec(w.x)
+    W1, W3, W2 = dec(w.W1), dec(w.W3), dec(w.W2)
+    ref = np.zeros((T * k, cfg.d))
+    for e in range(cfg.E):
+        if c[e]:
+            ref[o[e]:o[e + 1]] = oracle.swiglu_rows(x[p[o[e]:o[e + 1]]], W1[e], W3[e], W2[e])
+    assert max_rel_err(dec(Y_perm), ref) <= TOL_BF16
+    if cfg.shared_inter:
+        ref_s = oracle.swiglu_rows(x, dec(w.W1s), dec(w.W3s), dec(w.W2s))
+        assert max_rel_err(to_np(Y_sh).astype(np.float64), ref_s) <= TOL_BF16
+
+
+def test_grouped_swiglu_tiny_routing():
+    w = _tiny()
+    lg = oracle.logits(dec(w.x), dec(w.Wg))
+    idx, _, _ = oracle.route_topk_softmax(lg, w.cfg.k)
+    _experts_case(w, idx)
+
+
+def test_grouped_swiglu_oversize_and_empty_segments():
+    w = _medium(T=600, k=2)
+    idx = np.zeros((600, 2), dtype=np.int32)
+    idx[:, 0] = 7                                  # 600 rows: 5 tiles, ragged last
+    idx[:, 1] = 20 + (np.arange(600) % 2)          # two 300-row segments
+    _experts_case(w, idx)
+
+
+def test_grouped_swiglu_no_shared_expert():
+    w = _medium(T=300, shared_inter=0)
+    lg = oracle.logits(dec(w.x), dec(w.Wg))
+    idx, _, _ = oracle.route_topk_softmax(lg, w.cfg.k)
+    _experts_case(w, idx)
+
+
+# --------------------------------------------------------------- combine
+@pytest.mark.parametrize("shared", [True, False])
+def test_combine_matches_oracle(shared):
+    T, k, d, E = 333, 5, 768, 32
+    rng = np.random.default_rng(11)
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    _, _, _, row_of = oracle.dispatch(idx, E)
+    g = torch.Generator().manual_seed(3)
+    Yp = torch.randn(T * k, d, generator=g).to(torch.bfloat16)
+    Ys = torch.randn(T, d, generator=g) if shared else None
+    wts = torch.rand(T, k, generator=g)
+    shape = B.make_shape(T=T, d=d, E=E, k=k, inter=128, shared_inter=128 if shared else 0)
+    y = torch.empty(T, d, dtype=torch.float32, device="cuda")
+    cu = lambda t: None if t is None else t.cuda()
+    B.combine(shape, cu(Yp), cu(Ys), cu(torch.as_tensor(row_of)), cu(wts), y)
+    torch.cuda.synchronize()
+    ref = oracle.combine(dec(Yp), None if Ys is None else dec(Ys), row_of.reshape(T, k), dec(wts))
+    assert max_rel_err(to_np(y).astype(np.float64), ref) <= 1e-5
+
+
+# --------------------------------------------------------------- whole layer
+def _check_forward(w, tol=TOL_BF16):
+    y, idx, tw, counts, ws = run_forward(w)
+    y_o, idx_o, w_o, lg = oracle_full(w)
+    _, _, merged, report = route_with_exemptions(w, lg, to_np(idx))
+    if report:
+        y_o, *_ = oracle_full(w, force_idx=merged)
+    c, _, _, _ = oracle.dispatch(merged, w.cfg.E)
+    assert np.array_equal(to_np(counts), c)
+    err = max_rel_err(to_np(y).astype(np.float64), y_o)
+    assert err <= tol, err
+    return y, err
+
+
+def test_forward_tiny():
+    _check_forward(_tiny())
+
+
+def test_forward_medium_ragged():
+    _check_forward(_medium())
+
+
+@pytest.mark.parametrize("kw", [dict(T=1), dict(T=129, k=1), dict(T=64, E=32, k=32), dict(T=200, shared_inter=0)])
+def test_forward_edge_shapes(kw):
+    shape = dict(T=100, d=512, E=32, k=4, inter=256, shared_inter=256)
+    shape.update(kw)
+    _check_forward(to_device(workloads.make_small("prefill", **shape)))
+
+
+def test_forward_zero_down_projection_is_shared_only():
+    w = _tiny()
+    w.W2.zero_()
+    y, _, _, _, _ = run_forward(w)
+    ref = oracle.swiglu_rows(dec(w.x), dec(w.W1s), dec(w.W3s), dec(w.W2s))
+    assert max_rel_err(to_np(y).astype(np.float64), ref) <= TOL_BF16
+
+
+def test_forward_zero_input_gives_zero():
+    w = _tiny()
+    w.x.zero_()
+    y, _, _, _, _ = run_forward(w)
+    assert torch.count_nonzero(y) == 0
+
+
+def test_forward_bf16_output_is_rounded_fp32_output():
+    w = _tiny()
+    y32, *_ = run_forward(w, B.MOE_F32)
+    y16, *_ = run_forward(w, B.MOE_BF16)
+    assert torch.equal(y16, y32.to(torch.bfloat16))
+
+
+def test_forward_is_deterministic():
+    w = _medium()
+    a, ia, *_ = run_forward(w)
+    b, ib, *_ = run_forward(w)
+    assert torch.equal(a, b) and torch.equal(ia, ib)

@@ -387,3 +387,21 @@ def test_forward_force_idx_roundtrip():
     y2, idx2, w2, _ = oracle.moe_forward(**p, k=3, force_idx=idx)
     assert np.array_equal(idx, idx2) and np.array_equal(y, y2)
     assert np.allclose(oracle.weights_for(lg, idx), w, rtol=1e-14)
+
+
+def test_combine_special_cases():
+    rng = np.random.default_rng(18)
+    T, k, d = 6, 3, 5
+    Yp = rng.standard_normal((T * k, d))
+    Ys = rng.standard_normal((T, d))
+    # identity placement, unit weight on slot 0 only: y = Yp[t*k] + Ys
+    row_of = np.arange(T * k, dtype=np.int32).reshape(T, k)
+    w = np.zeros((T, k)); w[:, 0] = 1.0
+    assert np.array_equal(oracle.combine(Yp, Ys, row_of, w), Yp[::k] + Ys)
+    # equal rows with weights summing to 1 reproduce the row; no shared part
+    Yp2 = np.repeat(rng.standard_normal((1, d)), T * k, axis=0)
+    w2 = np.full((T, k), 1.0 / 4); w2[:, 0] = 0.5
+    assert np.allclose(oracle.combine(Yp2, None, row_of, w2), Yp2[:T], rtol=1e-15, atol=1e-15)
+    # skipped rows (row_of < 0) contribute nothing
+    row_of3 = row_of.copy(); row_of3[:, 1:] = -1
+    assert np.array_equal(oracle.combine(Yp, None, row_of3, np.ones((T, k))), Yp[::k])
