@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of one DeepSeek-V3 MoE feed-forward layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, same metric
+
+A step is one full layer forward (router, dispatch, grouped SwiGLU experts,
+shared expert, combine) over one batch of synthetic tokens already resident in
+HBM.  Default workload: the prefill layer, T=4096 tokens, d=7168, 256 routed
+experts top-8 + 1 shared expert, inter 2048, bf16 weights and activations,
+fp32 accumulation, fp32 output.  The weights (22.6 GB) are far larger than the
+126 MB L2, so no flush is needed between steps.
+
+With N > 1 (torchrun, one process per GPU) every rank runs an independent
+replica of the layer on its own batch (the layer needs no exchange on one GPU's
+worth of experts); time is the max over ranks and value counts all ranks'
+tokens.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "MoE-layer tokens/s and TFLOPS at V3 shapes (T=4096 bf16); % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 10  # router logits, top-k, hist, scan, scatter, gather, tile list, up, down, combine
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--workload", default="prefill", choices=("prefill", "decode", "skewed", "fp8", "tiny"))
+    p.add_argument("--tokens", type=int, default=None, help="override T (profiling small cases)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample", type=int, default=16, help="tokens the CPU baseline runs through the oracle")
+    p.add_argument("--ref-sample", type=int, default=2, help="tokens per step of the reference arm")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ plumbing
+class Dist:
+    def __init__(self):
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+        if self.world > 1:
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.pg:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+             0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+             0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.ok = False
+        self.samples = []
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that instead of clocks
+            self.err = str(e)
+
+    def _reasons(self):
+        fn = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM),
+                                     self._reasons(), self.nv.nvmlDeviceGetUtilizationRates(self.h).gpu))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": f"NVML unavailable: {self.err}"}
+        busy = [s for s in self.samples if s[2] > 0] or self.samples
+        if not busy:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        bits = 0
+        for s in busy:
+            bits |= s[1]
+        reasons = [n for b, n in self.NAMES.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(s[0] for s in busy), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(busy)}
+
+
+# ------------------------------------------------------------------ workload
+def touched_experts(counts) -> int:
+    return int((counts > 0).sum())
+
+
+def layer_work(cfg, counts, y_bytes_per_el):
+    """Algorithmic FLOPs and bytes of one layer forward (what the method must
+    do: router + touched experts' weights read once + shared expert + Wg + x
+    read + y written)."""
+    wb = 1 if cfg.fp8 else 2
+    flops = cfg.T * cfg.flops_per_token()
+    n_touched = touched_experts(counts)
+    routed_w = n_touched * 3 * cfg.d * cfg.inter * wb
+    if cfg.fp8:
+        routed_w += n_touched * 3 * (cfg.d // 128) * (cfg.inter // 128) * 4
+    shared_w = 3 * cfg.d * cfg.shared_inter * 2
+    act = cfg.T * cfg.d * 2 + cfg.T * cfg.d * y_bytes_per_el
+    return flops, routed_w + shared_w + cfg.E * cfg.d * 2 + act, n_touched
+
+
+def kernel_work(cfg, counts, stage):
+    """Algorithmic FLOPs / bytes of one launch of an expert kernel: the
+    touched experts' weight slices plus the shared expert's, the activation
+    rows read once, and the rows written."""
+    wb = 1 if cfg.fp8 else 2
+    n_touched = touched_experts(counts)
+    rows = cfg.T * cfg.k
+    if stage == "experts_up":
+        w = (n_touched * 2 * cfg.d * cfg.inter) * wb + 2 * cfg.d * cfg.shared_inter * 2
+        flops = rows * 4 * cfg.d * cfg.inter + cfg.T * 4 * cfg.d * cfg.shared_inter
+        act = cfg.T * cfg.d * 2 + rows * cfg.inter * 2 + cfg.T * cfg.shared_inter * 2
+    else:  # experts_down
+        w = (n_touched * cfg.d * cfg.inter) * wb + cfg.d * cfg.shared_inter * 2
+        flops = rows * 2 * cfg.d * cfg.inter + cfg.T * 2 * cfg.d * cfg.shared_inter
+        act = rows * cfg.inter * 2 + cfg.T * cfg.shared_inter * 2 + rows * cfg.d * 2 + cfg.T * cfg.d * 4
+    return flops, w + act
+
+
+# ------------------------------------------------------------------ oracle timing
+def oracle_sample(w, tokens, fetch_cache=None):
+    """Run the fp64 oracle on a sample of tokens of a device-resident workload.
+    Returns (seconds of oracle work, outputs).  Copies device->host are not
+    timed; decoding stored values and all arithmetic are."""
+    import oracle
+    cfg = w.cfg
+    tok = torch.as_tensor(tokens, device=w.x.device)
+    x_host = w.x[tok].cpu()
+    wg_host = w.Wg.cpu()
+    shared_host = [t.cpu() for t in (w.W1s, w.W3s, w.W2s)]
+    bias = None if w.bias is None else w.bias.double().cpu().numpy()
+    t0 = time.perf_counter()
+    x = oracle.decode(x_host)
+    lg = oracle.logits(x, oracle.decode(wg_host))
+    if cfg.route == 0:
+        idx, wts, _ = oracle.route_topk_softmax(lg, cfg.k)
+    else:
+        idx, wts, _, _ = oracle.route_sigmoid_group(lg, bias, cfg.k, cfg.n_group, cfg.topk_group, cfg.group_topn,
+                                                   cfg.route_scale)
+    spent = time.perf_counter() - t0
+    y = np.zeros((len(tokens), cfg.d))
+    for e in np.unique(idx):
+        rows, slots = np.nonzero(idx == e)
+        if cfg.fp8:
+            host = [(w.W1[e].cpu(), w.s1[e].cpu()), (w.W3[e].cpu(), w.s3[e].cpu()), (w.W2[e].cpu(), w.s2[e].cpu())]
+            t0 = time.perf_counter()
+            W = [oracle.decode_e4m3_blocks(q.numpy(), s.numpy()) for q, s in host]
+        else:
+            host = [w.W1[e].cpu(), w.W3[e].cpu(), w.W2[e].cpu()]
+            t0 = time.perf_counter()
+            W = [oracle.decode(t) for t in host]
+        o = oracle.swiglu_rows(x[rows], *W)
+        y[rows] += wts[rows, slots][:, None] * o
+        spent += time.perf_counter() - t0
+    t0 = time.perf_counter()
+    y += oracle.swiglu_rows(x, *[oracle.decode(t) for t in shared_host])
+    spent += time.perf_counter() - t0
+    return spent, y
+
+
+def cpu_threads():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args, dist):
+    """The oracle as the reference arm: every step runs a bounded sample of
+    the workload's tokens through the fp64 CPU oracle on the host cores."""
+    from mixture_experts_ffn_17_b200 import workloads
+    if dist.rank != 0:
+        return
+    cfg = workloads.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = cfg.replace(T=args.tokens)
+    w = workloads.make(cfg, device="cuda")
+    S = args.ref_sample
+    times = []
+    for step in range(args.warmup + args.steps):
+        toks = [(step * S + i) % cfg.T for i in range(S)]
+        t, _ = oracle_sample(w, toks)
+        if step >= args.warmup:
+            times.append(t)
+    per_tok = sum(times) / (S * len(times))
+    value = 1.0 / per_tok
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(cfg, args),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+                             "sample": f"{S} tokens per step of the {cfg.name} workload through the whole layer "
+                                       f"(fp64 oracle, OpenMP over rows)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_of(cfg, args):
+    return {"workload": f"{cfg.name}: MoE FFN layer T={cfg.T} d={cfg.d} E={cfg.E} top-{cfg.k} inter={cfg.inter} "
+                        f"+ shared {cfg.shared_inter}, {'e4m3 experts' if cfg.fp8 else 'bf16'}",
+            "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "inter": cfg.inter, "shared_inter": cfg.shared_inter,
+            "routing": "top-k then softmax" if cfg.route == 0 else "sigmoid group-limited (8 groups, top-4)",
+            "seed": cfg.seed, "l2": "inputs larger than L2 (weights 22.6 GB vs 126 MB L2); no flush",
+            "parallelism": f"replicas x{args.gpus}"}
+
+
+def run_ours(args, dist):
+    from mixture_experts_ffn_17_b200 import binding as B
+    from mixture_experts_ffn_17_b200 import workloads
+
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    cfg = workloads.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = cfg.replace(T=args.tokens)
+    w = workloads.make(cfg, device=dev)
+    shape = B.shape_of(cfg, B.MOE_F32)
+    ws = B.alloc_workspace(shape, dev)
+    y = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device=dev)
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    fwd_args = (shape, w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s, y, ws)
+
+    for _ in range(args.warmup):
+        B.forward(*fwd_args, counts=counts)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"device status after warm-up (raw {raw})")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.NUM_STAGE_EVENTS)] for _ in range(K)]
+    for row in evs:
+        for e in row:
+            e.record(stream)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        start.record(stream)
+        for i in range(K):
+            B.forward_profiled(*fwd_args, evs[i], counts=counts)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier()
+    ms = start.elapsed_time(end) / K
+    ms_max = dist.max(ms)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"device status after the timed steps (raw {raw})")
+
+    stage_ms = {name: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K))
+                for j, name in enumerate(B.STAGES)}
+    counts_np = counts.cpu().numpy()
+    peaks, peak_src = load_peaks()
+    flops, nbytes, n_touched = layer_work(cfg, counts_np, 4)
+    tokens_per_s = dist.world * cfg.T / (ms_max / 1e3)
+    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    roof_ms = 1e3 * max(t_tc, t_hbm)
+
+    dom = max(("experts_up", "experts_down"), key=lambda s: stage_ms[s])
+    kf, kb = kernel_work(cfg, counts_np, dom)
+    k_ms = stage_ms[dom]
+    k_tc = kf / (peaks["bf16_tflops_sustained"] * 1e12)
+    k_hbm = kb / (peaks["hbm_gbs"] * 1e9)
+    if k_hbm >= k_tc:
+        roof = {"bound": "hbm", "achieved": kb / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": kf / (k_ms / 1e3) / 1e12, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = f"grouped_gemm_kernel<{'SwiGLU' if dom == 'experts_up' else 'Down'}> ({dom})"
+    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if roof['bound'] == 'hbm' else 'bf16_tflops_sustained'})"
+    roof["algorithmic_bytes_per_launch"] = kb
+    roof["algorithmic_flops_per_launch"] = kf
+    roof["ms_per_launch"] = k_ms
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, B, fwd_args, w, cfg, y, dev, stream, dist)
+
+    line = {"metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": dist.world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(cfg, args),
+            "tflops": dist.world * flops / (ms_max / 1e3) / 1e12,
+            "roofline_layer": {"roofline_ms": roof_ms, "tensor_ms": 1e3 * t_tc, "hbm_ms": 1e3 * t_hbm,
+                               "bound": "hbm" if t_hbm >= t_tc else "tensor", "frac": roof_ms / ms,
+                               "flops": flops, "bytes": nbytes, "touched_experts": n_touched,
+                               "peaks": f"{peak_src}: hbm {peaks['hbm_gbs']} GB/s, bf16 "
+                                        f"{peaks['bf16_tflops_sustained']} TF/s sustained"},
+            "roofline": roof, "stage_ms": stage_ms, "clocks": sampler.summary(),
+            "gpu_launches": KERNELS_PER_STEP * K}
+    if e2e:
+        line["e2e"] = e2e
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = run_cpu_baseline(args, w, cfg)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, B, fwd_args, w, cfg, y, dev, stream, dist):
+    """Same metric through the public call with host buffers: each step copies
+    its tokens from pinned host memory, runs the layer and reads y back."""
+    x_host = w.x.cpu().pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    x_dev = torch.empty_like(w.x)
+    a = list(fwd_args)
+    a[1] = x_dev
+    for _ in range(max(1, args.warmup)):
+        x_dev.copy_(x_host, non_blocking=True)
+        B.forward(*a)
+        y_host.copy_(y, non_blocking=True)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    K = args.steps
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(K):
+        x_dev.copy_(x_host, non_blocking=True)
+        B.forward(*a)
+        y_host.copy_(y, non_blocking=True)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    ms = dist.max(start.elapsed_time(end) / K)
+    return {"value": dist.world * cfg.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+            "d2h_bytes_per_step": y_host.numel() * y_host.element_size()}
+
+
+def run_cpu_baseline(args, w, cfg):
+    S = min(args.cpu_sample, cfg.T)
+    rng = np.random.default_rng(cfg.seed)
+    toks = np.sort(rng.choice(cfg.T, size=S, replace=False))
+    spent, _ = oracle_sample(w, toks)
+    return {"value": S / spent, "unit": "tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{S} random tokens of the {cfg.name} workload through the whole layer (fp64 oracle: "
+                      f"routing, every selected expert, shared expert; {spent:.1f} s)"}
+
+
+def main():
+    args = parse_args()
+    dist = Dist()
+    try:
+        if args.impl == "reference":
+            run_reference(args, dist)
+        else:
+            run_ours(args, dist)
+    finally:
+        dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -153,6 +153,21 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const void* Wg, co
                        const void* W1s, const void* W3s, const void* W2s, void* y, int32_t* topk_idx_out,
                        float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_forward plus per-stage timing: records the caller's CUDA events
+ * (cudaEvent_t handles, created with timing enabled) on `stream` at the stage
+ * boundaries, without synchronising:
+ *   [0] start  [1] after the router  [2] after dispatch (permutation, row
+ *   gather, tile list)  [3] after the grouped SwiGLU up-projection
+ *   [4] after the grouped down-projection  [5] after the combine.
+ * Same results and launches as moe_forward.  Profiling aid; the pages have no
+ * counterpart. */
+#define MOE_NUM_STAGE_EVENTS 6
+moe_status moe_forward_profiled(const moe_shape* shape, const void* x, const void* Wg, const float* bias,
+                                const void* W1, const void* W3, const void* W2, const float* s1, const float* s3,
+                                const float* s2, const void* W1s, const void* W3s, const void* W2s, void* y,
+                                int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, void* ws,
+                                size_t ws_bytes, void* stream, void* const* stage_events);
+
 /* Synchronises `stream`, reads the status word of `ws` written by the last
  * call that used this workspace and returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT or
  * MOE_ERR_DEVICE_BOUNDS (timeout wins when both are set); `raw` (optional)

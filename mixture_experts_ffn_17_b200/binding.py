@@ -22,7 +22,9 @@ MOE_BF16, MOE_E4M3, MOE_F32 = 0, 1, 2
 MOE_ROUTE_TOPK_SOFTMAX, MOE_ROUTE_SIGMOID_GROUP = 0, 1
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
-            "moe_forward", "moe_check_device_status", "moe_status_string", "moe_version")
+            "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version")
+NUM_STAGE_EVENTS = 6
+STAGES = ("router", "dispatch", "experts_up", "experts_down", "combine")
 
 
 class MoeError(RuntimeError):
@@ -68,9 +70,10 @@ def lib() -> ctypes.CDLL:
         L.moe_grouped_swiglu.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_combine.argtypes = [S, P, P, P, P, P, P]
         L.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P, P]
         L.moe_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         for fn in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward",
-                   "moe_check_device_status"):
+                   "moe_forward_profiled", "moe_check_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -145,6 +148,23 @@ def forward(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, ws, to
                              _ptr(s1), _ptr(s3), _ptr(s2), _ptr(W1s), _ptr(W3s), _ptr(W2s), _ptr(y), _ptr(topk_idx),
                              _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel() if ws is not None else 0,
                              _stream(stream)), "moe_forward")
+
+
+def forward_profiled(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, ws, events, topk_idx=None,
+                     topk_w=None, counts=None, stream=None):
+    """forward() that also records `events` (NUM_STAGE_EVENTS torch.cuda.Event
+    objects with timing enabled) at the stage boundaries."""
+    if len(events) != NUM_STAGE_EVENTS:
+        raise ValueError(f"need {NUM_STAGE_EVENTS} events")
+    for ev in events:
+        if not ev.cuda_event:  # torch creates the CUDA event on its first record
+            ev.record()
+    handles = (ctypes.c_void_p * NUM_STAGE_EVENTS)(*[ev.cuda_event for ev in events])
+    _check(lib().moe_forward_profiled(ctypes.byref(shape), _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3),
+                                      _ptr(W2), _ptr(s1), _ptr(s3), _ptr(s2), _ptr(W1s), _ptr(W3s), _ptr(W2s),
+                                      _ptr(y), _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(ws),
+                                      ws.numel() if ws is not None else 0, _stream(stream), handles),
+           "moe_forward_profiled")
 
 
 def check_device_status(ws, stream=None) -> tuple[int, int]:

@@ -159,13 +159,14 @@ moe_status run_router(const moe_shape& s, const void* x, const void* Wg, const f
 moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void* x, const void* x_perm,
                        const int32_t* offsets, const void* W1, const void* W3, const void* W2, const void* W1s,
                        const void* W3s, const void* W2s, void* Y_perm, float* Y_shared, uint32_t* status,
-                       cudaStream_t st) {
+                       cudaStream_t st, const cudaEvent_t* ev = nullptr) {
   const bool sh = s.shared_inter > 0;
   const int64_t Tk = s.T * s.k;
   int4* tiles = at<int4>(ws, L.tiles);
   int32_t* ntiles = at<int32_t>(ws, L.ntiles);
   uint16_t* H = at<uint16_t>(ws, L.H);
   MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, sh, tiles, ntiles, st));
+  if (ev) MOE_CUDA(cudaEventRecord(ev[0], st));
 
   const int sms = num_sms();
   // SwiGLU: A = gathered rows (routed) or x (shared); B = W1 | W3 column blocks
@@ -199,6 +200,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   p1.status = status;
   const int grid1 = (int)std::min<int64_t>(sms, (int64_t)L.max_mtiles * p1.n_nb);
   MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, p1, grid1, st));
+  if (ev) MOE_CUDA(cudaEventRecord(ev[1], st));
 
   // down projection: A = H (routed rows, then shared rows); B = W2 column blocks
   CUtensorMap h_map, w2_r, w2_s;
@@ -222,11 +224,60 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   p2.ld_out = s.d;
   const int grid2 = (int)std::min<int64_t>(sms, (int64_t)L.max_mtiles * p2.n_nb);
   MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, p2, grid2, st));
+  if (ev) MOE_CUDA(cudaEventRecord(ev[2], st));
   return MOE_OK;
 }
 
 bool ws_ok(const void* ws, size_t ws_bytes, size_t need) {
   return ws && ws_bytes >= need && (reinterpret_cast<uintptr_t>(ws) % kAlign) == 0;
+}
+
+moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, const float* bias, const void* W1,
+                        const void* W3, const void* W2, const float* s1, const float* s3, const float* s2,
+                        const void* W1s, const void* W3s, const void* W2s, void* y, int32_t* topk_idx_out,
+                        float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes, void* stream,
+                        const cudaEvent_t* ev) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  const bool sh = s.shared_inter > 0;
+  if (!x || !Wg || !W1 || !W3 || !W2 || !y) return MOE_ERR_INVALID_ARG;
+  if (sh && (!W1s || !W3s || !W2s)) return MOE_ERR_INVALID_ARG;
+  if (s.w_dtype == MOE_E4M3 && (!s1 || !s3 || !s2)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out, counts_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (s.w_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
+  const Layout L = make_layout(s);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  if (s.T == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
+  if (ev) MOE_CUDA(cudaEventRecord(ev[0], st));
+
+  int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
+  float* w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
+  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  void* x_perm = at<void>(ws, L.x_perm);
+  void* Y_perm = at<void>(ws, L.Y_perm);
+  float* Y_shared = sh ? at<float>(ws, L.Y_shared) : nullptr;
+
+  moe_status r = run_router(s, x, Wg, bias, idx, w, at<float>(ws, L.logits), status, st);
+  if (r != MOE_OK) return r;
+  if (ev) MOE_CUDA(cudaEventRecord(ev[1], st));
+  MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
+                          perm, row_of, status, st));
+  MOE_CUDA(launch_gather_rows(x, perm, s.T * s.k, s.d, x_perm, num_sms(), st));
+  r = run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, W1s, W3s, W2s, Y_perm, Y_shared, status, st,
+                  ev ? ev + 2 : nullptr);
+  if (r != MOE_OK) return r;
+  MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16, st));
+  if (ev) MOE_CUDA(cudaEventRecord(ev[5], st));
+  return MOE_OK;
 }
 
 }  // namespace
@@ -331,43 +382,20 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const void* Wg, co
                        const void* W3, const void* W2, const float* s1, const float* s3, const float* s2,
                        const void* W1s, const void* W3s, const void* W2s, void* y, int32_t* topk_idx_out,
                        float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes, void* stream) {
-  moe_status v = validate_shape(shape);
-  if (v != MOE_OK) return v;
-  const moe_shape& s = *shape;
-  const bool sh = s.shared_inter > 0;
-  if (!x || !Wg || !W1 || !W3 || !W2 || !y) return MOE_ERR_INVALID_ARG;
-  if (sh && (!W1s || !W3s || !W2s)) return MOE_ERR_INVALID_ARG;
-  if (s.w_dtype == MOE_E4M3 && (!s1 || !s3 || !s2)) return MOE_ERR_INVALID_ARG;
-  const void* ptrs[] = {x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out, counts_out};
-  for (const void* p : ptrs)
-    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (s.w_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
-  const Layout L = make_layout(s);
-  if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
-  if (s.T == 0) return MOE_OK;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint32_t* status = at<uint32_t>(ws, L.status);
-  MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
+  return forward_impl(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out,
+                      counts_out, ws, ws_bytes, stream, nullptr);
+}
 
-  int32_t* idx = topk_idx_out ? topk_idx_out : at<int32_t>(ws, L.idx);
-  float* w = topk_w_out ? topk_w_out : at<float>(ws, L.w);
-  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
-  int32_t* offsets = at<int32_t>(ws, L.offsets);
-  int32_t* perm = at<int32_t>(ws, L.perm);
-  int32_t* row_of = at<int32_t>(ws, L.row_of);
-  void* x_perm = at<void>(ws, L.x_perm);
-  void* Y_perm = at<void>(ws, L.Y_perm);
-  float* Y_shared = sh ? at<float>(ws, L.Y_shared) : nullptr;
-
-  moe_status r = run_router(s, x, Wg, bias, idx, w, at<float>(ws, L.logits), status, st);
-  if (r != MOE_OK) return r;
-  MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
-                          perm, row_of, status, st));
-  MOE_CUDA(launch_gather_rows(x, perm, s.T * s.k, s.d, x_perm, num_sms(), st));
-  r = run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, W1s, W3s, W2s, Y_perm, Y_shared, status, st);
-  if (r != MOE_OK) return r;
-  MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16, st));
-  return MOE_OK;
+moe_status moe_forward_profiled(const moe_shape* shape, const void* x, const void* Wg, const float* bias,
+                                const void* W1, const void* W3, const void* W2, const float* s1, const float* s3,
+                                const float* s2, const void* W1s, const void* W3s, const void* W2s, void* y,
+                                int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, void* ws,
+                                size_t ws_bytes, void* stream, void* const* stage_events) {
+  if (!stage_events) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < MOE_NUM_STAGE_EVENTS; ++i)
+    if (!stage_events[i]) return MOE_ERR_INVALID_ARG;
+  return forward_impl(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out,
+                      counts_out, ws, ws_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events));
 }
 
 moe_status moe_check_device_status(const void* ws, void* stream, uint32_t* raw) {

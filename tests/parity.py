@@ -71,3 +71,12 @@ def compare_indices(idx_dev: np.ndarray, idx_ora: np.ndarray, scores: np.ndarray
 def max_rel_err(y_dev: np.ndarray, y_ora: np.ndarray) -> float:
     rms = float(np.sqrt(np.mean(y_ora ** 2)))
     return float(np.max(np.abs(y_dev - y_ora))) / rms
+
+
+def bf16_stored_ok(y_dev: np.ndarray, y_ora: np.ndarray, tol: float = 1e-2) -> bool:
+    """Check for an intermediate the device stores in bf16: per element,
+    |y_dev - y_ora| <= 2^-8 |y_ora| (the rounding of the store itself, half an
+    ulp of an 8-significant-bit format) + tol * rms(y_ora) (everything else)."""
+    rms = float(np.sqrt(np.mean(y_ora ** 2)))
+    bound = 2.0 ** -8 * np.abs(y_ora) + tol * rms
+    return bool(np.all(np.abs(y_dev - y_ora) <= bound))
