@@ -46,6 +46,7 @@ def parse_args():
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--workload", default="prefill", choices=("prefill", "decode", "skewed", "fp8", "tiny"))
     p.add_argument("--tokens", type=int, default=None, help="override T (profiling small cases)")
+    p.add_argument("--experts", type=int, default=None, help="override E (profiling small cases)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-sample", type=int, default=16, help="tokens the CPU baseline runs through the oracle")
     p.add_argument("--ref-sample", type=int, default=2, help="tokens per step of the reference arm")
@@ -251,6 +252,8 @@ def run_reference(args, dist):
     cfg = workloads.CONFIGS[args.workload]
     if args.tokens:
         cfg = cfg.replace(T=args.tokens)
+    if args.experts:
+        cfg = cfg.replace(E=args.experts)
     w = workloads.make(cfg, device="cuda")
     S = args.ref_sample
     times = []
@@ -290,6 +293,8 @@ def run_ours(args, dist):
     cfg = workloads.CONFIGS[args.workload]
     if args.tokens:
         cfg = cfg.replace(T=args.tokens)
+    if args.experts:
+        cfg = cfg.replace(E=args.experts)
     w = workloads.make(cfg, device=dev)
     shape = B.shape_of(cfg, B.MOE_F32)
     ws = B.alloc_workspace(shape, dev)
