@@ -119,6 +119,27 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t*
                        int32_t* perm_token, int32_t* row_of, const void* x, void* x_perm, void* ws,
                        size_t ws_bytes, void* stream);
 
+/* moe_permute for callers that cannot allocate device memory -- for example a
+ * plugin inside another runtime that is handed only its input and output
+ * buffers.  Same arguments and results as moe_permute, minus the workspace:
+ * the scratch (per-block histograms and bases, a status word) lives in a
+ * 512 KiB array inside the library that every GPU loading the library holds
+ * until the process exits.  No counterpart on the pages; it exists only for
+ * such callers.
+ *  - Limit: ceil(T / 256) * E <= 65472 (e.g. T <= 65280 with E = 256);
+ *    larger shapes return MOE_ERR_UNSUPPORTED and launch nothing.
+ *  - The first call on a device looks up the array's device address (once per
+ *    device, with that device current); make that first call before any
+ *    stream capture.
+ *  - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
+ *  - All calls share the one array and it keeps the last call's contents:
+ *    calls that overlap on the GPU (other streams, other threads) race;
+ *    serialise them.
+ *  - Out-of-range indices are skipped (row_of = -1); there is no workspace,
+ *    so no status word is reported to the caller. */
+moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
+                               int32_t* perm_token, int32_t* row_of, const void* x, void* x_perm, void* stream);
+
 /* Grouped SwiGLU experts over the permuted rows plus the shared expert:
  *   for each expert e and each permuted row r in [offsets[e], offsets[e+1]):
  *     Y_perm[r] = bf16( (bf16(silu(x_perm[r] W1[e]) * (x_perm[r] W3[e]))) W2[e] )

@@ -22,7 +22,8 @@ MOE_BF16, MOE_E4M3, MOE_F32 = 0, 1, 2
 MOE_ROUTE_TOPK_SOFTMAX, MOE_ROUTE_SIGMOID_GROUP = 0, 1
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
-            "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version")
+            "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version",
+            "moe_permute_noalloc")
 NUM_STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "experts_up", "experts_down", "combine")
 
@@ -67,6 +68,8 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_size.restype = sz
         L.moe_router_topk.argtypes = [S, P, P, P, P, P, P, P, sz, P]
         L.moe_permute.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_permute_noalloc.argtypes = [S, P, P, P, P, P, P, P, P]
+        L.moe_permute_noalloc.restype = ctypes.c_int
         L.moe_grouped_swiglu.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_combine.argtypes = [S, P, P, P, P, P, P]
         L.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]

@@ -426,3 +426,83 @@ const char* moe_status_string(moe_status status) {
 const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free dispatch (moe_permute_noalloc).
+//
+// Some callers cannot allocate device memory at all: a plugin running inside
+// another runtime that hands it only its input and output buffers, or an
+// embedding whose allocator is owned elsewhere.  For them the dispatch step
+// keeps its scratch (the per-block histograms and bases, and a status word) in
+// this file-scope device array instead of a caller workspace.  Every GPU that
+// loads the library holds the array (512 KiB) until the process exits.
+//
+// In host code `g_noalloc_scratch` names a host-side stand-in, not a device
+// address, so its device address is fetched once per device with
+// cudaGetSymbolAddress (with that device current) and passed to the kernels.
+// ---------------------------------------------------------------------------
+namespace moe {
+namespace {
+
+constexpr int64_t kNoallocScratchInts = 1 << 17;  // 512 KiB of int32
+constexpr int64_t kNoallocStatusInts = 64;        // status word, padded to 256 bytes
+constexpr int kNoallocMaxDevices = 64;
+
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocScratchInts];
+
+std::mutex g_noalloc_mu;
+int32_t* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Device address of the static scratch on the current device (set up on the
+// first call per device).
+moe_status noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kNoallocMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MOE_OK;
+}
+
+int64_t round64(int64_t v) { return (v + 63) / 64 * 64; }
+
+}  // namespace
+}  // namespace moe
+
+extern "C" moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts,
+                                          int32_t* offsets, int32_t* perm_token, int32_t* row_of, const void* x,
+                                          void* x_perm, void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  if (!topk_idx || !counts || !offsets || !perm_token || !row_of) return MOE_ERR_INVALID_ARG;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(topk_idx) || !aligned16(counts) || !aligned16(offsets) || !aligned16(perm_token) ||
+      !aligned16(row_of) || (x && !aligned16(x)) || (x_perm && !aligned16(x_perm)))
+    return MOE_ERR_INVALID_ARG;
+  const int64_t per = round64((int64_t)permute_blocks(s.T) * s.E);  // histogram (and base) entries
+  if (kNoallocStatusInts + 2 * per > kNoallocScratchInts) return MOE_ERR_UNSUPPORTED;
+  int32_t* scratch = nullptr;
+  moe_status r = noalloc_scratch(&scratch);
+  if (r != MOE_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = reinterpret_cast<uint32_t*>(scratch);
+  // the array keeps the previous call's contents: the status word must start
+  // at zero; the histograms and bases are fully rewritten by the kernels
+  MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
+  if (s.T == 0) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, (size_t)s.E * 4, st));
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, (size_t)(s.E + 1) * 4, st));
+    return MOE_OK;
+  }
+  int32_t* hist = scratch + kNoallocStatusInts;
+  int32_t* base = hist + per;
+  MOE_CUDA(launch_permute(topk_idx, s.T, s.k, s.E, hist, base, counts, offsets, perm_token, row_of, status, st));
+  if (x) MOE_CUDA(launch_gather_rows(x, perm_token, s.T * s.k, s.d, x_perm, num_sms(), st));
+  return MOE_OK;
+}
