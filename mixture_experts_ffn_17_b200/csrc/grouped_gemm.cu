@@ -6,15 +6,22 @@
 // activation dtype before W2 (model.py 643 excerpt); here h is stored bf16.
 //
 // Both kernels are persistent (one CTA per SM) and walk a device-side tile
-// list: one entry per 128-row slice of an expert's segment of permuted rows,
+// list: one entry per 256-row slice of an expert's segment of permuted rows,
 // plus the shared expert (group E) over all T tokens.  Tile t -> (row tile
-// t / n_nb, column block t % n_nb).  Warp roles:
-//   warp 0    TMA producer: A tile [128 rows x 64 K] (K-major, 128B swizzle)
-//             and B tiles [64 K x 64 N] boxes (N-major, the weights' natural
-//             [K, N] row-major layout) into a 4-stage ring;
+// t / n_nb, column block t % n_nb).  A tile is one or two 128-row halves that
+// share every weight stage loaded into shared memory, so each weight byte
+// crosses HBM once for up to 256 rows (an expert's segment at V3 prefill
+// shapes is about 128 +- 11 rows); a half with no rows is never computed.
+// Warp roles:
+//   warp 0    TMA producer: A halves [128 rows x 64 K] (K-major, 128B
+//             swizzle) and B tiles as [64 K x 64 N] boxes (N-major, 128B
+//             swizzle: the weights' natural [K, N] row-major layout) into a
+//             3-stage ring (the K depth and stage count are build-time knobs,
+//             MOE_GEMM_BK / MOE_GEMM_STAGES; 64 x 3 measured fastest);
 //   warp 1    single-thread tcgen05.mma issuer, M=128, K=16 per instruction,
-//             fp32 accumulators in TMEM, two accumulator buffers so the
-//             epilogue of one tile overlaps the main loop of the next;
+//             fp32 accumulators in TMEM: two 256-column slots handed out
+//             round-robin (a one-half tile takes one, a two-half tile both),
+//             so one-half tiles overlap their epilogue with the next main loop;
 //   warps 2-5 epilogue: tcgen05.ld the accumulator rows (one row per
 //             thread), apply silu(g)*u (SwiGLU kernel) and store.
 //
@@ -33,11 +40,19 @@ namespace moe {
 
 namespace {
 
-constexpr int kBK = 64;
-constexpr int kStages = 4;
-constexpr uint32_t kABytes = kTileM * kBK * 2;  // 16 KB
-constexpr uint32_t kBoxBytes = 64 * kBK * 2;    // one [64 K x 64 N] bf16 box, 8 KB
-constexpr uint32_t kTmemCols = 512;             // 2 accumulator buffers x 256 columns
+constexpr int kBK = kGemmBK;
+constexpr int kStages = kGemmStages;
+constexpr uint32_t kABytes = kTileM * kBK * 2;  // one 128-row half of the A tile
+constexpr uint32_t kBoxBytes = 64 * kBK * 2;    // one [kBK K x 64 N] bf16 box
+constexpr uint32_t kBBytes = 4 * kBoxBytes;     // B part of a stage
+constexpr uint32_t kStageBytes = 2 * kABytes + kBBytes;
+// A halves: K-major rows of kBK bf16 (64 or 128 bytes), swizzled to match
+// the tensor map; 8-row groups kBK*16 bytes apart.
+constexpr uint32_t kASwizzle = kBK == 64 ? ptx::kSwizzle128B : ptx::kSwizzle64B;
+constexpr uint32_t kASBO = 8 * kBK * 2;
+static_assert(kStages * kStageBytes + 1024 + 256 <= 232448, "shared memory budget");
+constexpr uint32_t kTmemCols = 512;             // two 256-column accumulator slots
+constexpr uint32_t kSlotCols = 256;
 
 enum class Mode { kSwiGLU, kDown };
 
@@ -45,24 +60,17 @@ template <Mode M>
 struct Cfg;
 template <>
 struct Cfg<Mode::kSwiGLU> {
-  static constexpr int BN = 128;                    // per weight matrix
-  static constexpr uint32_t kBBytes = 2 * kBoxBytes;  // W1 part (W3 part follows)
-  static constexpr uint32_t kStageBytes = kABytes + 2 * kBBytes;
+  static constexpr int BN = 128;  // columns of W1 (and the same columns of W3) per tile
 };
 template <>
 struct Cfg<Mode::kDown> {
-  static constexpr int BN = 256;
-  static constexpr uint32_t kBBytes = 4 * kBoxBytes;
-  static constexpr uint32_t kStageBytes = kABytes + kBBytes;
+  static constexpr int BN = 256;  // columns of W2 per tile
 };
 
-template <Mode M>
-constexpr size_t smem_bytes() {
-  return 1024 + kStages * Cfg<M>::kStageBytes + 256;
-}
+constexpr size_t smem_bytes() { return 1024 + kStages * kStageBytes + 256; }
 
 struct TileInfo {
-  int group, row0, rows, nb;
+  int group, row0, rows, nb, halves;
   bool shared;
 };
 
@@ -73,10 +81,23 @@ __device__ __forceinline__ bool tile_at(const GemmParams& p, int tile, int BN, T
   ti.group = e.x;
   ti.row0 = e.y;
   ti.rows = e.z;
+  ti.halves = e.z > kTileM ? 2 : 1;
   ti.shared = (e.x == p.E);
   const int N = ti.shared ? p.N_shared : p.N_routed;
   return ti.nb * BN < N;  // false: this column block does not exist for the group
 }
+
+// Accumulator slots are handed out round-robin: a one-half tile takes the next
+// slot, a two-half tile takes both.  MMA issuer and epilogue walk the same
+// tile sequence, so they derive the same slot sequence.
+struct SlotRing {
+  int next = 0;
+  uint32_t u0 = 0u, u1 = 0u;  // completed uses of slot 0 / slot 1
+  __device__ __forceinline__ uint32_t use(int sl) const { return sl ? u1 : u0; }
+  __device__ __forceinline__ void bump(int sl) {
+    if (sl) ++u1; else ++u0;
+  }
+};
 
 template <Mode M>
 __global__ void __launch_bounds__(192, 1)
@@ -84,12 +105,11 @@ __global__ void __launch_bounds__(192, 1)
                         const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
                         const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s,
                         const GemmParams p) {
-  using C = Cfg<M>;
   constexpr int S = kStages;
-  constexpr int BN = C::BN;
+  constexpr int BN = Cfg<M>::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stage0 = align_1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(stage0 + S * C::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage0 + S * kStageBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
@@ -138,7 +158,7 @@ __global__ void __launch_bounds__(192, 1)
         ptx::prefetch_tmap(&tmC_s);
       }
       const uint64_t pol_a = ptx::policy_evict_last();   // A rows are reused by every column block
-      const uint64_t pol_w = ptx::policy_evict_first();  // weights stream through once
+      const uint64_t pol_w = ptx::policy_evict_first();  // each weight tile is read once
       int kg = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
@@ -151,6 +171,7 @@ __global__ void __launch_bounds__(192, 1)
         const int e3 = ti.shared ? 0 : ti.group;
         const int nk = (ti.shared ? p.K_shared : p.K_routed) / kBK;
         const int n0 = ti.nb * BN;
+        const uint32_t bytes = ti.halves * kABytes + kBBytes;
         for (int kb = 0; kb < nk; ++kb, ++kg) {
           const int s = kg % S;
           const uint32_t ph = (kg / S) & 1;
@@ -159,18 +180,21 @@ __global__ void __launch_bounds__(192, 1)
             ok = false;
             break;
           }
-          uint8_t* st = stage0 + s * C::kStageBytes;
-          ptx::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          uint8_t* st = stage0 + s * kStageBytes;
+          ptx::mbar_arrive_expect_tx(&full[s], bytes);
           ptx::tma_load_2d(st, mA, &full[s], kb * kBK, arow, pol_a);
-          uint8_t* sb = st + kABytes;
-#pragma unroll
-          for (int h = 0; h < BN / 64; ++h)
-            ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
+          if (ti.halves == 2) ptx::tma_load_2d(st + kABytes, mA, &full[s], kb * kBK, arow + kTileM, pol_a);
+          uint8_t* sb = st + 2 * kABytes;
           if (M == Mode::kSwiGLU) {
-            uint8_t* sc = sb + C::kBBytes;
 #pragma unroll
-            for (int h = 0; h < BN / 64; ++h)
-              ptx::tma_load_3d(sc + h * kBoxBytes, mC, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
+            for (int h = 0; h < 2; ++h) {
+              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
+              ptx::tma_load_3d(sb + (2 + h) * kBoxBytes, mC, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
           }
         }
       }
@@ -180,21 +204,24 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = ptx::idesc_bf16(kTileM, BN, false, true);
-      int kg = 0, it = 0;
+      // SwiGLU: two N=128 MMAs (W1 -> g, W3 -> u) per half; down: one N=256
+      constexpr uint32_t idesc = ptx::idesc_bf16(kTileM, M == Mode::kSwiGLU ? 128 : 256, false, true);
+      int kg = 0;
+      SlotRing ring;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
         if (!tile_at(p, tile, BN, ti)) continue;
         const int nk = (ti.shared ? p.K_shared : p.K_routed) / kBK;
-        const int b = it & 1;
-        const uint32_t use = (uint32_t)it >> 1;
-        if (!ptx::wait_bounded(&tempty[b], (use & 1) ^ 1, abort_flag)) {
-          raise_status(p.status, abort_flag, kStatusTimeout);
-          break;
+        for (int h = 0; h < ti.halves; ++h) {
+          const int sl = (ring.next + h) & 1;
+          if (!ptx::wait_bounded(&tempty[sl], (ring.use(sl) & 1) ^ 1, abort_flag)) {
+            raise_status(p.status, abort_flag, kStatusTimeout);
+            ok = false;
+          }
         }
+        if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t d0 = tmem + b * 256;
         for (int kb = 0; kb < nk; ++kb, ++kg) {
           const int s = kg % S;
           const uint32_t ph = (kg / S) & 1;
@@ -204,22 +231,29 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t a0 = ptx::smem_u32(stage0 + s * C::kStageBytes);
-          const uint32_t b0 = a0 + kABytes;
+          const uint32_t a0 = ptx::smem_u32(stage0 + s * kStageBytes);
+          const uint32_t b0 = a0 + 2 * kABytes;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = ptx::sdesc_sw128(a0 + kk * 32, 16, 1024);
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-            ptx::mma_bf16(d0, ad, ptx::sdesc_sw128(b0 + kk * 2048, kBoxBytes, 1024), idesc, acc);
-            if (M == Mode::kSwiGLU)
-              ptx::mma_bf16(d0 + 128, ad, ptx::sdesc_sw128(b0 + C::kBBytes + kk * 2048, kBoxBytes, 1024), idesc,
-                            acc);
+            const uint64_t bd = ptx::sdesc_sw128(b0 + kk * 2048, kBoxBytes, 1024);
+            const uint64_t cd = ptx::sdesc_sw128(b0 + 2 * kBoxBytes + kk * 2048, kBoxBytes, 1024);
+            for (int h = 0; h < ti.halves; ++h) {
+              const uint64_t ad = ptx::sdesc(a0 + h * kABytes + kk * 32, 16, kASBO, kASwizzle);
+              const uint32_t d = tmem + ((ring.next + h) & 1) * kSlotCols;
+              ptx::mma_bf16(d, ad, bd, idesc, acc);
+              if (M == Mode::kSwiGLU) ptx::mma_bf16(d + 128, ad, cd, idesc, acc);
+            }
           }
           ptx::mma_commit(&empty[s]);
         }
         if (!ok) break;
-        ptx::mma_commit(&tfull[b]);
-        ++it;
+        for (int h = 0; h < ti.halves; ++h) {
+          const int sl = (ring.next + h) & 1;
+          ptx::mma_commit(&tfull[sl]);
+          ring.bump(sl);
+        }
+        ring.next = (ring.next + ti.halves) & 1;
       }
       ptx::mma_commit(done);
       if (!ptx::wait_bounded(done, 0, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
@@ -227,81 +261,89 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    int it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    SlotRing ring;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       TileInfo ti;
       if (!tile_at(p, tile, BN, ti)) continue;
-      const int b = it & 1;
-      const uint32_t use = (uint32_t)it >> 1;
-      if (!ptx::wait_bounded(&tfull[b], use & 1, abort_flag)) {
-        raise_status(p.status, abort_flag, kStatusTimeout);
-        break;
-      }
-      ptx::tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + b * 256;
-      const bool valid = row < ti.rows;
       const int n0 = ti.nb * BN;
-      if (M == Mode::kSwiGLU) {
-        const int64_t hrow = (int64_t)ti.row0 + row + (ti.shared ? p.out_shared_row_offset : 0);
-        uint16_t* base = static_cast<uint16_t*>(ti.shared ? p.out_shared : p.out_routed);
-        uint4* out = reinterpret_cast<uint4*>(base + hrow * p.ld_out + n0);
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t g[32], u[32];
-          ptx::tmem_ld32(tbase + c * 32, g);
-          ptx::tmem_ld32(tbase + 128 + c * 32, u);
-          ptx::tmem_ld_wait2(g, u);
-          if (c == BN / 32 - 1) {
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&tempty[b]);
-          }
-          if (valid) {
-            uint32_t hp[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-              const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-              const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
-              hp[i] = ptx::pack_bf16x2(h0, h1);
-            }
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              out[c * 4 + v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
-          }
+      for (int h = 0; h < ti.halves; ++h) {
+        const int sl = (ring.next + h) & 1;
+        if (!ptx::wait_bounded(&tfull[sl], ring.use(sl) & 1, abort_flag)) {
+          raise_status(p.status, abort_flag, kStatusTimeout);
+          ok = false;
+          break;
         }
-      } else {
-        const int64_t orow = (int64_t)ti.row0 + row + (ti.shared ? p.out_shared_row_offset : 0);
+        ptx::tc_fence_after();
+        const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + sl * kSlotCols;
+        const int r = h * kTileM + row;  // row within the tile
+        const bool valid = r < ti.rows;
+        if (M == Mode::kSwiGLU) {
+          const int64_t hrow = (int64_t)ti.row0 + r + (ti.shared ? p.out_shared_row_offset : 0);
+          uint16_t* base = static_cast<uint16_t*>(ti.shared ? p.out_shared : p.out_routed);
+          uint4* out = reinterpret_cast<uint4*>(base + hrow * p.ld_out + n0);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t r[32];
-          ptx::tmem_ld32(tbase + c * 32, r);
-          ptx::tmem_ld_wait(r);
-          if (c == BN / 32 - 1) {
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&tempty[b]);
-          }
-          if (valid && n0 + c * 32 < (ti.shared ? p.N_shared : p.N_routed)) {
-            if (ti.shared) {
-              float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.out_shared) + orow * p.ld_out + n0 + c * 32);
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t g[32], u[32];
+            ptx::tmem_ld32(tbase + c * 32, g);
+            ptx::tmem_ld32(tbase + 128 + c * 32, u);
+            ptx::tmem_ld_wait2(g, u);
+            if (c == BN / 32 - 1) {
+              ptx::tc_fence_before();
+              ptx::mbar_arrive(&tempty[sl]);
+            }
+            if (valid) {
+              uint32_t hp[16];
 #pragma unroll
-              for (int v = 0; v < 8; ++v)
-                out[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                     __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-            } else {
-              uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out_routed) + orow * p.ld_out + n0 + c * 32);
+              for (int i = 0; i < 16; ++i) {
+                const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                hp[i] = ptx::pack_bf16x2(h0, h1);
+              }
 #pragma unroll
               for (int v = 0; v < 4; ++v)
-                out[v] = make_uint4(
-                    ptx::pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
-                    ptx::pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                    ptx::pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                    ptx::pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+                out[c * 4 + v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
+            }
+          }
+        } else {
+          const int64_t orow = (int64_t)ti.row0 + r + (ti.shared ? p.out_shared_row_offset : 0);
+          const int N = ti.shared ? p.N_shared : p.N_routed;
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t v32[32];
+            ptx::tmem_ld32(tbase + c * 32, v32);
+            ptx::tmem_ld_wait(v32);
+            if (c == BN / 32 - 1) {
+              ptx::tc_fence_before();
+              ptx::mbar_arrive(&tempty[sl]);
+            }
+            if (valid && n0 + c * 32 < N) {
+              if (ti.shared) {
+                float4* out =
+                    reinterpret_cast<float4*>(static_cast<float*>(p.out_shared) + orow * p.ld_out + n0 + c * 32);
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                  out[v] = make_float4(__uint_as_float(v32[4 * v]), __uint_as_float(v32[4 * v + 1]),
+                                       __uint_as_float(v32[4 * v + 2]), __uint_as_float(v32[4 * v + 3]));
+              } else {
+                uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out_routed) + orow * p.ld_out + n0 +
+                                                      c * 32);
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                  out[v] = make_uint4(
+                      ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 0]), __uint_as_float(v32[8 * v + 1])),
+                      ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 2]), __uint_as_float(v32[8 * v + 3])),
+                      ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 4]), __uint_as_float(v32[8 * v + 5])),
+                      ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 6]), __uint_as_float(v32[8 * v + 7])));
+              }
             }
           }
         }
+        ring.bump(sl);
       }
-      ++it;
+      ring.next = (ring.next + ti.halves) & 1;
     }
   }
 
@@ -318,7 +360,7 @@ template <Mode M>
 cudaError_t launch(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtensorMap& b_r, const CUtensorMap& b_s,
                    const CUtensorMap& c_r, const CUtensorMap& c_s, const GemmParams& p, int grid,
                    cudaStream_t stream) {
-  const size_t smem = smem_bytes<M>();
+  const size_t smem = smem_bytes();
   cudaError_t err =
       cudaFuncSetAttribute(grouped_gemm_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;

@@ -54,7 +54,7 @@ Layout make_layout(const moe_shape& s) {
   const int64_t T = s.T, Tk = s.T * s.k;
   const bool sh = s.shared_inter > 0;
   L.nb = permute_blocks(T);
-  L.max_mtiles = (int)((Tk + kTileM - 1) / kTileM + s.E + (sh ? (T + kTileM - 1) / kTileM : 0));
+  L.max_mtiles = (int)((Tk + kTileRows - 1) / kTileRows + s.E + (sh ? (T + kTileRows - 1) / kTileRows : 0));
   L.Hld = std::max(s.inter, s.shared_inter);
   L.Hrows = Tk + (sh ? T : 0);
   size_t off = 0;
@@ -104,9 +104,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // bf16 row-major [outer, inner]; box [box_outer rows x box_inner elements];
-// 128-byte swizzle (box_inner * 2 must be 128 bytes).
+// the swizzle span equals the box row (64 or 128 bytes).
 bool map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
             uint32_t box_outer) {
+  const CUtensorMapSwizzle swz = box_inner * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -114,17 +115,17 @@ bool map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uin
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 row-major [outer, mid, inner]; box [1 x 64 x 64], 128-byte swizzle.
-bool map_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer) {
+// bf16 row-major [outer, mid, inner]; box [1 x box_mid x 64], 128-byte swizzle.
+bool map_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer, uint32_t box_mid) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {inner, mid, outer};
   cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, box_mid, 1};
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -171,11 +172,11 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   const int sms = num_sms();
   // SwiGLU: A = gathered rows (routed) or x (shared); B = W1 | W3 column blocks
   CUtensorMap a_r, a_s, w1_r, w1_s, w3_r, w3_s;
-  if (!map_2d(&a_r, x_perm, s.d, Tk, 64, kTileM) || !map_2d(&a_s, x, s.d, s.T, 64, kTileM) ||
-      !map_3d(&w1_r, W1, s.inter, s.d, s.E) || !map_3d(&w3_r, W3, s.inter, s.d, s.E))
+  if (!map_2d(&a_r, x_perm, s.d, Tk, kGemmBK, kTileM) || !map_2d(&a_s, x, s.d, s.T, kGemmBK, kTileM) ||
+      !map_3d(&w1_r, W1, s.inter, s.d, s.E, kGemmBK) || !map_3d(&w3_r, W3, s.inter, s.d, s.E, kGemmBK))
     return MOE_ERR_CUDA;
   if (sh) {
-    if (!map_3d(&w1_s, W1s, s.shared_inter, s.d, 1) || !map_3d(&w3_s, W3s, s.shared_inter, s.d, 1))
+    if (!map_3d(&w1_s, W1s, s.shared_inter, s.d, 1, kGemmBK) || !map_3d(&w3_s, W3s, s.shared_inter, s.d, 1, kGemmBK))
       return MOE_ERR_CUDA;
   } else {
     w1_s = w1_r;
@@ -204,9 +205,10 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
 
   // down projection: A = H (routed rows, then shared rows); B = W2 column blocks
   CUtensorMap h_map, w2_r, w2_s;
-  if (!map_2d(&h_map, H, L.Hld, L.Hrows, 64, kTileM) || !map_3d(&w2_r, W2, s.d, s.inter, s.E)) return MOE_ERR_CUDA;
+  if (!map_2d(&h_map, H, L.Hld, L.Hrows, kGemmBK, kTileM) || !map_3d(&w2_r, W2, s.d, s.inter, s.E, kGemmBK))
+    return MOE_ERR_CUDA;
   if (sh) {
-    if (!map_3d(&w2_s, W2s, s.d, s.shared_inter, 1)) return MOE_ERR_CUDA;
+    if (!map_3d(&w2_s, W2s, s.d, s.shared_inter, 1, kGemmBK)) return MOE_ERR_CUDA;
   } else {
     w2_s = w2_r;
   }

@@ -7,7 +7,20 @@
 
 namespace moe {
 
-constexpr int kTileM = 128;  // rows per grouped-GEMM tile (tcgen05 M)
+constexpr int kTileM = 128;     // rows per MMA (tcgen05 M) and per A box
+constexpr int kTileRows = 256;  // rows per grouped-GEMM tile list entry (two M halves)
+
+// K depth of one grouped-GEMM pipeline stage (32: A halves use a 64-byte
+// swizzle; 64: a 128-byte swizzle) and the number of stages.
+#ifndef MOE_GEMM_BK
+#define MOE_GEMM_BK 64
+#endif
+#ifndef MOE_GEMM_STAGES
+#define MOE_GEMM_STAGES 3
+#endif
+constexpr int kGemmBK = MOE_GEMM_BK;
+constexpr int kGemmStages = MOE_GEMM_STAGES;
+static_assert(kGemmBK == 32 || kGemmBK == 64, "stage K depth must be 32 or 64");
 
 // Device status bits OR-ed into the status word at the head of the workspace.
 enum : uint32_t {

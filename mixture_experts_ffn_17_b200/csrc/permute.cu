@@ -14,7 +14,7 @@
 //                and entry (t, j) lands at offsets-based position r:
 //                perm_token[r] = t, row_of[t*k + j] = r.
 // A separate gather copies x rows into permuted order (x_perm), and the tile
-// builder lists the 128-row tiles of every expert segment (plus the shared
+// builder lists the 256-row tiles of every expert segment (plus the shared
 // expert's tiles over all T tokens) for the grouped GEMMs.
 #include <algorithm>
 #include <cstdint>
@@ -171,7 +171,7 @@ __global__ void __launch_bounds__(256)
 }
 
 // Tile list for the grouped GEMMs: one int4 {group, row_start, rows, 0} per
-// 128-row tile of each expert segment (group e, rows in permuted order), then
+// 256-row tile of each expert segment (group e, rows in permuted order), then
 // the shared expert's tiles (group E, rows in token order).  ntiles[0] = count.
 __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, int T, int with_shared,
                                    int4* __restrict__ tiles, int32_t* __restrict__ ntiles) {
@@ -183,7 +183,7 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
   if (e < E) {
     start = offsets[e];
     cnt = offsets[e + 1] - start;
-    mt = (cnt + kTileM - 1) / kTileM;
+    mt = (cnt + kTileRows - 1) / kTileRows;
   }
   int32_t incl = mt;
 #pragma unroll
@@ -208,14 +208,14 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
   __syncthreads();
   const int32_t first = warp_sums[warp] + incl - mt;
   for (int m = 0; m < mt; ++m) {
-    const int32_t r0 = m * kTileM;
-    tiles[first + m] = make_int4(e, start + r0, min(kTileM, cnt - r0), 0);
+    const int32_t r0 = m * kTileRows;
+    tiles[first + m] = make_int4(e, start + r0, min(kTileRows, cnt - r0), 0);
   }
   const int32_t routed = total;
-  const int32_t shared_tiles = with_shared ? (T + kTileM - 1) / kTileM : 0;
+  const int32_t shared_tiles = with_shared ? (T + kTileRows - 1) / kTileRows : 0;
   for (int m = threadIdx.x; m < shared_tiles; m += blockDim.x) {
-    const int32_t r0 = m * kTileM;
-    tiles[routed + m] = make_int4(E, r0, min(kTileM, T - r0), 0);
+    const int32_t r0 = m * kTileRows;
+    tiles[routed + m] = make_int4(E, r0, min(kTileRows, T - r0), 0);
   }
   if (threadIdx.x == 0) ntiles[0] = routed + shared_tiles;
 }

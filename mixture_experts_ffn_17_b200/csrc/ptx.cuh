@@ -196,14 +196,23 @@ __device__ __forceinline__ void tmem_ld_wait2(uint32_t (&r)[32], uint32_t (&q)[3
 // Shared-memory matrix descriptor (tcgen05 format): start address, leading
 // and stride byte offsets (all in 16-byte units), descriptor version 1 at
 // bits 46-47, swizzle mode at bits 61-63 (2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+// Swizzle modes of the descriptor (bits 61-63).
+constexpr uint32_t kSwizzle128B = 2;
+constexpr uint32_t kSwizzle64B = 4;
+
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                          uint32_t swizzle) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
+  d |= (uint64_t)swizzle << 61;
   return d;
+}
+
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return sdesc(saddr, lbo_bytes, sbo_bytes, kSwizzle128B);
 }
 
 // Instruction descriptor for kind::f16 with bf16 A and B and an fp32
