@@ -23,11 +23,19 @@
 //             round-robin (a one-half tile takes one, a two-half tile both),
 //             so one-half tiles overlap their epilogue with the next main loop;
 //   warps 2-5 epilogue: tcgen05.ld the accumulator rows (one row per
-//             thread), apply silu(g)*u (SwiGLU kernel) and store.
+//             thread), apply silu(g)*u (SwiGLU kernel) and store;
+//   warps 6-13 (FP8 weights only) converters: the producer brings raw e4m3
+//             weight tiles [64 K x 128 N] into the stage; these warps turn
+//             them into bf16 (code * the tile's 128 x 128 block scale) in the
+//             swizzled N-major layout the MMA reads, through a 2-deep ring.
+//             The tensor cores take A and B of one type and the activations
+//             stay bf16, so the weights are widened in shared memory and the
+//             MMA runs kind::f16.
 //
-// Kernel A (SwiGLU):  N = 128 columns of W1 and the same 128 of W3 per tile
-//                     (two MMAs per K step into two 128-column accumulators),
-//                     H[row, n0:n0+128] = bf16(silu(g) * u).
+// Kernel A (SwiGLU):  N = 128 columns of W1 and the same 128 of W3 per tile,
+//                     one N=256 MMA per K step over [W1 | W3] (g and u side by
+//                     side in the accumulator), H[row, n0:n0+128] =
+//                     bf16(silu(g) * u).
 // Kernel B (down):    N = 256 columns of W2 per tile; routed rows are stored
 //                     bf16 into Y_perm, shared-expert rows fp32 into Y_shared.
 #include <algorithm>
@@ -44,15 +52,30 @@ constexpr int kBK = kGemmBK;
 constexpr int kStages = kGemmStages;
 constexpr uint32_t kABytes = kTileM * kBK * 2;  // one 128-row half of the A tile
 constexpr uint32_t kBoxBytes = 64 * kBK * 2;    // one [kBK K x 64 N] bf16 box
-constexpr uint32_t kBBytes = 4 * kBoxBytes;     // B part of a stage
+constexpr uint32_t kBBytes = 4 * kBoxBytes;     // bf16 B part of a stage
 constexpr uint32_t kStageBytes = 2 * kABytes + kBBytes;
 // A halves: K-major rows of kBK bf16 (64 or 128 bytes), swizzled to match
 // the tensor map; 8-row groups kBK*16 bytes apart.
 constexpr uint32_t kASwizzle = kBK == 64 ? ptx::kSwizzle128B : ptx::kSwizzle64B;
 constexpr uint32_t kASBO = 8 * kBK * 2;
-static_assert(kStages * kStageBytes + 1024 + 256 <= 232448, "shared memory budget");
-constexpr uint32_t kTmemCols = 512;             // two 256-column accumulator slots
+constexpr uint32_t kTmemCols = 512;  // two 256-column accumulator slots
 constexpr uint32_t kSlotCols = 256;
+
+// FP8 weights: a stage holds the A halves and two raw e4m3 boxes
+// [64 K x 128 N] (16 KB); converted bf16 B tiles live in their own ring.
+constexpr int kF8BK = 64;
+constexpr int kF8Stages = 3;
+constexpr int kF8ConvStages = 2;
+constexpr uint32_t kF8ABytes = kTileM * kF8BK * 2;      // 16 KB
+constexpr uint32_t kF8RawBox = 64 * 128;                // 8 KB of codes
+constexpr uint32_t kF8StageBytes = 2 * kF8ABytes + 2 * kF8RawBox;
+constexpr uint32_t kF8BoxBytes = 64 * kF8BK * 2;        // bf16 [64 K x 64 N] box, 8 KB
+constexpr uint32_t kF8ConvBytes = 4 * kF8BoxBytes;      // 32 KB
+constexpr int kConvWarps = 8;
+
+static_assert(kStages * kStageBytes + 1024 + 256 <= 232448, "shared memory budget");
+static_assert(kF8Stages * kF8StageBytes + kF8ConvStages * kF8ConvBytes + 1024 + 256 <= 232448,
+              "shared memory budget (FP8)");
 
 enum class Mode { kSwiGLU, kDown };
 
@@ -67,16 +90,28 @@ struct Cfg<Mode::kDown> {
   static constexpr int BN = 256;  // columns of W2 per tile
 };
 
-constexpr size_t smem_bytes() { return 1024 + kStages * kStageBytes + 256; }
+template <bool F8>
+constexpr size_t smem_bytes() {
+  return F8 ? 1024 + kF8Stages * kF8StageBytes + kF8ConvStages * kF8ConvBytes + 256
+            : 1024 + kStages * kStageBytes + 256;
+}
 
 struct TileInfo {
-  int group, row0, rows, nb, halves;
+  int group, row0, rows, nb, halves, k_routed;
   bool shared;
 };
 
-__device__ __forceinline__ bool tile_at(const GemmParams& p, int tile, int BN, TileInfo& ti) {
-  const int mt = tile / p.n_nb;
-  ti.nb = tile - mt * p.n_nb;
+// Range of tile-list rows [mt_begin, mt_end) this launch walks.
+__device__ __forceinline__ void tile_range(const GemmParams& p, int& mt_begin, int& mt_end) {
+  const int all = min(p.ntiles[0], p.max_mtiles);
+  const int routed = min(p.ntiles[1], all);
+  mt_begin = p.tile_set == kTilesShared ? routed : 0;
+  mt_end = p.tile_set == kTilesRouted ? routed : all;
+}
+
+__device__ __forceinline__ bool tile_at(const GemmParams& p, int mt_begin, int tile, int BN, TileInfo& ti) {
+  const int mt = mt_begin + tile / p.n_nb;
+  ti.nb = tile - (tile / p.n_nb) * p.n_nb;
   const int4 e = p.tiles[mt];
   ti.group = e.x;
   ti.row0 = e.y;
@@ -99,21 +134,54 @@ struct SlotRing {
   }
 };
 
-template <Mode M>
-__global__ void __launch_bounds__(192, 1)
+// e4m3 codes (4 per word) * scale -> 4 bf16 (two packed words).  The e4m3 ->
+// f16 widening is exact; the product is rounded once to bf16.
+__device__ __forceinline__ uint2 e4m3x4_to_bf16x4(uint32_t q, float scale) {
+  uint32_t h01, h23;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "mov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, hi;\n\t}\n"
+      : "=r"(h01), "=r"(h23)
+      : "r"(q));
+  float a0, a1, b0, b1;
+  asm("{\n\t.reg .b16 l0, h0, l1, h1;\n\t"
+      "mov.b32 {l0, h0}, %4;\n\t"
+      "mov.b32 {l1, h1}, %5;\n\t"
+      "cvt.f32.f16 %0, l0;\n\t"
+      "cvt.f32.f16 %1, h0;\n\t"
+      "cvt.f32.f16 %2, l1;\n\t"
+      "cvt.f32.f16 %3, h1;\n\t}\n"
+      : "=f"(a0), "=f"(a1), "=f"(b0), "=f"(b1)
+      : "r"(h01), "r"(h23));
+  return make_uint2(ptx::pack_bf16x2(a0 * scale, a1 * scale), ptx::pack_bf16x2(b0 * scale, b1 * scale));
+}
+
+template <Mode M, bool F8>
+__global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
                         const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
                         const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s,
                         const GemmParams p) {
-  constexpr int S = kStages;
+  constexpr int S = F8 ? kF8Stages : kStages;
+  constexpr int BK = F8 ? kF8BK : kBK;
+  constexpr uint32_t ABytes = F8 ? kF8ABytes : kABytes;
+  constexpr uint32_t StageBytes = F8 ? kF8StageBytes : kStageBytes;
+  constexpr uint32_t BoxBytes = F8 ? kF8BoxBytes : kBoxBytes;
+  constexpr uint32_t ASwz = F8 ? ptx::kSwizzle128B : kASwizzle;
+  constexpr uint32_t ASBO = F8 ? 1024 : kASBO;
   constexpr int BN = Cfg<M>::BN;
+  constexpr int CS = kF8ConvStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stage0 = align_1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(stage0 + S * kStageBytes);
+  uint8_t* conv0 = stage0 + S * StageBytes;  // FP8: converted bf16 B ring
+  uint64_t* full = reinterpret_cast<uint64_t*>(conv0 + (F8 ? CS * kF8ConvBytes : 0));
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
-  uint64_t* done = tempty + 2;
+  uint64_t* cfull = tempty + 2;
+  uint64_t* cempty = cfull + CS;
+  uint64_t* done = cempty + CS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   __shared__ uint32_t never;
@@ -130,6 +198,10 @@ __global__ void __launch_bounds__(192, 1)
       ptx::mbar_init(&tfull[b], 1);
       ptx::mbar_init(&tempty[b], 128);
     }
+    for (int c = 0; c < CS; ++c) {
+      ptx::mbar_init(&cfull[c], kConvWarps * 32);
+      ptx::mbar_init(&cempty[c], 1);
+    }
     ptx::mbar_init(done, 1);
     *abort_flag = 0u;
     never = 0u;
@@ -145,33 +217,37 @@ __global__ void __launch_bounds__(192, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const int total = min(p.ntiles[0], p.max_mtiles) * p.n_nb;
+  int mt_begin, mt_end;
+  tile_range(p, mt_begin, mt_end);
+  const int total = max(0, mt_end - mt_begin) * p.n_nb;
 
   if (warp == 0) {
     if (lane == 0) {
       ptx::prefetch_tmap(&tmA_r);
-      ptx::prefetch_tmap(&tmA_s);
       ptx::prefetch_tmap(&tmB_r);
-      ptx::prefetch_tmap(&tmB_s);
+      if (!F8) {
+        ptx::prefetch_tmap(&tmA_s);
+        ptx::prefetch_tmap(&tmB_s);
+      }
       if (M == Mode::kSwiGLU) {
         ptx::prefetch_tmap(&tmC_r);
-        ptx::prefetch_tmap(&tmC_s);
+        if (!F8) ptx::prefetch_tmap(&tmC_s);
       }
       const uint64_t pol_a = ptx::policy_evict_last();   // A rows are reused by every column block
       const uint64_t pol_w = ptx::policy_evict_first();  // each weight tile is read once
       int kg = 0;
-      bool ok = true;
+      bool ok = !p.debug_withhold_loads;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
-        if (!tile_at(p, tile, BN, ti)) continue;
+        if (!tile_at(p, mt_begin, tile, BN, ti)) continue;
         const CUtensorMap* mA = ti.shared ? &tmA_s : &tmA_r;
         const CUtensorMap* mB = ti.shared ? &tmB_s : &tmB_r;
         const CUtensorMap* mC = ti.shared ? &tmC_s : &tmC_r;
         const int arow = ti.row0 + (ti.shared ? p.a_shared_row_offset : 0);
         const int e3 = ti.shared ? 0 : ti.group;
-        const int nk = (ti.shared ? p.K_shared : p.K_routed) / kBK;
+        const int nk = (ti.shared ? p.K_shared : p.K_routed) / BK;
         const int n0 = ti.nb * BN;
-        const uint32_t bytes = ti.halves * kABytes + kBBytes;
+        const uint32_t bytes = ti.halves * ABytes + (F8 ? 2 * kF8RawBox : kBBytes);
         for (int kb = 0; kb < nk; ++kb, ++kg) {
           const int s = kg % S;
           const uint32_t ph = (kg / S) & 1;
@@ -180,21 +256,42 @@ __global__ void __launch_bounds__(192, 1)
             ok = false;
             break;
           }
-          uint8_t* st = stage0 + s * kStageBytes;
+          if (kGemmL2Prefetch > 0 && !F8 && kb + kGemmL2Prefetch < nk) {
+            const int kp = (kb + kGemmL2Prefetch) * BK;
+            if (M == Mode::kSwiGLU) {
+              ptx::tma_prefetch_3d(mB, n0, kp, e3);
+              ptx::tma_prefetch_3d(mB, n0 + 64, kp, e3);
+              ptx::tma_prefetch_3d(mC, n0, kp, e3);
+              ptx::tma_prefetch_3d(mC, n0 + 64, kp, e3);
+            } else {
+#pragma unroll
+              for (int h = 0; h < 4; ++h) ptx::tma_prefetch_3d(mB, n0 + 64 * h, kp, e3);
+            }
+          }
+          uint8_t* st = stage0 + s * StageBytes;
           ptx::mbar_arrive_expect_tx(&full[s], bytes);
-          ptx::tma_load_2d(st, mA, &full[s], kb * kBK, arow, pol_a);
-          if (ti.halves == 2) ptx::tma_load_2d(st + kABytes, mA, &full[s], kb * kBK, arow + kTileM, pol_a);
-          uint8_t* sb = st + 2 * kABytes;
-          if (M == Mode::kSwiGLU) {
+          ptx::tma_load_2d(st, mA, &full[s], kb * BK, arow, pol_a);
+          if (ti.halves == 2) ptx::tma_load_2d(st + ABytes, mA, &full[s], kb * BK, arow + kTileM, pol_a);
+          uint8_t* sb = st + 2 * ABytes;
+          if (F8) {
+            // raw codes: box 0 = W1 (or W2 columns n0..n0+127), box 1 = W3 (or W2 n0+128..)
+            if (M == Mode::kSwiGLU) {
+              ptx::tma_load_3d(sb, mB, &full[s], n0, kb * BK, e3, pol_w);
+              ptx::tma_load_3d(sb + kF8RawBox, mC, &full[s], n0, kb * BK, e3, pol_w);
+            } else {
+              ptx::tma_load_3d(sb, mB, &full[s], n0, kb * BK, e3, pol_w);
+              ptx::tma_load_3d(sb + kF8RawBox, mB, &full[s], n0 + 128, kb * BK, e3, pol_w);
+            }
+          } else if (M == Mode::kSwiGLU) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
-              ptx::tma_load_3d(sb + (2 + h) * kBoxBytes, mC, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
+              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * BK, e3, pol_w);
+              ptx::tma_load_3d(sb + (2 + h) * kBoxBytes, mC, &full[s], n0 + 64 * h, kb * BK, e3, pol_w);
             }
           } else {
 #pragma unroll
             for (int h = 0; h < 4; ++h)
-              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * kBK, e3, pol_w);
+              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * BK, e3, pol_w);
           }
         }
       }
@@ -204,15 +301,18 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      // SwiGLU: two N=128 MMAs (W1 -> g, W3 -> u) per half; down: one N=256
-      constexpr uint32_t idesc = ptx::idesc_bf16(kTileM, M == Mode::kSwiGLU ? 128 : 256, false, true);
+      // One N=256 MMA per half and K step.  SwiGLU: the stage holds W1's two
+      // 64-column boxes followed by W3's, one box stride apart, so columns
+      // 0-127 of the accumulator are g = x W1 and 128-255 are u = x W3 (A is
+      // read once for both).  Down: 256 columns of W2.
+      constexpr uint32_t idesc = ptx::idesc_bf16(kTileM, 256, false, true);
       int kg = 0;
       SlotRing ring;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
-        if (!tile_at(p, tile, BN, ti)) continue;
-        const int nk = (ti.shared ? p.K_shared : p.K_routed) / kBK;
+        if (!tile_at(p, mt_begin, tile, BN, ti)) continue;
+        const int nk = (ti.shared ? p.K_shared : p.K_routed) / BK;
         for (int h = 0; h < ti.halves; ++h) {
           const int sl = (ring.next + h) & 1;
           if (!ptx::wait_bounded(&tempty[sl], (ring.use(sl) & 1) ^ 1, abort_flag)) {
@@ -225,27 +325,27 @@ __global__ void __launch_bounds__(192, 1)
         for (int kb = 0; kb < nk; ++kb, ++kg) {
           const int s = kg % S;
           const uint32_t ph = (kg / S) & 1;
-          if (!ptx::wait_bounded(&full[s], ph, abort_flag)) {
+          const int c = kg % CS;
+          if (!ptx::wait_bounded(&full[s], ph, abort_flag) ||
+              (F8 && !ptx::wait_bounded(&cfull[c], (kg / CS) & 1, abort_flag))) {
             raise_status(p.status, abort_flag, kStatusTimeout);
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t a0 = ptx::smem_u32(stage0 + s * kStageBytes);
-          const uint32_t b0 = a0 + 2 * kABytes;
+          const uint32_t a0 = ptx::smem_u32(stage0 + s * StageBytes);
+          const uint32_t b0 = F8 ? ptx::smem_u32(conv0 + c * kF8ConvBytes) : a0 + 2 * ABytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
+          for (int kk = 0; kk < BK / 16; ++kk) {
             const uint32_t acc = (kb | kk) != 0 ? 1u : 0u;
-            const uint64_t bd = ptx::sdesc_sw128(b0 + kk * 2048, kBoxBytes, 1024);
-            const uint64_t cd = ptx::sdesc_sw128(b0 + 2 * kBoxBytes + kk * 2048, kBoxBytes, 1024);
+            const uint64_t bd = ptx::sdesc_sw128(b0 + kk * 2048, BoxBytes, 1024);
             for (int h = 0; h < ti.halves; ++h) {
-              const uint64_t ad = ptx::sdesc(a0 + h * kABytes + kk * 32, 16, kASBO, kASwizzle);
-              const uint32_t d = tmem + ((ring.next + h) & 1) * kSlotCols;
-              ptx::mma_bf16(d, ad, bd, idesc, acc);
-              if (M == Mode::kSwiGLU) ptx::mma_bf16(d + 128, ad, cd, idesc, acc);
+              const uint64_t ad = ptx::sdesc(a0 + h * ABytes + kk * 32, 16, ASBO, ASwz);
+              ptx::mma_bf16(tmem + ((ring.next + h) & 1) * kSlotCols, ad, bd, idesc, acc);
             }
           }
           ptx::mma_commit(&empty[s]);
+          if (F8) ptx::mma_commit(&cempty[c]);
         }
         if (!ok) break;
         for (int h = 0; h < ti.halves; ++h) {
@@ -258,14 +358,14 @@ __global__ void __launch_bounds__(192, 1)
       ptx::mma_commit(done);
       if (!ptx::wait_bounded(done, 0, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
     }
-  } else {
+  } else if (warp < 6) {
     const int q = warp & 3;
     const int row = q * 32 + lane;
     SlotRing ring;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       TileInfo ti;
-      if (!tile_at(p, tile, BN, ti)) continue;
+      if (!tile_at(p, mt_begin, tile, BN, ti)) continue;
       const int n0 = ti.nb * BN;
       for (int h = 0; h < ti.halves; ++h) {
         const int sl = (ring.next + h) & 1;
@@ -345,6 +445,61 @@ __global__ void __launch_bounds__(192, 1)
       }
       ring.next = (ring.next + ti.halves) & 1;
     }
+  } else if (F8) {
+    // converters: kConvWarps warps.  A raw stage is 2 boxes x 64 K rows of 128
+    // codes = 128 rows; a warp step covers 4 rows, a lane 16 codes (one
+    // 16-byte load, two 16-byte stores of bf16).
+    const int cw = warp - 6;
+    const int sub_row = lane >> 3;          // row within the 4-row step
+    const int col16 = lane & 7;             // 16-code column group within the row
+    int kg = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      TileInfo ti;
+      if (!tile_at(p, mt_begin, tile, BN, ti)) continue;
+      const int nk = p.K_routed / BK;
+      const int n0 = ti.nb * BN;
+      const int ksb = p.K_routed / 128, nsb = p.N_routed / 128;  // scale blocks per expert
+      for (int kb = 0; kb < nk; ++kb, ++kg) {
+        const int s = kg % S;
+        const int c = kg % CS;
+        if (!ptx::wait_bounded(&full[s], (kg / S) & 1, abort_flag) ||
+            !ptx::wait_bounded(&cempty[c], ((kg / CS) & 1) ^ 1, abort_flag)) {
+          raise_status(p.status, abort_flag, kStatusTimeout);
+          ok = false;
+          break;
+        }
+        const uint8_t* raw = stage0 + s * kF8StageBytes + 2 * kF8ABytes;
+        uint8_t* conv = conv0 + c * kF8ConvBytes;
+        const int kblk = (kb * BK) / 128;
+        const int64_t sbase = ((int64_t)ti.group * ksb + kblk) * nsb;
+        float sc[2];
+        if (M == Mode::kSwiGLU) {
+          sc[0] = p.scale_b[sbase + n0 / 128];
+          sc[1] = p.scale_c[sbase + n0 / 128];
+        } else {
+          sc[0] = p.scale_b[sbase + n0 / 128];
+          sc[1] = n0 + 128 < p.N_routed ? p.scale_b[sbase + n0 / 128 + 1] : 0.0f;  // past the last column
+        }
+#pragma unroll
+        for (int i = 0; i < 128 / (4 * kConvWarps); ++i) {
+          const int rr = (cw * (128 / kConvWarps)) + i * 4 + sub_row;  // 0..127
+          const int box = rr >> 6, k = rr & 63;
+          const uint4 q = *reinterpret_cast<const uint4*>(raw + box * kF8RawBox + k * 128 + col16 * 16);
+          const float scale = box ? sc[1] : sc[0];
+          const uint2 v0 = e4m3x4_to_bf16x4(q.x, scale), v1 = e4m3x4_to_bf16x4(q.y, scale);
+          const uint2 v2 = e4m3x4_to_bf16x4(q.z, scale), v3 = e4m3x4_to_bf16x4(q.w, scale);
+          // codes col16*16 .. +15 of box `box` = bf16 sub-box 2*box + col16/4,
+          // 16-byte chunks 2*(col16%4) and 2*(col16%4)+1 of row k (swizzled)
+          uint8_t* dst = conv + (2 * box + (col16 >> 2)) * kF8BoxBytes + k * 128;
+          const int ch = 2 * (col16 & 3);
+          *reinterpret_cast<uint4*>(dst + ((ch ^ (k & 7)) << 4)) = make_uint4(v0.x, v0.y, v1.x, v1.y);
+          *reinterpret_cast<uint4*>(dst + (((ch + 1) ^ (k & 7)) << 4)) = make_uint4(v2.x, v2.y, v3.x, v3.y);
+        }
+        ptx::fence_proxy_async();
+        ptx::mbar_arrive(&cfull[c]);
+      }
+    }
   }
 
   ptx::tc_fence_before();
@@ -356,16 +511,16 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
-template <Mode M>
+template <Mode M, bool F8>
 cudaError_t launch(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtensorMap& b_r, const CUtensorMap& b_s,
                    const CUtensorMap& c_r, const CUtensorMap& c_s, const GemmParams& p, int grid,
                    cudaStream_t stream) {
-  const size_t smem = smem_bytes();
+  const size_t smem = smem_bytes<F8>();
   cudaError_t err =
-      cudaFuncSetAttribute(grouped_gemm_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(grouped_gemm_kernel<M, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   if (grid <= 0) return cudaSuccess;
-  grouped_gemm_kernel<M><<<grid, 192, smem, stream>>>(a_r, a_s, b_r, b_s, c_r, c_s, p);
+  grouped_gemm_kernel<M, F8><<<grid, F8 ? 192 + 32 * kConvWarps : 192, smem, stream>>>(a_r, a_s, b_r, b_s, c_r, c_s, p);
   return cudaGetLastError();
 }
 
@@ -377,12 +532,23 @@ int gemm_block_n_down() { return Cfg<Mode::kDown>::BN; }
 cudaError_t launch_grouped_swiglu(const CUtensorMap& tmA_r, const CUtensorMap& tmA_s, const CUtensorMap& tmW1_r,
                                   const CUtensorMap& tmW1_s, const CUtensorMap& tmW3_r, const CUtensorMap& tmW3_s,
                                   const GemmParams& p, int grid, cudaStream_t stream) {
-  return launch<Mode::kSwiGLU>(tmA_r, tmA_s, tmW1_r, tmW1_s, tmW3_r, tmW3_s, p, grid, stream);
+  return launch<Mode::kSwiGLU, false>(tmA_r, tmA_s, tmW1_r, tmW1_s, tmW3_r, tmW3_s, p, grid, stream);
 }
 
 cudaError_t launch_grouped_down(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
                                 const GemmParams& p, int grid, cudaStream_t stream) {
-  return launch<Mode::kDown>(tmA, tmA, tmW2_r, tmW2_s, tmW2_r, tmW2_s, p, grid, stream);
+  return launch<Mode::kDown, false>(tmA, tmA, tmW2_r, tmW2_s, tmW2_r, tmW2_s, p, grid, stream);
+}
+
+cudaError_t launch_grouped_swiglu_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,
+                                      const CUtensorMap& tmW3_r, const GemmParams& p, int grid,
+                                      cudaStream_t stream) {
+  return launch<Mode::kSwiGLU, true>(tmA_r, tmA_r, tmW1_r, tmW1_r, tmW3_r, tmW3_r, p, grid, stream);
+}
+
+cudaError_t launch_grouped_down_fp8(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const GemmParams& p, int grid,
+                                    cudaStream_t stream) {
+  return launch<Mode::kDown, true>(tmA, tmA, tmW2_r, tmW2_r, tmW2_r, tmW2_r, p, grid, stream);
 }
 
 }  // namespace moe

@@ -4,6 +4,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -74,7 +75,7 @@ Layout make_layout(const moe_shape& s) {
   L.perm = take((size_t)Tk * 4);
   L.row_of = take((size_t)Tk * 4);
   L.tiles = take((size_t)L.max_mtiles * 16);
-  L.ntiles = take(4);
+  L.ntiles = take(8);
   L.x_perm = take((size_t)Tk * s.d * 2);
   L.H = take((size_t)L.Hrows * L.Hld * 2);
   L.Y_perm = take((size_t)Tk * s.d * 2);
@@ -132,6 +133,28 @@ bool map_3d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint6
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// uint8 (e4m3 codes) row-major [outer, mid, inner]; box [1 x 64 x 128], no
+// swizzle (the converter warps read the codes row by row).
+bool map_3d_u8(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t mid, uint64_t outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, mid, outer};
+  cuuint64_t strides[2] = {inner, inner * mid};
+  cuuint32_t box[3] = {128, 64, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// MOE_DEBUG_WITHHOLD_LOADS=1 in the environment makes the grouped-GEMM
+// producers issue no loads (failure-path testing: their consumers' bounded
+// waits run out and the call reports MOE_ERR_DEVICE_TIMEOUT).
+bool debug_withhold_loads() {
+  const char* v = std::getenv("MOE_DEBUG_WITHHOLD_LOADS");
+  return v && v[0] == '1';
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 148;
@@ -158,9 +181,11 @@ moe_status run_router(const moe_shape& s, const void* x, const void* Wg, const f
 }
 
 moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void* x, const void* x_perm,
-                       const int32_t* offsets, const void* W1, const void* W3, const void* W2, const void* W1s,
-                       const void* W3s, const void* W2s, void* Y_perm, float* Y_shared, uint32_t* status,
-                       cudaStream_t st, const cudaEvent_t* ev = nullptr) {
+                       const int32_t* offsets, const void* W1, const void* W3, const void* W2, const float* s1,
+                       const float* s3, const float* s2, const void* W1s, const void* W3s, const void* W2s,
+                       void* Y_perm, float* Y_shared, uint32_t* status, cudaStream_t st,
+                       const cudaEvent_t* ev = nullptr) {
+  const bool f8 = s.w_dtype == MOE_E4M3;
   const bool sh = s.shared_inter > 0;
   const int64_t Tk = s.T * s.k;
   int4* tiles = at<int4>(ws, L.tiles);
@@ -171,10 +196,19 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
 
   const int sms = num_sms();
   // SwiGLU: A = gathered rows (routed) or x (shared); B = W1 | W3 column blocks
-  CUtensorMap a_r, a_s, w1_r, w1_s, w3_r, w3_s;
-  if (!map_2d(&a_r, x_perm, s.d, Tk, kGemmBK, kTileM) || !map_2d(&a_s, x, s.d, s.T, kGemmBK, kTileM) ||
-      !map_3d(&w1_r, W1, s.inter, s.d, s.E, kGemmBK) || !map_3d(&w3_r, W3, s.inter, s.d, s.E, kGemmBK))
+  CUtensorMap a_r, a_s, w1_r, w1_s, w3_r, w3_s, a8_r, w18_r, w38_r;
+  if (!map_2d(&a_r, x_perm, s.d, Tk, kGemmBK, kTileM) || !map_2d(&a_s, x, s.d, s.T, kGemmBK, kTileM))
     return MOE_ERR_CUDA;
+  if (f8) {
+    // FP8 launches use a 64-deep K stage whatever the bf16 kernel's depth
+    if (!map_2d(&a8_r, x_perm, s.d, Tk, 64, kTileM) || !map_3d_u8(&w18_r, W1, s.inter, s.d, s.E) ||
+        !map_3d_u8(&w38_r, W3, s.inter, s.d, s.E))
+      return MOE_ERR_CUDA;
+    w1_r = a_r;  // placeholders: the bf16 launch below only walks the shared expert's tiles
+    w3_r = a_r;
+  } else if (!map_3d(&w1_r, W1, s.inter, s.d, s.E, kGemmBK) || !map_3d(&w3_r, W3, s.inter, s.d, s.E, kGemmBK)) {
+    return MOE_ERR_CUDA;
+  }
   if (sh) {
     if (!map_3d(&w1_s, W1s, s.shared_inter, s.d, 1, kGemmBK) || !map_3d(&w3_s, W3s, s.shared_inter, s.d, 1, kGemmBK))
       return MOE_ERR_CUDA;
@@ -199,14 +233,35 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   p1.out_shared_row_offset = Tk;
   p1.ld_out = L.Hld;
   p1.status = status;
+  p1.tile_set = kTilesAll;
+  p1.debug_withhold_loads = debug_withhold_loads() ? 1 : 0;
   const int grid1 = (int)std::min<int64_t>(sms, (int64_t)L.max_mtiles * p1.n_nb);
-  MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, p1, grid1, st));
+  if (f8) {
+    GemmParams q = p1;
+    q.tile_set = kTilesRouted;
+    q.scale_b = s1;
+    q.scale_c = s3;
+    MOE_CUDA(launch_grouped_swiglu_fp8(a8_r, w18_r, w38_r, q, grid1, st));
+    if (sh) {
+      q = p1;
+      q.tile_set = kTilesShared;
+      MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, q, grid1, st));
+    }
+  } else {
+    MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, p1, grid1, st));
+  }
   if (ev) MOE_CUDA(cudaEventRecord(ev[1], st));
 
   // down projection: A = H (routed rows, then shared rows); B = W2 column blocks
-  CUtensorMap h_map, w2_r, w2_s;
-  if (!map_2d(&h_map, H, L.Hld, L.Hrows, kGemmBK, kTileM) || !map_3d(&w2_r, W2, s.d, s.inter, s.E, kGemmBK))
+  CUtensorMap h_map, w2_r, w2_s, h8_map, w28_r;
+  if (!map_2d(&h_map, H, L.Hld, L.Hrows, kGemmBK, kTileM)) return MOE_ERR_CUDA;
+  if (f8) {
+    if (!map_2d(&h8_map, H, L.Hld, L.Hrows, 64, kTileM) || !map_3d_u8(&w28_r, W2, s.d, s.inter, s.E))
+      return MOE_ERR_CUDA;
+    w2_r = h_map;  // placeholder: the bf16 launch below only walks the shared expert's tiles
+  } else if (!map_3d(&w2_r, W2, s.d, s.inter, s.E, kGemmBK)) {
     return MOE_ERR_CUDA;
+  }
   if (sh) {
     if (!map_3d(&w2_s, W2s, s.d, s.shared_inter, 1, kGemmBK)) return MOE_ERR_CUDA;
   } else {
@@ -225,7 +280,20 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   p2.out_shared_row_offset = 0;
   p2.ld_out = s.d;
   const int grid2 = (int)std::min<int64_t>(sms, (int64_t)L.max_mtiles * p2.n_nb);
-  MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, p2, grid2, st));
+  if (f8) {
+    GemmParams q = p2;
+    q.tile_set = kTilesRouted;
+    q.scale_b = s2;
+    q.scale_c = s2;
+    MOE_CUDA(launch_grouped_down_fp8(h8_map, w28_r, q, grid2, st));
+    if (sh) {
+      q = p2;
+      q.tile_set = kTilesShared;
+      MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, q, grid2, st));
+    }
+  } else {
+    MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, p2, grid2, st));
+  }
   if (ev) MOE_CUDA(cudaEventRecord(ev[2], st));
   return MOE_OK;
 }
@@ -249,7 +317,6 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   const void* ptrs[] = {x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out, counts_out};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (s.w_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
   const Layout L = make_layout(s);
   if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
   if (s.T == 0) return MOE_OK;
@@ -274,7 +341,7 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
                           perm, row_of, status, st));
   MOE_CUDA(launch_gather_rows(x, perm, s.T * s.k, s.d, x_perm, num_sms(), st));
-  r = run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, W1s, W3s, W2s, Y_perm, Y_shared, status, st,
+  r = run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared, status, st,
                   ev ? ev + 2 : nullptr);
   if (r != MOE_OK) return r;
   MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16, st));
@@ -354,15 +421,14 @@ moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const void*
   const void* ptrs[] = {x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
-  if (s.w_dtype == MOE_E4M3) return MOE_ERR_UNSUPPORTED;
   const Layout L = make_layout(s);
   if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t* status = at<uint32_t>(ws, L.status);
   MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
   if (s.T == 0) return MOE_OK;
-  return run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, W1s, W3s, W2s, Y_perm, sh ? Y_shared : nullptr,
-                     status, st);
+  return run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm,
+                     sh ? Y_shared : nullptr, status, st);
 }
 
 moe_status moe_combine(const moe_shape* shape, const void* Y_perm, const float* Y_shared, const int32_t* row_of,

@@ -18,6 +18,12 @@ constexpr int kTileRows = 256;  // rows per grouped-GEMM tile list entry (two M 
 #ifndef MOE_GEMM_STAGES
 #define MOE_GEMM_STAGES 3
 #endif
+// Weight boxes are prefetched into L2 this many K stages ahead of their load
+// (0 = off).
+#ifndef MOE_GEMM_L2_PREFETCH
+#define MOE_GEMM_L2_PREFETCH 0
+#endif
+constexpr int kGemmL2Prefetch = MOE_GEMM_L2_PREFETCH;
 constexpr int kGemmBK = MOE_GEMM_BK;
 constexpr int kGemmStages = MOE_GEMM_STAGES;
 static_assert(kGemmBK == 32 || kGemmBK == 64, "stage K depth must be 32 or 64");
@@ -58,20 +64,31 @@ cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, bool wi
                                int32_t* ntiles, cudaStream_t stream);
 
 // grouped_gemm.cu
+// Which part of the tile list a grouped-GEMM launch walks.
+enum TileSet : int { kTilesAll = 0, kTilesRouted = 1, kTilesShared = 2 };
+
 struct GemmParams {
   const int4* tiles;
-  const int32_t* ntiles;
-  int max_mtiles;        // capacity of the tile list (clamps the device count)
-  int E;                 // group index E = shared expert
-  int n_nb;              // N blocks per tile row (max over routed / shared)
+  const int32_t* ntiles;  // [0] = all tiles, [1] = routed tiles (the shared expert's follow)
+  int max_mtiles;         // capacity of the tile list (clamps the device counts)
+  int tile_set;           // TileSet
+  int E;                  // group index E = shared expert
+  int n_nb;               // N blocks per tile row (max over routed / shared)
   int K_routed, K_shared;
   int N_routed, N_shared;
   int a_shared_row_offset;  // row of the shared expert's first A row in its map
-  void* out_routed;      // bf16 rows
-  void* out_shared;      // SwiGLU: bf16 rows; down: fp32 rows
+  void* out_routed;       // bf16 rows
+  void* out_shared;       // SwiGLU: bf16 rows; down: fp32 rows
   int64_t out_shared_row_offset;  // rows to skip in out_shared
-  int ld_out;            // output row stride (elements)
+  int ld_out;             // output row stride (elements)
+  // FP8 routed weights: fp32 block scales [E, K/128, N/128] of the B (and,
+  // SwiGLU, C = W3) operand
+  const float* scale_b;
+  const float* scale_c;
   uint32_t* status;
+  // Failure-path testing: when nonzero the producer issues no loads, so the
+  // MMA issuer's bounded wait runs out and the launch reports a timeout.
+  int debug_withhold_loads;
 };
 
 int gemm_block_n_swiglu();
@@ -81,6 +98,13 @@ cudaError_t launch_grouped_swiglu(const CUtensorMap& tmA_r, const CUtensorMap& t
                                   const GemmParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_grouped_down(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
                                 const GemmParams& p, int grid, cudaStream_t stream);
+// FP8 (e4m3 + 128x128 block scales) routed experts; the tensor maps of W are
+// uint8 [E, K, N] with [1 x 64 x 128] boxes and no swizzle.
+cudaError_t launch_grouped_swiglu_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,
+                                      const CUtensorMap& tmW3_r, const GemmParams& p, int grid,
+                                      cudaStream_t stream);
+cudaError_t launch_grouped_down_fp8(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const GemmParams& p, int grid,
+                                    cudaStream_t stream);
 
 // combine.cu
 cudaError_t launch_combine(const void* Y_perm, const float* Y_shared, const int32_t* row_of, const float* topk_w,

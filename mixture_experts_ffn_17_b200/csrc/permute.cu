@@ -172,7 +172,8 @@ __global__ void __launch_bounds__(256)
 
 // Tile list for the grouped GEMMs: one int4 {group, row_start, rows, 0} per
 // 256-row tile of each expert segment (group e, rows in permuted order), then
-// the shared expert's tiles (group E, rows in token order).  ntiles[0] = count.
+// the shared expert's tiles (group E, rows in token order).  ntiles[0] = all
+// tiles, ntiles[1] = routed tiles.
 __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, int T, int with_shared,
                                    int4* __restrict__ tiles, int32_t* __restrict__ ntiles) {
   __shared__ int32_t warp_sums[32];
@@ -217,7 +218,10 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
     const int32_t r0 = m * kTileRows;
     tiles[routed + m] = make_int4(E, r0, min(kTileRows, T - r0), 0);
   }
-  if (threadIdx.x == 0) ntiles[0] = routed + shared_tiles;
+  if (threadIdx.x == 0) {
+    ntiles[0] = routed + shared_tiles;
+    ntiles[1] = routed;
+  }
 }
 
 }  // namespace

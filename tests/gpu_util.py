@@ -59,24 +59,50 @@ def oracle_full(w: workloads.Workload, force_idx=None):
                               route_scale=cfg.route_scale, force_idx=force_idx, **shared)
 
 
-def oracle_sampled(w: workloads.Workload, lg: np.ndarray, idx: np.ndarray, tokens: np.ndarray):
+def oracle_sampled(w: workloads.Workload, lg: np.ndarray, idx: np.ndarray, tokens: np.ndarray, threads=None):
     """Oracle outputs for a sample of tokens, fetching one expert at a time.
 
     lg: fp64 logits [T, E]; idx: the routing to use [T, k] (the oracle's, with
-    near-tie tokens replaced by the device's choice)."""
+    near-tie tokens replaced by the device's choice).  Experts run in a few
+    host threads (each oracle call is independent)."""
+    import concurrent.futures
+    import os
     cfg = w.cfg
     x = dec(w.x[torch.as_tensor(tokens, device=w.x.device)])
     wts = oracle.weights_for(lg[tokens], idx[tokens], cfg.route, cfg.route_scale)
-    y = np.zeros((len(tokens), cfg.d))
     sel = idx[tokens]
-    for e in np.unique(sel):
+
+    def one(e):
         rows, slots = np.nonzero(sel == e)
         W1, W3, W2 = expert_weights_f64(w, int(e))
-        o = oracle.swiglu_rows(x[rows], W1, W3, W2)
-        y[rows] += wts[rows, slots][:, None] * o
+        return rows, wts[rows, slots][:, None] * oracle.swiglu_rows(x[rows], W1, W3, W2)
+
+    y = np.zeros((len(tokens), cfg.d))
+    n = threads or max(1, min(8, (os.cpu_count() or 2) // 2))
+    with concurrent.futures.ThreadPoolExecutor(n) as ex:
+        for rows, contrib in ex.map(one, [int(e) for e in np.unique(sel)]):
+            np.add.at(y, rows, contrib)
     if cfg.shared_inter > 0:
         y += oracle.swiglu_rows(x, dec(w.W1s), dec(w.W3s), dec(w.W2s))
     return y
+
+
+def choose_sample(idx: np.ndarray, counts: np.ndarray, near_tie_tokens, size: int, seed: int) -> np.ndarray:
+    """Sample of tokens for output checks at full size: every near-tie token,
+    tokens on the 3 most- and 3 least-loaded non-empty experts, the first and
+    last token, the rest seeded random."""
+    T = idx.shape[0]
+    pick = set(int(t) for t in near_tie_tokens)
+    pick.update((0, T - 1))
+    nz = np.nonzero(counts > 0)[0]
+    order = nz[np.argsort(counts[nz], kind="stable")]
+    for e in list(order[:3]) + list(order[-3:]):
+        toks = np.nonzero((idx == e).any(axis=1))[0]
+        pick.update(int(t) for t in toks[:2])
+    rng = np.random.default_rng(seed)
+    rest = [t for t in rng.permutation(T) if t not in pick]
+    pick.update(int(t) for t in rest[:max(0, size - len(pick))])
+    return np.array(sorted(pick), dtype=np.int64)
 
 
 def oracle_logits(w: workloads.Workload) -> np.ndarray:

@@ -11,8 +11,8 @@ from mixture_experts_ffn_17_b200 import binding as B
 from mixture_experts_ffn_17_b200 import build as libbuild
 from mixture_experts_ffn_17_b200 import workloads
 
-from gpu_util import oracle_full, route_with_exemptions, run_forward, to_device
-from parity import TOL_BF16, bf16_stored_ok, dec, max_rel_err, to_np
+from gpu_util import expert_weights_f64, oracle_full, route_with_exemptions, run_forward, to_device
+from parity import TOL_BF16, TOL_FP8, bf16_stored_ok, dec, max_rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -149,17 +149,17 @@ def _experts_case(w, idx_np):
     offsets = torch.as_tensor(o, device="cuda")
     Y_perm = torch.empty(T * k, cfg.d, dtype=torch.bfloat16, device="cuda")
     Y_sh = torch.empty(T, cfg.d, dtype=torch.float32, device="cuda") if cfg.shared_inter else None
-    B.grouped_swiglu(shape, w.x, x_perm, offsets, w.W1, w.W3, w.W2, None, None, None, w.W1s, w.W3s, w.W2s, Y_perm,
+    B.grouped_swiglu(shape, w.x, x_perm, offsets, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s, Y_perm,
                      Y_sh, ws)
     rc, raw = B.check_device_status(ws)
     assert rc == B.MOE_OK, raw
     x = dec(w.x)
-    W1, W3, W2 = dec(w.W1), dec(w.W3), dec(w.W2)
     ref = np.zeros((T * k, cfg.d))
     for e in range(cfg.E):
         if c[e]:
-            ref[o[e]:o[e + 1]] = oracle.swiglu_rows(x[p[o[e]:o[e + 1]]], W1[e], W3[e], W2[e])
-    assert bf16_stored_ok(dec(Y_perm), ref), max_rel_err(dec(Y_perm), ref)
+            W1, W3, W2 = expert_weights_f64(w, e)
+            ref[o[e]:o[e + 1]] = oracle.swiglu_rows(x[p[o[e]:o[e + 1]]], W1, W3, W2)
+    assert bf16_stored_ok(dec(Y_perm), ref, tol=(3e-2 if cfg.fp8 else 1e-2)), max_rel_err(dec(Y_perm), ref)
     if cfg.shared_inter:
         ref_s = oracle.swiglu_rows(x, dec(w.W1s), dec(w.W3s), dec(w.W2s))
         assert max_rel_err(to_np(Y_sh).astype(np.float64), ref_s) <= TOL_BF16
@@ -263,3 +263,33 @@ def test_forward_is_deterministic():
     a, ia, *_ = run_forward(w)
     b, ib, *_ = run_forward(w)
     assert torch.equal(a, b) and torch.equal(ia, ib)
+
+
+# --------------------------------------------------------------- FP8 experts
+def _fp8(**kw):
+    shape = dict(T=700, d=512, E=64, k=6, inter=256, shared_inter=256, n_group=8, topk_group=3)
+    shape.update(kw)
+    return to_device(workloads.make_small("fp8", **shape))
+
+
+def test_grouped_swiglu_fp8_weights():
+    w = _fp8()
+    lg = oracle.logits(dec(w.x), dec(w.Wg))
+    idx, _, _, _ = oracle.route_sigmoid_group(lg, dec(w.bias), w.cfg.k, w.cfg.n_group, w.cfg.topk_group, 2, 2.5)
+    _experts_case(w, idx)
+
+
+def test_grouped_swiglu_fp8_oversize_segments():
+    w = _fp8(T=600, k=2, E=32, n_group=4, topk_group=2, d=768, inter=384)
+    idx = np.zeros((600, 2), dtype=np.int32)
+    idx[:, 0] = 5
+    idx[:, 1] = 30 + (np.arange(600) % 2)
+    _experts_case(w, idx)
+
+
+def test_forward_fp8_group_routing():
+    _check_forward(_fp8(), tol=TOL_FP8)
+
+
+def test_forward_fp8_no_shared_expert():
+    _check_forward(_fp8(T=300, shared_inter=0), tol=TOL_FP8)
