@@ -72,6 +72,7 @@ constexpr uint32_t kF8StageBytes = 2 * kF8ABytes + 2 * kF8RawBox;
 constexpr uint32_t kF8BoxBytes = 64 * kF8BK * 2;        // bf16 [64 K x 64 N] box, 8 KB
 constexpr uint32_t kF8ConvBytes = 4 * kF8BoxBytes;      // 32 KB
 constexpr int kConvWarps = 8;
+constexpr int kSchedDepth = 4;  // tile indices the producer may publish ahead
 
 static_assert(kStages * kStageBytes + 1024 + 256 <= 232448, "shared memory budget");
 static_assert(kF8Stages * kF8StageBytes + kF8ConvStages * kF8ConvBytes + 1024 + 256 <= 232448,
@@ -101,18 +102,37 @@ struct TileInfo {
   bool shared;
 };
 
-// Range of tile-list rows [mt_begin, mt_end) this launch walks.
-__device__ __forceinline__ void tile_range(const GemmParams& p, int& mt_begin, int& mt_end) {
+// The part of the tile list this launch walks: `count` tile-list rows.  A
+// launch over the whole list interleaves the shared expert's rows evenly among
+// the routed ones (the shared weights stay in L2 while routed tiles keep HBM
+// busy); the routed-only and shared-only launches walk their range in order.
+struct TileSpan {
+  int begin, count, routed, shared;
+};
+
+__device__ __forceinline__ TileSpan tile_span(const GemmParams& p) {
   const int all = min(p.ntiles[0], p.max_mtiles);
   const int routed = min(p.ntiles[1], all);
-  mt_begin = p.tile_set == kTilesShared ? routed : 0;
-  mt_end = p.tile_set == kTilesRouted ? routed : all;
+  TileSpan t;
+  t.routed = routed;
+  t.shared = all - routed;
+  t.begin = p.tile_set == kTilesShared ? routed : 0;
+  t.count = p.tile_set == kTilesRouted ? routed : (p.tile_set == kTilesShared ? all - routed : all);
+  return t;
 }
 
-__device__ __forceinline__ bool tile_at(const GemmParams& p, int mt_begin, int tile, int BN, TileInfo& ti) {
-  const int mt = mt_begin + tile / p.n_nb;
-  ti.nb = tile - (tile / p.n_nb) * p.n_nb;
-  const int4 e = p.tiles[mt];
+__device__ __forceinline__ int tile_row(const GemmParams& p, const TileSpan& sp, int q) {
+  if (p.tile_set != kTilesAll || sp.shared == 0) return sp.begin + q;
+  const int stride = sp.count / sp.shared;  // >= 1; shared row j sits at slot (j+1)*stride-1
+  const int before = min(sp.shared, (q + 1) / stride);
+  if ((q + 1) % stride == 0 && (q + 1) / stride <= sp.shared) return sp.routed + (q + 1) / stride - 1;
+  return q - before;
+}
+
+__device__ __forceinline__ bool tile_at(const GemmParams& p, const TileSpan& sp, int tile, int BN, TileInfo& ti) {
+  const int q = tile / p.n_nb;
+  ti.nb = tile - q * p.n_nb;
+  const int4 e = p.tiles[tile_row(p, sp, q)];
   ti.group = e.x;
   ti.row0 = e.y;
   ti.rows = e.z;
@@ -181,9 +201,12 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
   uint64_t* tempty = tfull + 2;
   uint64_t* cfull = tempty + 2;
   uint64_t* cempty = cfull + CS;
-  uint64_t* done = cempty + CS;
+  uint64_t* sfull = cempty + CS;  // tile-index ring: producer -> other roles
+  uint64_t* sempty = sfull + kSchedDepth;
+  uint64_t* done = sempty + kSchedDepth;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
+  volatile int* sched_tile = reinterpret_cast<volatile int*>(tmem_slot + 2);
   __shared__ uint32_t never;
 
   const int warp = threadIdx.x >> 5;
@@ -202,6 +225,10 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
       ptx::mbar_init(&cfull[c], kConvWarps * 32);
       ptx::mbar_init(&cempty[c], 1);
     }
+    for (int i = 0; i < kSchedDepth; ++i) {
+      ptx::mbar_init(&sfull[i], 1);
+      ptx::mbar_init(&sempty[i], 1 + 128 + (F8 ? kConvWarps * 32 : 0));
+    }
     ptx::mbar_init(done, 1);
     *abort_flag = 0u;
     never = 0u;
@@ -217,9 +244,23 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  int mt_begin, mt_end;
-  tile_range(p, mt_begin, mt_end);
-  const int total = max(0, mt_end - mt_begin) * p.n_nb;
+  const TileSpan span = tile_span(p);
+  const int total = span.count * p.n_nb;
+
+  // Consumers take tile indices from the ring in the order the producer
+  // claimed them; -1 ends the sequence.
+  auto next_tile = [&](int& n, bool& ok) -> int {
+    const int sd = n % kSchedDepth;
+    if (!ptx::wait_bounded(&sfull[sd], (n / kSchedDepth) & 1, abort_flag)) {
+      raise_status(p.status, abort_flag, kStatusTimeout);
+      ok = false;
+      return -1;
+    }
+    const int t = sched_tile[sd];
+    ptx::mbar_arrive(&sempty[sd]);
+    ++n;
+    return t;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -235,11 +276,26 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
       }
       const uint64_t pol_a = ptx::policy_evict_last();   // A rows are reused by every column block
       const uint64_t pol_w = ptx::policy_evict_first();  // each weight tile is read once
-      int kg = 0;
+      const uint64_t pol_ws = ptx::policy_evict_last();  // the shared expert's weights serve every row tile
+      int kg = 0, ns = 0;
       bool ok = !p.debug_withhold_loads;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      while (ok) {
+        // claim the next tile and publish it to the other roles
+        int tile = atomicAdd(p.sched_counter, 1);
+        if (tile >= total) tile = -1;
+        const int sd = ns % kSchedDepth;
+        if (!ptx::wait_bounded(&sempty[sd], ((ns / kSchedDepth) & 1) ^ 1, abort_flag)) {
+          raise_status(p.status, abort_flag, kStatusTimeout);
+          ok = false;
+          break;
+        }
+        sched_tile[sd] = tile;
+        ptx::mbar_arrive(&sfull[sd]);
+        ++ns;
+        if (tile < 0) break;
         TileInfo ti;
-        if (!tile_at(p, mt_begin, tile, BN, ti)) continue;
+        if (!tile_at(p, span, tile, BN, ti)) continue;
+        const uint64_t pol_b = ti.shared ? pol_ws : pol_w;
         const CUtensorMap* mA = ti.shared ? &tmA_s : &tmA_r;
         const CUtensorMap* mB = ti.shared ? &tmB_s : &tmB_r;
         const CUtensorMap* mC = ti.shared ? &tmC_s : &tmC_r;
@@ -276,22 +332,22 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
           if (F8) {
             // raw codes: box 0 = W1 (or W2 columns n0..n0+127), box 1 = W3 (or W2 n0+128..)
             if (M == Mode::kSwiGLU) {
-              ptx::tma_load_3d(sb, mB, &full[s], n0, kb * BK, e3, pol_w);
-              ptx::tma_load_3d(sb + kF8RawBox, mC, &full[s], n0, kb * BK, e3, pol_w);
+              ptx::tma_load_3d(sb, mB, &full[s], n0, kb * BK, e3, pol_b);
+              ptx::tma_load_3d(sb + kF8RawBox, mC, &full[s], n0, kb * BK, e3, pol_b);
             } else {
-              ptx::tma_load_3d(sb, mB, &full[s], n0, kb * BK, e3, pol_w);
-              ptx::tma_load_3d(sb + kF8RawBox, mB, &full[s], n0 + 128, kb * BK, e3, pol_w);
+              ptx::tma_load_3d(sb, mB, &full[s], n0, kb * BK, e3, pol_b);
+              ptx::tma_load_3d(sb + kF8RawBox, mB, &full[s], n0 + 128, kb * BK, e3, pol_b);
             }
           } else if (M == Mode::kSwiGLU) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * BK, e3, pol_w);
-              ptx::tma_load_3d(sb + (2 + h) * kBoxBytes, mC, &full[s], n0 + 64 * h, kb * BK, e3, pol_w);
+              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * BK, e3, pol_b);
+              ptx::tma_load_3d(sb + (2 + h) * kBoxBytes, mC, &full[s], n0 + 64 * h, kb * BK, e3, pol_b);
             }
           } else {
 #pragma unroll
             for (int h = 0; h < 4; ++h)
-              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * BK, e3, pol_w);
+              ptx::tma_load_3d(sb + h * kBoxBytes, mB, &full[s], n0 + 64 * h, kb * BK, e3, pol_b);
           }
         }
       }
@@ -306,12 +362,14 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
       // 0-127 of the accumulator are g = x W1 and 128-255 are u = x W3 (A is
       // read once for both).  Down: 256 columns of W2.
       constexpr uint32_t idesc = ptx::idesc_bf16(kTileM, 256, false, true);
-      int kg = 0;
+      int kg = 0, ns = 0;
       SlotRing ring;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      while (ok) {
+        const int tile = next_tile(ns, ok);
+        if (tile < 0) break;
         TileInfo ti;
-        if (!tile_at(p, mt_begin, tile, BN, ti)) continue;
+        if (!tile_at(p, span, tile, BN, ti)) continue;
         const int nk = (ti.shared ? p.K_shared : p.K_routed) / BK;
         for (int h = 0; h < ti.halves; ++h) {
           const int sl = (ring.next + h) & 1;
@@ -363,9 +421,12 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
     const int row = q * 32 + lane;
     SlotRing ring;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+    int ns = 0;
+    while (ok) {
+      const int tile = next_tile(ns, ok);
+      if (tile < 0) break;
       TileInfo ti;
-      if (!tile_at(p, mt_begin, tile, BN, ti)) continue;
+      if (!tile_at(p, span, tile, BN, ti)) continue;
       const int n0 = ti.nb * BN;
       for (int h = 0; h < ti.halves; ++h) {
         const int sl = (ring.next + h) & 1;
@@ -452,11 +513,13 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
     const int cw = warp - 6;
     const int sub_row = lane >> 3;          // row within the 4-row step
     const int col16 = lane & 7;             // 16-code column group within the row
-    int kg = 0;
+    int kg = 0, ns = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+    while (ok) {
+      const int tile = next_tile(ns, ok);
+      if (tile < 0) break;
       TileInfo ti;
-      if (!tile_at(p, mt_begin, tile, BN, ti)) continue;
+      if (!tile_at(p, span, tile, BN, ti)) continue;
       const int nk = p.K_routed / BK;
       const int n0 = ti.nb * BN;
       const int ksb = p.K_routed / 128, nsb = p.N_routed / 128;  // scale blocks per expert

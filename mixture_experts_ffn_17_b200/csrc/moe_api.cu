@@ -44,7 +44,7 @@ moe_status validate_shape(const moe_shape* s) {
 }
 
 struct Layout {
-  size_t status, logits, idx, w, hist, base, counts, offsets, perm, row_of, tiles, ntiles, x_perm, H, Y_perm,
+  size_t status, logits, idx, w, hist, base, counts, offsets, perm, row_of, tiles, ntiles, sched, x_perm, H, Y_perm,
       Y_shared, total;
   int nb, max_mtiles, Hld;
   int64_t Hrows;
@@ -76,6 +76,7 @@ Layout make_layout(const moe_shape& s) {
   L.row_of = take((size_t)Tk * 4);
   L.tiles = take((size_t)L.max_mtiles * 16);
   L.ntiles = take(8);
+  L.sched = take(kNumSchedCounters * 4);
   L.x_perm = take((size_t)Tk * s.d * 2);
   L.H = take((size_t)L.Hrows * L.Hld * 2);
   L.Y_perm = take((size_t)Tk * s.d * 2);
@@ -191,7 +192,8 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   int4* tiles = at<int4>(ws, L.tiles);
   int32_t* ntiles = at<int32_t>(ws, L.ntiles);
   uint16_t* H = at<uint16_t>(ws, L.H);
-  MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, sh, tiles, ntiles, st));
+  int* sched = at<int>(ws, L.sched);
+  MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, sh, tiles, ntiles, sched, st));
   if (ev) MOE_CUDA(cudaEventRecord(ev[0], st));
 
   const int sms = num_sms();
@@ -235,6 +237,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   p1.status = status;
   p1.tile_set = kTilesAll;
   p1.debug_withhold_loads = debug_withhold_loads() ? 1 : 0;
+  p1.sched_counter = sched + 0;
   const int grid1 = (int)std::min<int64_t>(sms, (int64_t)L.max_mtiles * p1.n_nb);
   if (f8) {
     GemmParams q = p1;
@@ -245,6 +248,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
     if (sh) {
       q = p1;
       q.tile_set = kTilesShared;
+      q.sched_counter = sched + 1;
       MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, q, grid1, st));
     }
   } else {
@@ -268,6 +272,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
     w2_s = w2_r;
   }
   GemmParams p2 = p1;
+  p2.sched_counter = sched + 2;
   const int bn2 = gemm_block_n_down();
   p2.n_nb = (s.d + bn2 - 1) / bn2;
   p2.K_routed = s.inter;
@@ -289,6 +294,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
     if (sh) {
       q = p2;
       q.tile_set = kTilesShared;
+      q.sched_counter = sched + 3;
       MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, q, grid2, st));
     }
   } else {

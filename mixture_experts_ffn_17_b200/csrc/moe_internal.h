@@ -60,8 +60,10 @@ cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int32_t*
                            uint32_t* status, cudaStream_t stream);
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t rows, int d, void* x_perm,
                                int num_sms, cudaStream_t stream);
+// Also zeroes the grouped GEMMs' tile counters (kNumSchedCounters ints).
+constexpr int kNumSchedCounters = 4;
 cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, bool with_shared, int4* tiles,
-                               int32_t* ntiles, cudaStream_t stream);
+                               int32_t* ntiles, int* sched_counters, cudaStream_t stream);
 
 // grouped_gemm.cu
 // Which part of the tile list a grouped-GEMM launch walks.
@@ -86,6 +88,7 @@ struct GemmParams {
   const float* scale_b;
   const float* scale_c;
   uint32_t* status;
+  int* sched_counter;     // tiles claimed so far (zeroed by the tile-list kernel)
   // Failure-path testing: when nonzero the producer issues no loads, so the
   // MMA issuer's bounded wait runs out and the launch reports a timeout.
   int debug_withhold_loads;

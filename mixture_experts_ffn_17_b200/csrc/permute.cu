@@ -175,7 +175,8 @@ __global__ void __launch_bounds__(256)
 // the shared expert's tiles (group E, rows in token order).  ntiles[0] = all
 // tiles, ntiles[1] = routed tiles.
 __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, int T, int with_shared,
-                                   int4* __restrict__ tiles, int32_t* __restrict__ ntiles) {
+                                   int4* __restrict__ tiles, int32_t* __restrict__ ntiles,
+                                   int* __restrict__ sched_counters) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t total;
   const int e = threadIdx.x;
@@ -222,6 +223,7 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
     ntiles[0] = routed + shared_tiles;
     ntiles[1] = routed;
   }
+  if (threadIdx.x < kNumSchedCounters) sched_counters[threadIdx.x] = 0;
 }
 
 }  // namespace
@@ -257,10 +259,10 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t
 }
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, bool with_shared, int4* tiles,
-                               int32_t* ntiles, cudaStream_t stream) {
+                               int32_t* ntiles, int* sched_counters, cudaStream_t stream) {
   const int threads = ((E + 31) / 32) * 32;
   build_tiles_kernel<<<1, threads < 32 ? 32 : threads, 0, stream>>>(offsets, E, (int)T, with_shared ? 1 : 0,
-                                                                    tiles, ntiles);
+                                                                    tiles, ntiles, sched_counters);
   return cudaGetLastError();
 }
 
