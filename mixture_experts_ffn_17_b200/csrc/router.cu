@@ -11,7 +11,7 @@
 //   warp 0 : TMA producer (x tile [128 x 64] and Wg tile [EB x 64] per stage,
 //            128-byte swizzle, 4-stage ring)
 //   warp 1 : tcgen05.mma issuer, M=128 N=EB K=16, fp32 accumulator in TMEM;
-//            each 64-wide K chunk goes to one of two TMEM buffers
+//            each 64-wide K chunk goes to the next of four TMEM buffers
 //   warps 2-5: drain each finished chunk from TMEM and add it into fp64
 //            registers, so the logit carries one fp32 rounding per 64 terms;
 //            at the end write fp32 logits [T, E].
@@ -30,11 +30,13 @@ constexpr int kRouterBM = 128;
 constexpr int kRouterBK = 64;
 constexpr int kRouterStages = 4;
 
+constexpr int kRouterAccBufs = 4;  // TMEM buffers: the MMA may run this many K chunks ahead of the drain
+
 template <int EB>
 struct RouterSmem {
   static constexpr uint32_t kABytes = kRouterBM * kRouterBK * 2;
   static constexpr uint32_t kBBytes = EB * kRouterBK * 2;
-  static constexpr uint32_t kTmemCols = (2 * EB <= 32) ? 32 : (2 * EB <= 64 ? 64 : (2 * EB <= 128 ? 128 : 256));
+  static constexpr uint32_t kTmemCols = kRouterAccBufs * EB <= 128 ? 128 : 256;
   static constexpr size_t kBytes = 1024 + kRouterStages * (kABytes + kBBytes) + 256;
 };
 
@@ -51,8 +53,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * L::kBBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* done = tempty + 2;
+  uint64_t* tempty = tfull + kRouterAccBufs;
+  uint64_t* done = tempty + kRouterAccBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   __shared__ uint32_t never;  // a flag nobody raises (drain waits)
@@ -68,7 +70,7 @@ __global__ void __launch_bounds__(192, 1)
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kRouterAccBufs; ++b) {
       ptx::mbar_init(&tfull[b], 1);
       ptx::mbar_init(&tempty[b], 128);
     }
@@ -115,8 +117,8 @@ __global__ void __launch_bounds__(192, 1)
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % S;
         const uint32_t ph = (kb / S) & 1;
-        const int b = kb & 1;
-        const uint32_t use = kb >> 1;
+        const int b = kb % kRouterAccBufs;
+        const uint32_t use = kb / kRouterAccBufs;
         if (!ptx::wait_bounded(&tempty[b], (use & 1) ^ 1, abort_flag) ||
             !ptx::wait_bounded(&full[s], ph, abort_flag)) {
           raise_status(status, abort_flag, kStatusTimeout);
@@ -143,8 +145,8 @@ __global__ void __launch_bounds__(192, 1)
     for (int j = 0; j < EB; ++j) acc[j] = 0.0;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
-      const int b = kb & 1;
-      const uint32_t use = kb >> 1;
+      const int b = kb % kRouterAccBufs;
+      const uint32_t use = kb / kRouterAccBufs;
       if (!ptx::wait_bounded(&tfull[b], use & 1, abort_flag)) {
         raise_status(status, abort_flag, kStatusTimeout);
         ok = false;
@@ -152,17 +154,27 @@ __global__ void __launch_bounds__(192, 1)
       }
       ptx::tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + b * EB;
+      if (EB == 64) {
+        // both 32-column halves in flight before one wait
+        uint32_t r0[32], r1[32];
+        ptx::tmem_ld32(taddr, r0);
+        ptx::tmem_ld32(taddr + 32, r1);
+        ptx::tmem_ld_wait2(r0, r1);
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&tempty[b]);
 #pragma unroll
-      for (int c = 0; c < EB / 32; ++c) {
-        uint32_t r[32];
-        ptx::tmem_ld32(taddr + c * 32, r);
-        ptx::tmem_ld_wait(r);
-        if (c == EB / 32 - 1) {
-          ptx::tc_fence_before();
-          ptx::mbar_arrive(&tempty[b]);
+        for (int i = 0; i < 32; ++i) {
+          acc[i] += (double)__uint_as_float(r0[i]);
+          acc[32 + i] += (double)__uint_as_float(r1[i]);
         }
+      } else {
+        uint32_t r[32];
+        ptx::tmem_ld32(taddr, r);
+        ptx::tmem_ld_wait(r);
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&tempty[b]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[c * 32 + i] += (double)__uint_as_float(r[i]);
+        for (int i = 0; i < 32; ++i) acc[i] += (double)__uint_as_float(r[i]);
       }
     }
     if (ok && m0 + row < T) {
