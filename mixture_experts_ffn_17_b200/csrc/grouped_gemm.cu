@@ -274,7 +274,14 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
         ptx::prefetch_tmap(&tmC_r);
         if (!F8) ptx::prefetch_tmap(&tmC_s);
       }
-      const uint64_t pol_a = ptx::policy_evict_last();   // A rows are reused by every column block
+#ifndef MOE_GEMM_A_POLICY
+#define MOE_GEMM_A_POLICY 1
+#endif
+      // A rows are reused by the column blocks of their row tile, which run at
+      // about the same time
+      const uint64_t pol_a = MOE_GEMM_A_POLICY == 0 ? ptx::policy_evict_first()
+                             : MOE_GEMM_A_POLICY == 1 ? ptx::policy_evict_normal()
+                                                      : ptx::policy_evict_last();
       const uint64_t pol_w = ptx::policy_evict_first();  // each weight tile is read once
       const uint64_t pol_ws = ptx::policy_evict_last();  // the shared expert's weights serve every row tile
       int kg = 0, ns = 0;

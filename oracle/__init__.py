@@ -47,8 +47,10 @@ def build(force: bool = False) -> str:
 def lib():
     global _lib
     if _lib is None:
-        build()
-        L = ctypes.CDLL(_LIB)
+        # ORACLE_LIB: load another build of moe_oracle.c instead (the mutation
+        # test points it at deliberately broken copies to show the pins fail)
+        path = os.environ.get("ORACLE_LIB") or build()
+        L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         i64, i32, f64 = ctypes.c_int64, ctypes.c_int, ctypes.c_double
         sig = {
