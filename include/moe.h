@@ -105,6 +105,26 @@ moe_status moe_router_topk(const moe_shape* shape, const void* x, const void* Wg
                            int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t ws_bytes,
                            void* stream);
 
+/* Device-limited routing (n4n page, "Why 256 experts with top-8 routing?",
+ * device-limited routing code): experts with allowed[e] == 0 (those not held
+ * by this device) get -inf added to their logit before the top-k; then the
+ * top-k / softmax rule of moe_router_topk.  allowed [E] uint8 device array.
+ * Top-k/softmax mode only (MOE_ERR_UNSUPPORTED otherwise).  With fewer than k
+ * allowed experts the remaining slots hold the lowest-index masked experts
+ * with weight 0. */
+moe_status moe_router_topk_limited(const moe_shape* shape, const void* x, const void* Wg, const uint8_t* allowed,
+                                   int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/* Expert-utilisation monitor (n4n page, "Where the architecture struggles",
+ * log_expert_utilization): from per-expert counts [E] (moe_permute,
+ * moe_forward's counts_out) computes utilisation[e] = counts[e] / sum(counts)
+ * (fp32) and flags[e] = +1 when counts[e] > 2x the mean count, -1 when below
+ * 0.1x the mean, else 0 (decided exactly: counts*E > 2*total,
+ * 10*counts*E < total).  Either output may be NULL (not both). */
+moe_status moe_expert_utilisation(const moe_shape* shape, const int32_t* counts, float* utilisation, int32_t* flags,
+                                  void* stream);
+
 /* Dispatch: counts = bincount(topk_idx, minlength=E); offsets = exclusive
  * prefix sum (E+1 entries); the permuted order lists experts ascending and,
  * within an expert, its (token, slot) entries ascending -- the order of the

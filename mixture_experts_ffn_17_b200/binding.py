@@ -23,7 +23,7 @@ MOE_ROUTE_TOPK_SOFTMAX, MOE_ROUTE_SIGMOID_GROUP = 0, 1
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
             "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version",
-            "moe_permute_noalloc")
+            "moe_permute_noalloc", "moe_router_topk_limited", "moe_expert_utilisation")
 NUM_STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "experts_up", "experts_down", "combine")
 
@@ -69,6 +69,10 @@ def lib() -> ctypes.CDLL:
         L.moe_router_topk.argtypes = [S, P, P, P, P, P, P, P, sz, P]
         L.moe_permute.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
         L.moe_permute_noalloc.argtypes = [S, P, P, P, P, P, P, P, P]
+        L.moe_router_topk_limited.argtypes = [S, P, P, P, P, P, P, P, sz, P]
+        L.moe_router_topk_limited.restype = ctypes.c_int
+        L.moe_expert_utilisation.argtypes = [S, P, P, P, P]
+        L.moe_expert_utilisation.restype = ctypes.c_int
         L.moe_permute_noalloc.restype = ctypes.c_int
         L.moe_grouped_swiglu.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_combine.argtypes = [S, P, P, P, P, P, P]
@@ -124,6 +128,17 @@ def router_topk(shape, x, Wg, bias, topk_idx, topk_w, logits, ws, stream=None):
     _check(lib().moe_router_topk(ctypes.byref(shape), _ptr(x), _ptr(Wg), _ptr(bias), _ptr(topk_idx), _ptr(topk_w),
                                  _ptr(logits), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
            "moe_router_topk")
+
+
+def router_topk_limited(shape, x, Wg, allowed, topk_idx, topk_w, logits, ws, stream=None):
+    _check(lib().moe_router_topk_limited(ctypes.byref(shape), _ptr(x), _ptr(Wg), _ptr(allowed), _ptr(topk_idx),
+                                         _ptr(topk_w), _ptr(logits), _ptr(ws), ws.numel() if ws is not None else 0,
+                                         _stream(stream)), "moe_router_topk_limited")
+
+
+def expert_utilisation(shape, counts, utilisation, flags, stream=None):
+    _check(lib().moe_expert_utilisation(ctypes.byref(shape), _ptr(counts), _ptr(utilisation), _ptr(flags),
+                                        _stream(stream)), "moe_expert_utilisation")
 
 
 def permute(shape, topk_idx, counts, offsets, perm_token, row_of, x, x_perm, ws, stream=None):

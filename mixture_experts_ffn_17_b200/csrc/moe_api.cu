@@ -170,14 +170,14 @@ int num_sms() {
 
 // ------------------------------------------------------------ stages
 moe_status run_router(const moe_shape& s, const void* x, const void* Wg, const float* bias, int32_t* idx, float* w,
-                      float* logits, uint32_t* status, cudaStream_t st) {
+                      float* logits, uint32_t* status, cudaStream_t st, const uint8_t* allowed = nullptr) {
   CUtensorMap tm_x, tm_wg;
   const int eb = router_expert_block(s.E);
   if (!map_2d(&tm_x, x, s.d, s.T, 64, 128) || !map_2d(&tm_wg, Wg, s.d, s.E, 64, eb)) return MOE_ERR_CUDA;
   MOE_CUDA(launch_router_logits(tm_x, tm_wg, (int)s.T, s.d, s.E, logits, status, st));
   RouteParams rp{s.route, s.n_group, s.topk_group, s.group_topn, s.route_scale};
-  MOE_CUDA(launch_router_topk(logits, s.route == MOE_ROUTE_SIGMOID_GROUP ? bias : nullptr, rp, (int)s.T, s.E, s.k,
-                              idx, w, st));
+  MOE_CUDA(launch_router_topk(logits, s.route == MOE_ROUTE_SIGMOID_GROUP ? bias : nullptr, allowed, rp, (int)s.T, s.E,
+                              s.k, idx, w, st));
   return MOE_OK;
 }
 
@@ -384,6 +384,36 @@ moe_status moe_router_topk(const moe_shape* shape, const void* x, const void* Wg
   uint32_t* status = at<uint32_t>(ws, L.status);
   MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
   return run_router(s, x, Wg, bias, topk_idx, topk_w, logits ? logits : at<float>(ws, L.logits), status, st);
+}
+
+moe_status moe_router_topk_limited(const moe_shape* shape, const void* x, const void* Wg, const uint8_t* allowed,
+                                   int32_t* topk_idx, float* topk_w, float* logits, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  if (s.route != MOE_ROUTE_TOPK_SOFTMAX) return MOE_ERR_UNSUPPORTED;
+  if (!x || !Wg || !allowed || !topk_idx || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(Wg) || !aligned16(topk_idx) || !aligned16(topk_w) ||
+      (logits && !aligned16(logits)))
+    return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(s);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  if (s.T == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
+  return run_router(s, x, Wg, nullptr, topk_idx, topk_w, logits ? logits : at<float>(ws, L.logits), status, st,
+                    allowed);
+}
+
+moe_status moe_expert_utilisation(const moe_shape* shape, const int32_t* counts, float* utilisation, int32_t* flags,
+                                  void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  if (!counts || (!utilisation && !flags)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(launch_expert_utilisation(counts, shape->E, utilisation, flags, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
 }
 
 moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,

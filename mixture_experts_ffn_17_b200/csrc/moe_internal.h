@@ -50,8 +50,12 @@ struct RouteParams {
 int router_expert_block(int E);
 cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E,
                                  float* logits, uint32_t* status, cudaStream_t stream);
-cudaError_t launch_router_topk(const float* logits, const float* bias, const RouteParams& rp, int T, int E, int k,
-                               int32_t* idx, float* w, cudaStream_t stream);
+cudaError_t launch_router_topk(const float* logits, const float* bias, const uint8_t* allowed, const RouteParams& rp,
+                               int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream);
+
+// monitor.cu
+cudaError_t launch_expert_utilisation(const int32_t* counts, int E, float* util, int32_t* flags,
+                                      cudaStream_t stream);
 
 // permute.cu
 int permute_blocks(int64_t T);

@@ -216,9 +216,10 @@ __device__ __forceinline__ Cand warp_best(Cand c) {
 // NV = values per lane (expert e lives in lane e % 32, slot e / 32).
 template <int NV>
 __global__ void __launch_bounds__(128)
-    router_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T, int E, int k,
-                       int route, int n_group, int topk_group, int group_topn, float route_scale,
-                       int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    router_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
+                       const uint8_t* __restrict__ allowed, int T, int E, int k, int route, int n_group,
+                       int topk_group, int group_topn, float route_scale, int32_t* __restrict__ topk_idx,
+                       float* __restrict__ topk_w) {
   __shared__ float sel_sh[4][NV * 32];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -233,7 +234,8 @@ __global__ void __launch_bounds__(128)
   for (int v = 0; v < NV; ++v) {
     const int e = v * 32 + lane;
     if (e < E) {
-      const float l = lrow[e];
+      // device-limited routing: experts this device does not hold get -inf
+      const float l = (allowed && !allowed[e]) ? NEG : lrow[e];
       if (route == 0) {
         key[v] = l;
         aux[v] = l;
@@ -339,9 +341,9 @@ cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_
 }
 
 template <int NV>
-cudaError_t launch_topk_nv(const float* logits, const float* bias, const RouteParams& rp, int T, int E, int k,
-                           int32_t* idx, float* w, cudaStream_t stream) {
-  router_topk_kernel<NV><<<(T + 3) / 4, 128, 0, stream>>>(logits, bias, T, E, k, rp.route, rp.n_group,
+cudaError_t launch_topk_nv(const float* logits, const float* bias, const uint8_t* allowed, const RouteParams& rp,
+                           int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream) {
+  router_topk_kernel<NV><<<(T + 3) / 4, 128, 0, stream>>>(logits, bias, allowed, T, E, k, rp.route, rp.n_group,
                                                           rp.topk_group, rp.group_topn, rp.route_scale, idx, w);
   return cudaGetLastError();
 }
@@ -363,15 +365,15 @@ cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_
   }
 }
 
-cudaError_t launch_router_topk(const float* logits, const float* bias, const RouteParams& rp, int T, int E, int k,
-                               int32_t* idx, float* w, cudaStream_t stream) {
+cudaError_t launch_router_topk(const float* logits, const float* bias, const uint8_t* allowed, const RouteParams& rp,
+                               int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream) {
   const int nv = (E + 31) / 32;
-  if (nv <= 1) return launch_topk_nv<1>(logits, bias, rp, T, E, k, idx, w, stream);
-  if (nv <= 2) return launch_topk_nv<2>(logits, bias, rp, T, E, k, idx, w, stream);
-  if (nv <= 4) return launch_topk_nv<4>(logits, bias, rp, T, E, k, idx, w, stream);
-  if (nv <= 8) return launch_topk_nv<8>(logits, bias, rp, T, E, k, idx, w, stream);
-  if (nv <= 16) return launch_topk_nv<16>(logits, bias, rp, T, E, k, idx, w, stream);
-  if (nv <= 32) return launch_topk_nv<32>(logits, bias, rp, T, E, k, idx, w, stream);
+  if (nv <= 1) return launch_topk_nv<1>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
+  if (nv <= 2) return launch_topk_nv<2>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
+  if (nv <= 4) return launch_topk_nv<4>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
+  if (nv <= 8) return launch_topk_nv<8>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
+  if (nv <= 16) return launch_topk_nv<16>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
+  if (nv <= 32) return launch_topk_nv<32>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
   return cudaErrorInvalidValue;
 }
 

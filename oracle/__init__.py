@@ -65,6 +65,8 @@ def lib():
             "oracle_dispatch": [i64, i32, i32, P, P, P, P, P],
             "oracle_swiglu_rows": [i64, i64, i64, P, P, P, P, P],
             "oracle_combine": [i64, i32, i64, P, P, P, P, P],
+            "oracle_route_topk_softmax_limited": [i64, i32, i32, P, P, P, P, P],
+            "oracle_expert_utilisation": [i32, P, P, P],
             "oracle_moe_forward": [i64, i64, i32, i32, i64, i64, i32, i32, i32, i32, f64,
                                    P, P, P, P, P, P, P, P, P, P, P, P, P, P],
         }
@@ -151,6 +153,29 @@ def route_topk_softmax(lg: np.ndarray, k: int):
     gaps = np.empty((T, k), dtype=np.float64)
     lib().oracle_route_topk_softmax(T, E, k, _p(lg), _p(idx), _p(w), _p(gaps))
     return idx, w, gaps
+
+
+def route_topk_softmax_limited(lg: np.ndarray, allowed: np.ndarray, k: int):
+    """Device-limited page-1 routing: experts with allowed[e] == 0 are masked
+    to -inf before the top-k.  -> idx, w, gaps as route_topk_softmax."""
+    lg = _c(lg, np.float64)
+    al = _c(allowed, np.uint8)
+    T, E = lg.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    gaps = np.empty((T, k), dtype=np.float64)
+    lib().oracle_route_topk_softmax_limited(T, E, k, _p(lg), _p(al), _p(idx), _p(w), _p(gaps))
+    return idx, w, gaps
+
+
+def expert_utilisation(counts: np.ndarray):
+    """-> utilisation [E] fp64 (counts / total), flags [E] int32 (+1 > 2x mean, -1 < 0.1x mean)."""
+    c = _c(counts, np.int32)
+    E = c.shape[0]
+    util = np.empty(E, dtype=np.float64)
+    flag = np.empty(E, dtype=np.int32)
+    lib().oracle_expert_utilisation(E, _p(c), _p(util), _p(flag))
+    return util, flag
 
 
 def route_sigmoid_group(lg: np.ndarray, bias, k: int, n_group: int, topk_group: int,

@@ -428,3 +428,39 @@ ORACLE_EXPORT void oracle_combine(int64_t T, int k, int64_t d, const double *Yp,
             for (int64_t c = 0; c < d; ++c) yt[c] += Ys[t * d + c];
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Device-limited routing (n4n page, "Why 256 experts with top-8 routing?",   */
+/* device-limited routing code): experts not on this device get a -inf mask   */
+/* added to their logits before the top-k; then the page-1 rule.  allowed[e] */
+/* is nonzero for the experts this device holds.                              */
+/* ------------------------------------------------------------------------ */
+ORACLE_EXPORT void oracle_route_topk_softmax_limited(int64_t T, int E, int k, const double *logits,
+                                                     const uint8_t *allowed, int32_t *idx, double *w, double *gaps)
+{
+    double *masked = (double *)malloc(sizeof(double) * T * E);
+    for (int64_t t = 0; t < T; ++t)
+        for (int e = 0; e < E; ++e)
+            masked[t * E + e] = allowed[e] ? logits[t * E + e] : -INFINITY;
+    oracle_route_topk_softmax(T, E, k, masked, idx, w, gaps);
+    free(masked);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Expert-utilisation monitor (n4n page, "Where the architecture struggles",  */
+/* log_expert_utilization): utilisation = counts / sum(counts); an expert is  */
+/* flagged +1 when its count exceeds 2x the mean count, -1 when it is below   */
+/* 0.1x the mean, 0 otherwise.  With mean = total / E the two tests are the   */
+/* integer comparisons count*E > 2*total and 10*count*E < total, decided      */
+/* exactly.                                                                   */
+/* ------------------------------------------------------------------------ */
+ORACLE_EXPORT void oracle_expert_utilisation(int E, const int32_t *counts, double *util, int32_t *flag)
+{
+    int64_t total = 0;
+    for (int e = 0; e < E; ++e) total += counts[e];
+    for (int e = 0; e < E; ++e) {
+        int64_t c = counts[e];
+        util[e] = total > 0 ? (double)c / (double)total : 0.0;
+        flag[e] = (c * E > 2 * total) ? 1 : ((10 * c * E < total) ? -1 : 0);
+    }
+}

@@ -293,3 +293,82 @@ def test_forward_fp8_group_routing():
 
 def test_forward_fp8_no_shared_expert():
     _check_forward(_fp8(T=300, shared_inter=0), tol=TOL_FP8)
+
+
+# --------------------------------------------------- device-limited routing
+def test_router_limited_matches_oracle():
+    w = _medium()
+    cfg = w.cfg
+    rng = np.random.default_rng(21)
+    allowed = (rng.random(cfg.E) < 0.4).astype(np.uint8)
+    allowed[:cfg.k] = 1
+    shape = B.shape_of(cfg)
+    ws = B.alloc_workspace(shape)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    B.router_topk_limited(shape, w.x, w.Wg, torch.as_tensor(allowed, device="cuda"), idx, tw, None, ws)
+    torch.cuda.synchronize()
+    lg = oracle.logits(dec(w.x), dec(w.Wg))
+    idx_o, w_o, gaps = oracle.route_topk_softmax_limited(lg, allowed, cfg.k)
+    masked = np.where(allowed[None, :] > 0, lg, -np.inf)
+    from parity import compare_indices
+    n_ex, report = compare_indices(to_np(idx), idx_o, masked, gaps, None, cfg.E)
+    assert all(allowed[e] for e in to_np(idx).ravel())
+    ok = np.all(to_np(idx) == idx_o, axis=1)
+    assert np.allclose(to_np(tw)[ok], w_o[ok], rtol=0, atol=2e-6)
+
+
+def test_router_limited_fewer_allowed_than_k():
+    w = _tiny()
+    cfg = w.cfg
+    allowed = np.zeros(cfg.E, dtype=np.uint8)
+    allowed[[3, 17]] = 1                     # 2 allowed experts, k = 4
+    shape = B.shape_of(cfg)
+    ws = B.alloc_workspace(shape)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    tw = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    B.router_topk_limited(shape, w.x, w.Wg, torch.as_tensor(allowed, device="cuda"), idx, tw, None, ws)
+    torch.cuda.synchronize()
+    lg = oracle.logits(dec(w.x), dec(w.Wg))
+    idx_o, w_o, _ = oracle.route_topk_softmax_limited(lg, allowed, cfg.k)
+    assert np.array_equal(to_np(idx), idx_o)
+    assert np.allclose(to_np(tw), w_o, rtol=0, atol=2e-6)
+    assert np.all(to_np(tw)[:, 2:] == 0)
+
+
+# ------------------------------------------------------ utilisation monitor
+@pytest.mark.parametrize("kind", ["random", "crafted", "zero", "skewed"])
+def test_expert_utilisation_matches_oracle(kind):
+    E = 256
+    rng = np.random.default_rng(22)
+    if kind == "random":
+        counts = rng.integers(0, 300, size=E)
+    elif kind == "crafted":   # exactly on the thresholds: mean 10 -> hot above 20, cold below 1
+        counts = np.full(E, 10); counts[:4] = [20, 21, 1, 0]; counts[4] = 10 + (20 - 21 - 1 - 0 + 10 * 4 - 40)
+    elif kind == "zero":
+        counts = np.zeros(E)
+    else:
+        counts = (1e5 / np.arange(1, E + 1) ** 1.1).astype(np.int64)
+    counts = counts.astype(np.int32)
+    cfg = workloads.CONFIGS["prefill"]
+    shape = B.shape_of(cfg)
+    c = torch.as_tensor(counts, device="cuda")
+    util = torch.empty(E, dtype=torch.float32, device="cuda")
+    flags = torch.empty(E, dtype=torch.int32, device="cuda")
+    B.expert_utilisation(shape, c, util, flags)
+    torch.cuda.synchronize()
+    u_o, f_o = oracle.expert_utilisation(counts)
+    assert np.array_equal(to_np(flags), f_o)
+    assert np.allclose(to_np(util).astype(np.float64), u_o, rtol=1e-6, atol=1e-9)
+
+
+def test_expert_utilisation_of_a_forward_pass():
+    w = _medium()
+    y, idx, tw, counts, ws = run_forward(w)
+    shape = B.shape_of(w.cfg)
+    util = torch.empty(w.cfg.E, dtype=torch.float32, device="cuda")
+    B.expert_utilisation(shape, counts, util, None)
+    torch.cuda.synchronize()
+    c, _, _, _ = oracle.dispatch(to_np(idx), w.cfg.E)
+    u_o, _ = oracle.expert_utilisation(c)
+    assert np.allclose(to_np(util), u_o, rtol=1e-6) and abs(float(util.sum()) - 1.0) < 1e-5

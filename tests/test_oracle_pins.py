@@ -405,3 +405,43 @@ def test_combine_special_cases():
     # skipped rows (row_of < 0) contribute nothing
     row_of3 = row_of.copy(); row_of3[:, 1:] = -1
     assert np.array_equal(oracle.combine(Yp, None, row_of3, np.ones((T, k))), Yp[::k])
+
+
+# ------------------------------------------------- device-limited routing
+def test_device_limited_routing_brute_force_and_special_cases():
+    rng = np.random.default_rng(19)
+    E, k = 10, 3
+    lg = rng.standard_normal((30, E))
+    allowed = np.zeros(E, dtype=np.uint8)
+    allowed[[1, 2, 5, 7, 8]] = 1
+    idx, w, _ = oracle.route_topk_softmax_limited(lg, allowed, k)
+    for t in range(30):
+        cand = [e for e in range(E) if allowed[e]]
+        sub = _brute_topk([lg[t, e] for e in cand], k)
+        assert idx[t].tolist() == [cand[i] for i in sub]
+        assert all(allowed[e] for e in idx[t])
+    assert np.allclose(w.sum(1), 1.0, atol=1e-12)
+    # everything allowed == page-1 routing
+    i1, w1, _ = oracle.route_topk_softmax_limited(lg, np.ones(E, dtype=np.uint8), k)
+    i0, w0, _ = oracle.route_topk_softmax(lg, k)
+    assert np.array_equal(i0, i1) and np.array_equal(w0, w1)
+    # exactly k allowed: those k, in descending logit order
+    al = np.zeros(E, dtype=np.uint8); al[[0, 4, 9]] = 1
+    idx, _, _ = oracle.route_topk_softmax_limited(lg, al, 3)
+    for t in range(30):
+        assert sorted(idx[t].tolist()) == [0, 4, 9]
+        assert list(np.diff(lg[t, idx[t]]) <= 0) == [True, True]
+
+
+# ------------------------------------------------- utilisation monitor
+def test_expert_utilisation_definition_cases():
+    counts = np.array([0, 1, 10, 10, 10, 10, 39, 0], dtype=np.int32)   # total 80, mean 10
+    util, flag = oracle.expert_utilisation(counts)
+    assert np.allclose(util, counts / 80.0, rtol=0, atol=0)
+    # > 2x mean (20): expert 6; < 0.1x mean (1): experts 0 and 7 (1 is not below 1)
+    assert flag.tolist() == [-1, 0, 0, 0, 0, 0, 1, -1]
+    u0, f0 = oracle.expert_utilisation(np.zeros(4, dtype=np.int32))
+    assert np.all(u0 == 0) and np.all(f0 == 0)
+    # uniform load: nothing flagged, utilisation 1/E
+    u, f = oracle.expert_utilisation(np.full(16, 7, dtype=np.int32))
+    assert np.allclose(u, 1 / 16) and np.all(f == 0)
