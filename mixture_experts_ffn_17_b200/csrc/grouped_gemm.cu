@@ -22,8 +22,10 @@
 //             fp32 accumulators in TMEM: two 256-column slots handed out
 //             round-robin (a one-half tile takes one, a two-half tile both),
 //             so one-half tiles overlap their epilogue with the next main loop;
-//   warps 2-5 epilogue: tcgen05.ld the accumulator rows (one row per
-//             thread), apply silu(g)*u (SwiGLU kernel) and store;
+//   warps 2-9 epilogue (2-5 with FP8 weights): tcgen05.ld the accumulator
+//             rows (one row per thread, two warps per TMEM lane quarter each
+//             taking half of the columns), apply silu(g)*u (SwiGLU kernel)
+//             and store;
 //   warps 6-13 (FP8 weights only) converters: the producer brings raw e4m3
 //             weight tiles [64 K x 128 N] into the stage; these warps turn
 //             them into bf16 (code * the tile's 128 x 128 block scale) in the
@@ -177,8 +179,20 @@ __device__ __forceinline__ uint2 e4m3x4_to_bf16x4(uint32_t q, float scale) {
   return make_uint2(ptx::pack_bf16x2(a0 * scale, a1 * scale), ptx::pack_bf16x2(b0 * scale, b1 * scale));
 }
 
+// Epilogue warps: two per TMEM lane quarter with bf16 weights (each drains
+// half of the columns), one per quarter with FP8 weights (whose converter
+// warps take the rest of the thread budget).
+template <bool F8>
+constexpr int epi_warps() {
+  return F8 ? 4 : 8;
+}
+template <bool F8>
+constexpr int kernel_threads() {
+  return 64 + 32 * epi_warps<F8>() + (F8 ? 32 * kConvWarps : 0);
+}
+
 template <Mode M, bool F8>
-__global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
+__global__ void __launch_bounds__(kernel_threads<F8>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
                         const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
                         const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s,
@@ -219,7 +233,7 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
     }
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&tfull[b], 1);
-      ptx::mbar_init(&tempty[b], 128);
+      ptx::mbar_init(&tempty[b], 32 * epi_warps<F8>());
     }
     for (int c = 0; c < CS; ++c) {
       ptx::mbar_init(&cfull[c], kConvWarps * 32);
@@ -227,7 +241,7 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
     }
     for (int i = 0; i < kSchedDepth; ++i) {
       ptx::mbar_init(&sfull[i], 1);
-      ptx::mbar_init(&sempty[i], 1 + 128 + (F8 ? kConvWarps * 32 : 0));
+      ptx::mbar_init(&sempty[i], 1 + 32 * epi_warps<F8>() + (F8 ? kConvWarps * 32 : 0));
     }
     ptx::mbar_init(done, 1);
     *abort_flag = 0u;
@@ -423,8 +437,11 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
       ptx::mma_commit(done);
       if (!ptx::wait_bounded(done, 0, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
     }
-  } else if (warp < 6) {
-    const int q = warp & 3;
+  } else if (warp < 2 + epi_warps<F8>()) {
+    constexpr int kParts = epi_warps<F8>() / 4;           // column parts per lane quarter
+    constexpr int kChunks = BN / 32 / kParts;             // 32-column chunks per part
+    const int q = warp & 3;                               // TMEM lane quarter this warp may access
+    const int part = (warp - 2) / 4;
     const int row = q * 32 + lane;
     SlotRing ring;
     bool ok = true;
@@ -451,12 +468,13 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
           uint16_t* base = static_cast<uint16_t*>(ti.shared ? p.out_shared : p.out_routed);
           uint4* out = reinterpret_cast<uint4*>(base + hrow * p.ld_out + n0);
 #pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
+          for (int cc = 0; cc < kChunks; ++cc) {
+            const int c = part * kChunks + cc;
             uint32_t g[32], u[32];
             ptx::tmem_ld32(tbase + c * 32, g);
             ptx::tmem_ld32(tbase + 128 + c * 32, u);
             ptx::tmem_ld_wait2(g, u);
-            if (c == BN / 32 - 1) {
+            if (cc == kChunks - 1) {
               ptx::tc_fence_before();
               ptx::mbar_arrive(&tempty[sl]);
             }
@@ -479,25 +497,30 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
           const int64_t orow = (int64_t)ti.row0 + r + (ti.shared ? p.out_shared_row_offset : 0);
           const int N = ti.shared ? p.N_shared : p.N_routed;
 #pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
-            uint32_t v32[32];
-            ptx::tmem_ld32(tbase + c * 32, v32);
-            ptx::tmem_ld_wait(v32);
-            if (c == BN / 32 - 1) {
+          for (int cc = 0; cc < kChunks; cc += 2) {
+            // two 32-column chunks in flight before one wait
+            const int c = part * kChunks + cc;
+            uint32_t va[32], vb[32];
+            ptx::tmem_ld32(tbase + c * 32, va);
+            ptx::tmem_ld32(tbase + (c + 1) * 32, vb);
+            ptx::tmem_ld_wait2(va, vb);
+            if (cc + 2 >= kChunks) {
               ptx::tc_fence_before();
               ptx::mbar_arrive(&tempty[sl]);
             }
-            if (valid && n0 + c * 32 < N) {
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+              const uint32_t* v32 = z ? vb : va;
+              const int col = n0 + (c + z) * 32;
+              if (!valid || col >= N) continue;
               if (ti.shared) {
-                float4* out =
-                    reinterpret_cast<float4*>(static_cast<float*>(p.out_shared) + orow * p.ld_out + n0 + c * 32);
+                float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.out_shared) + orow * p.ld_out + col);
 #pragma unroll
                 for (int v = 0; v < 8; ++v)
                   out[v] = make_float4(__uint_as_float(v32[4 * v]), __uint_as_float(v32[4 * v + 1]),
                                        __uint_as_float(v32[4 * v + 2]), __uint_as_float(v32[4 * v + 3]));
               } else {
-                uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out_routed) + orow * p.ld_out + n0 +
-                                                      c * 32);
+                uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out_routed) + orow * p.ld_out + col);
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
                   out[v] = make_uint4(
@@ -517,7 +540,7 @@ __global__ void __launch_bounds__(F8 ? 192 + 32 * kConvWarps : 192, 1)
     // converters: kConvWarps warps.  A raw stage is 2 boxes x 64 K rows of 128
     // codes = 128 rows; a warp step covers 4 rows, a lane 16 codes (one
     // 16-byte load, two 16-byte stores of bf16).
-    const int cw = warp - 6;
+    const int cw = warp - 2 - epi_warps<F8>();
     const int sub_row = lane >> 3;          // row within the 4-row step
     const int col16 = lane & 7;             // 16-code column group within the row
     int kg = 0, ns = 0;
@@ -590,7 +613,7 @@ cudaError_t launch(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtenso
       cudaFuncSetAttribute(grouped_gemm_kernel<M, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   if (grid <= 0) return cudaSuccess;
-  grouped_gemm_kernel<M, F8><<<grid, F8 ? 192 + 32 * kConvWarps : 192, smem, stream>>>(a_r, a_s, b_r, b_s, c_r, c_s, p);
+  grouped_gemm_kernel<M, F8><<<grid, kernel_threads<F8>(), smem, stream>>>(a_r, a_s, b_r, b_s, c_r, c_s, p);
   return cudaGetLastError();
 }
 

@@ -28,7 +28,10 @@ namespace {
 
 constexpr int kRouterBM = 128;
 constexpr int kRouterBK = 64;
-constexpr int kRouterStages = 4;
+#ifndef MOE_ROUTER_STAGES
+#define MOE_ROUTER_STAGES 4
+#endif
+constexpr int kRouterStages = MOE_ROUTER_STAGES;
 
 constexpr int kRouterAccBufs = 4;  // TMEM buffers: the MMA may run this many K chunks ahead of the drain
 
