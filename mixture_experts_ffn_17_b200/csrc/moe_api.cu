@@ -44,7 +44,7 @@ moe_status validate_shape(const moe_shape* s) {
 }
 
 struct Layout {
-  size_t status, logits, idx, w, hist, base, counts, offsets, perm, row_of, tiles, ntiles, sched, x_perm, H, Y_perm,
+  size_t status, logits, rpart, idx, w, hist, base, counts, offsets, perm, row_of, tiles, ntiles, sched, x_perm, H, Y_perm,
       Y_shared, total;
   int nb, max_mtiles, Hld;
   int64_t Hrows;
@@ -66,6 +66,8 @@ Layout make_layout(const moe_shape& s) {
   };
   L.status = take(64);
   L.logits = take((size_t)T * s.E * 4);
+  const int rsplits = router_splits(T, s.d, s.E, kRouterMaxSms);
+  L.rpart = take(rsplits > 1 ? (size_t)rsplits * T * s.E * 8 : 0);
   L.idx = take((size_t)Tk * 4);
   L.w = take((size_t)Tk * 4);
   L.hist = take((size_t)L.nb * s.E * 4);
@@ -170,14 +172,17 @@ int num_sms() {
 
 // ------------------------------------------------------------ stages
 moe_status run_router(const moe_shape& s, const void* x, const void* Wg, const float* bias, int32_t* idx, float* w,
-                      float* logits, uint32_t* status, cudaStream_t st, const uint8_t* allowed = nullptr) {
+                      float* logits, double* part, uint32_t* status, cudaStream_t st,
+                      const uint8_t* allowed = nullptr) {
   CUtensorMap tm_x, tm_wg;
   const int eb = router_expert_block(s.E);
   if (!map_2d(&tm_x, x, s.d, s.T, 64, 128) || !map_2d(&tm_wg, Wg, s.d, s.E, 64, eb)) return MOE_ERR_CUDA;
-  MOE_CUDA(launch_router_logits(tm_x, tm_wg, (int)s.T, s.d, s.E, logits, status, st));
+  // small batches split the gate GEMM's K so that the grid covers the device
+  const int splits = router_splits(s.T, s.d, s.E, std::min(num_sms(), kRouterMaxSms));
+  MOE_CUDA(launch_router_logits(tm_x, tm_wg, (int)s.T, s.d, s.E, splits, logits, part, status, st));
   RouteParams rp{s.route, s.n_group, s.topk_group, s.group_topn, s.route_scale};
-  MOE_CUDA(launch_router_topk(logits, s.route == MOE_ROUTE_SIGMOID_GROUP ? bias : nullptr, allowed, rp, (int)s.T, s.E,
-                              s.k, idx, w, st));
+  MOE_CUDA(launch_router_topk(logits, part, splits, s.route == MOE_ROUTE_SIGMOID_GROUP ? bias : nullptr, allowed, rp,
+                              (int)s.T, s.E, s.k, idx, w, st));
   return MOE_OK;
 }
 
@@ -341,7 +346,7 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   void* Y_perm = at<void>(ws, L.Y_perm);
   float* Y_shared = sh ? at<float>(ws, L.Y_shared) : nullptr;
 
-  moe_status r = run_router(s, x, Wg, bias, idx, w, at<float>(ws, L.logits), status, st);
+  moe_status r = run_router(s, x, Wg, bias, idx, w, at<float>(ws, L.logits), at<double>(ws, L.rpart), status, st);
   if (r != MOE_OK) return r;
   if (ev) MOE_CUDA(cudaEventRecord(ev[1], st));
   MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
@@ -383,7 +388,8 @@ moe_status moe_router_topk(const moe_shape* shape, const void* x, const void* Wg
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t* status = at<uint32_t>(ws, L.status);
   MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
-  return run_router(s, x, Wg, bias, topk_idx, topk_w, logits ? logits : at<float>(ws, L.logits), status, st);
+  return run_router(s, x, Wg, bias, topk_idx, topk_w, logits ? logits : at<float>(ws, L.logits),
+                    at<double>(ws, L.rpart), status, st);
 }
 
 moe_status moe_router_topk_limited(const moe_shape* shape, const void* x, const void* Wg, const uint8_t* allowed,
@@ -403,8 +409,8 @@ moe_status moe_router_topk_limited(const moe_shape* shape, const void* x, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t* status = at<uint32_t>(ws, L.status);
   MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
-  return run_router(s, x, Wg, nullptr, topk_idx, topk_w, logits ? logits : at<float>(ws, L.logits), status, st,
-                    allowed);
+  return run_router(s, x, Wg, nullptr, topk_idx, topk_w, logits ? logits : at<float>(ws, L.logits),
+                    at<double>(ws, L.rpart), status, st, allowed);
 }
 
 moe_status moe_expert_utilisation(const moe_shape* shape, const int32_t* counts, float* utilisation, int32_t* flags,

@@ -48,10 +48,20 @@ struct RouteParams {
 
 // router.cu
 int router_expert_block(int E);
-cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E,
-                                 float* logits, uint32_t* status, cudaStream_t stream);
-cudaError_t launch_router_topk(const float* logits, const float* bias, const uint8_t* allowed, const RouteParams& rp,
-                               int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream);
+// Number of K splits of the gate GEMM on a device with `sms` SMs (1 when the
+// (128-token, expert-block) tiles alone fill half the device); non-decreasing
+// in sms.  Split partial sums are fp64 [splits, T, E].
+int router_splits(int64_t T, int d, int E, int sms);
+constexpr int kRouterMaxSms = 256;  // workspace is sized for router_splits(.., kRouterMaxSms)
+// splits == 1: fp32 logits written directly; splits > 1: fp64 partials to
+// `part`, summed in split order by the top-k launch.
+cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E, int splits,
+                                 float* logits, double* part, uint32_t* status, cudaStream_t stream);
+// part != nullptr: logits[t][e] = (float) sum_s part[s][t][e] is computed
+// (and stored to `logits`) before the selection; otherwise logits are read.
+cudaError_t launch_router_topk(float* logits, const double* part, int splits, const float* bias,
+                               const uint8_t* allowed, const RouteParams& rp, int T, int E, int k, int32_t* idx,
+                               float* w, cudaStream_t stream);
 
 // monitor.cu
 cudaError_t launch_expert_utilisation(const int32_t* counts, int E, float* util, int32_t* flags,

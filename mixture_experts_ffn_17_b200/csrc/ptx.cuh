@@ -203,6 +203,19 @@ __device__ __forceinline__ void tmem_ld_wait2(uint32_t (&r)[32], uint32_t (&q)[3
                "+r"(q[28]), "+r"(q[29]), "+r"(q[30]), "+r"(q[31])::"memory");
 }
 
+// 16 consecutive fp32 columns (32x32b.x16) and its wait.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : MOE_R8(0), MOE_R8(8)
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : MOE_W8(0), MOE_W8(8)::"memory");
+}
+
 #undef MOE_R8
 #undef MOE_W8
 

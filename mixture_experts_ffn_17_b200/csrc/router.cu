@@ -7,14 +7,19 @@
 // 8 contiguous groups, group score = sum of the group's top-2, keep the top-4
 // groups, top-k inside them, weights = 2.5 * s / sum(s).
 //
-// Kernel 1 (router_logits_kernel): one CTA per (128 tokens, EB experts).
+// Kernel 1 (router_logits_kernel): one CTA per (128 tokens, EB experts, K
+// split).
 //   warp 0 : TMA producer (x tile [128 x 64] and Wg tile [EB x 64] per stage,
 //            128-byte swizzle, 4-stage ring)
 //   warp 1 : tcgen05.mma issuer, M=128 N=EB K=16, fp32 accumulator in TMEM;
 //            each 64-wide K chunk goes to the next of four TMEM buffers
-//   warps 2-5: drain each finished chunk from TMEM and add it into fp64
-//            registers, so the logit carries one fp32 rounding per 64 terms;
-//            at the end write fp32 logits [T, E].
+//   warps 2..: EB/16 drain warps per TMEM lane quarter, 16 columns each: each
+//            finished chunk is read from TMEM and added into fp64 registers,
+//            so a logit carries one fp32 rounding per 64 terms.  Without a K
+//            split the fp32 logits [T, E] are written at the end; with one,
+//            the fp64 partial sums [split, T, E] are, and kernel 2 adds them
+//            in split order.  Small batches split K so that the grid still
+//            covers the device.
 // Kernel 2 (router_topk_kernel): one warp per token, k rounds of a warp
 //   arg-max on (value desc, index asc), then the weights.
 #include <cstdint>
@@ -33,10 +38,13 @@ constexpr int kRouterBK = 64;
 #endif
 constexpr int kRouterStages = MOE_ROUTER_STAGES;
 
-constexpr int kRouterAccBufs = 4;  // TMEM buffers: the MMA may run this many K chunks ahead of the drain
+constexpr int kRouterAccBufs = 4;    // TMEM buffers: the MMA may run this many K chunks ahead of the drain
+constexpr int kRouterDrainCols = 16; // accumulator columns per drain warp
 
 template <int EB>
 struct RouterSmem {
+  static constexpr int kDrainWarps = 4 * (EB / kRouterDrainCols);
+  static constexpr int kThreads = 64 + 32 * kDrainWarps;
   static constexpr uint32_t kABytes = kRouterBM * kRouterBK * 2;
   static constexpr uint32_t kBBytes = EB * kRouterBK * 2;
   static constexpr uint32_t kTmemCols = kRouterAccBufs * EB <= 128 ? 128 : 256;
@@ -44,9 +52,10 @@ struct RouterSmem {
 };
 
 template <int EB>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
     router_logits_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wg,
-                         int T, int d, int E, float* __restrict__ logits, uint32_t* __restrict__ status) {
+                         int T, int d, int E, int chunks_per_split, float* __restrict__ logits,
+                         double* __restrict__ part, uint32_t* __restrict__ status) {
   using L = RouterSmem<EB>;
   constexpr int S = kRouterStages;
   extern __shared__ uint8_t smem_raw[];
@@ -66,7 +75,8 @@ __global__ void __launch_bounds__(192, 1)
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kRouterBM;
   const int e0 = blockIdx.y * EB;
-  const int nk = d / kRouterBK;
+  const int kc0 = blockIdx.z * chunks_per_split;  // first K chunk of this split
+  const int nk = min(d / kRouterBK, kc0 + chunks_per_split) - kc0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -75,7 +85,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < kRouterAccBufs; ++b) {
       ptx::mbar_init(&tfull[b], 1);
-      ptx::mbar_init(&tempty[b], 128);
+      ptx::mbar_init(&tempty[b], 32 * L::kDrainWarps);
     }
     ptx::mbar_init(done, 1);
     *abort_flag = 0u;
@@ -106,8 +116,8 @@ __global__ void __launch_bounds__(192, 1)
           break;
         }
         ptx::mbar_arrive_expect_tx(&full[s], L::kABytes + L::kBBytes);
-        ptx::tma_load_2d(sA + s * L::kABytes, &tm_x, &full[s], kb * kRouterBK, m0, pol);
-        ptx::tma_load_2d(sB + s * L::kBBytes, &tm_wg, &full[s], kb * kRouterBK, e0, pol);
+        ptx::tma_load_2d(sA + s * L::kABytes, &tm_x, &full[s], (kc0 + kb) * kRouterBK, m0, pol);
+        ptx::tma_load_2d(sB + s * L::kBBytes, &tm_wg, &full[s], (kc0 + kb) * kRouterBK, e0, pol);
         issued = kb + 1;
       }
       // every issued copy must land before the CTA may exit
@@ -141,11 +151,12 @@ __global__ void __launch_bounds__(192, 1)
       if (!ptx::wait_bounded(done, 0, &never)) raise_status(status, abort_flag, kStatusTimeout);
     }
   } else {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;                             // TMEM lane quarter this warp may access
+    const int c0 = ((warp - 2) >> 2) * kRouterDrainCols;  // first accumulator column it drains
     const int row = q * 32 + lane;
-    double acc[EB];
+    double acc[kRouterDrainCols];
 #pragma unroll
-    for (int j = 0; j < EB; ++j) acc[j] = 0.0;
+    for (int j = 0; j < kRouterDrainCols; ++j) acc[j] = 0.0;
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       const int b = kb % kRouterAccBufs;
@@ -156,35 +167,25 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       ptx::tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + b * EB;
-      if (EB == 64) {
-        // both 32-column halves in flight before one wait
-        uint32_t r0[32], r1[32];
-        ptx::tmem_ld32(taddr, r0);
-        ptx::tmem_ld32(taddr + 32, r1);
-        ptx::tmem_ld_wait2(r0, r1);
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&tempty[b]);
+      uint32_t r[kRouterDrainCols];
+      ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + b * EB + c0, r);
+      ptx::tmem_ld_wait(r);
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&tempty[b]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          acc[i] += (double)__uint_as_float(r0[i]);
-          acc[32 + i] += (double)__uint_as_float(r1[i]);
-        }
-      } else {
-        uint32_t r[32];
-        ptx::tmem_ld32(taddr, r);
-        ptx::tmem_ld_wait(r);
-        ptx::tc_fence_before();
-        ptx::mbar_arrive(&tempty[b]);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] += (double)__uint_as_float(r[i]);
-      }
+      for (int i = 0; i < kRouterDrainCols; ++i) acc[i] += (double)__uint_as_float(r[i]);
     }
     if (ok && m0 + row < T) {
-      float4* out = reinterpret_cast<float4*>(logits + (size_t)(m0 + row) * E + e0);
+      if (part == nullptr) {
+        float4* out = reinterpret_cast<float4*>(logits + (size_t)(m0 + row) * E + e0 + c0);
 #pragma unroll
-      for (int j = 0; j < EB / 4; ++j)
-        out[j] = make_float4((float)acc[4 * j], (float)acc[4 * j + 1], (float)acc[4 * j + 2], (float)acc[4 * j + 3]);
+        for (int j = 0; j < kRouterDrainCols / 4; ++j)
+          out[j] = make_float4((float)acc[4 * j], (float)acc[4 * j + 1], (float)acc[4 * j + 2], (float)acc[4 * j + 3]);
+      } else {
+        double2* out = reinterpret_cast<double2*>(part + ((size_t)blockIdx.z * T + m0 + row) * E + e0 + c0);
+#pragma unroll
+        for (int j = 0; j < kRouterDrainCols / 2; ++j) out[j] = make_double2(acc[2 * j], acc[2 * j + 1]);
+      }
     }
   }
 
@@ -219,8 +220,9 @@ __device__ __forceinline__ Cand warp_best(Cand c) {
 // NV = values per lane (expert e lives in lane e % 32, slot e / 32).
 template <int NV>
 __global__ void __launch_bounds__(128)
-    router_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias,
-                       const uint8_t* __restrict__ allowed, int T, int E, int k, int route, int n_group,
+    router_topk_kernel(float* __restrict__ logits, const double* __restrict__ part, int splits,
+                       const float* __restrict__ bias, const uint8_t* __restrict__ allowed, int T, int E, int k,
+                       int route, int n_group,
                        int topk_group, int group_topn, float route_scale, int32_t* __restrict__ topk_idx,
                        float* __restrict__ topk_w) {
   __shared__ float sel_sh[4][NV * 32];
@@ -232,13 +234,23 @@ __global__ void __launch_bounds__(128)
 
   float key[NV], aux[NV];
   uint32_t taken = 0;  // bit v: slot v of this lane is out of the running
-  const float* lrow = logits + (size_t)t * E;
+  float* lrow = logits + (size_t)t * E;
 #pragma unroll
   for (int v = 0; v < NV; ++v) {
     const int e = v * 32 + lane;
     if (e < E) {
+      float l0;
+      if (part) {
+        // K-split gate GEMM: add the fp64 partial sums in split order
+        double a = 0.0;
+        for (int sp = 0; sp < splits; ++sp) a += part[((size_t)sp * T + t) * E + e];
+        l0 = (float)a;
+        lrow[e] = l0;
+      } else {
+        l0 = lrow[e];
+      }
       // device-limited routing: experts this device does not hold get -inf
-      const float l = (allowed && !allowed[e]) ? NEG : lrow[e];
+      const float l = (allowed && !allowed[e]) ? NEG : l0;
       if (route == 0) {
         key[v] = l;
         aux[v] = l;
@@ -332,22 +344,28 @@ __global__ void __launch_bounds__(128)
 }
 
 template <int EB>
-cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E,
-                                 float* logits, uint32_t* status, cudaStream_t stream) {
+cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E, int splits,
+                                 float* logits, double* part, uint32_t* status, cudaStream_t stream) {
   const size_t smem = RouterSmem<EB>::kBytes;
   cudaError_t err = cudaFuncSetAttribute(router_logits_kernel<EB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
   if (err != cudaSuccess) return err;
-  dim3 grid((T + kRouterBM - 1) / kRouterBM, E / EB);
-  router_logits_kernel<EB><<<grid, 192, smem, stream>>>(tm_x, tm_wg, T, d, E, logits, status);
+  const int nk = d / kRouterBK;
+  if (splits < 1 || splits > nk || (splits > 1 && part == nullptr)) return cudaErrorInvalidValue;
+  const int cps = (nk + splits - 1) / splits;
+  if ((nk + cps - 1) / cps != splits) return cudaErrorInvalidValue;  // a split would get no chunk
+  dim3 grid((T + kRouterBM - 1) / kRouterBM, E / EB, splits);
+  router_logits_kernel<EB><<<grid, RouterSmem<EB>::kThreads, smem, stream>>>(
+      tm_x, tm_wg, T, d, E, cps, logits, splits > 1 ? part : nullptr, status);
   return cudaGetLastError();
 }
 
 template <int NV>
-cudaError_t launch_topk_nv(const float* logits, const float* bias, const uint8_t* allowed, const RouteParams& rp,
-                           int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream) {
-  router_topk_kernel<NV><<<(T + 3) / 4, 128, 0, stream>>>(logits, bias, allowed, T, E, k, rp.route, rp.n_group,
-                                                          rp.topk_group, rp.group_topn, rp.route_scale, idx, w);
+cudaError_t launch_topk_nv(float* logits, const double* part, int splits, const float* bias, const uint8_t* allowed,
+                           const RouteParams& rp, int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream) {
+  router_topk_kernel<NV><<<(T + 3) / 4, 128, 0, stream>>>(logits, part, splits, bias, allowed, T, E, k, rp.route,
+                                                          rp.n_group, rp.topk_group, rp.group_topn, rp.route_scale,
+                                                          idx, w);
   return cudaGetLastError();
 }
 
@@ -359,24 +377,40 @@ int router_expert_block(int E) {
   return 0;
 }
 
-cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E,
-                                 float* logits, uint32_t* status, cudaStream_t stream) {
+int router_splits(int64_t T, int d, int E, int sms) {
+  const int eb = router_expert_block(E);
+  const int nk = d / kRouterBK;
+  if (eb == 0 || T <= 0 || nk <= 1) return 1;
+  sms = sms < 1 ? 1 : (sms > kRouterMaxSms ? kRouterMaxSms : sms);
+  const int64_t ctas = (T + kRouterBM - 1) / kRouterBM * (E / eb);
+  if (ctas * 2 > sms) return 1;
+  const int want = (int)(sms / ctas);
+  const int cps = (nk + want - 1) / want;
+  return (nk + cps - 1) / cps;
+}
+
+cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E, int splits,
+                                 float* logits, double* part, uint32_t* status, cudaStream_t stream) {
   switch (router_expert_block(E)) {
-    case 64: return launch_router_logits<64>(tm_x, tm_wg, T, d, E, logits, status, stream);
-    case 32: return launch_router_logits<32>(tm_x, tm_wg, T, d, E, logits, status, stream);
+    case 64: return launch_router_logits<64>(tm_x, tm_wg, T, d, E, splits, logits, part, status, stream);
+    case 32: return launch_router_logits<32>(tm_x, tm_wg, T, d, E, splits, logits, part, status, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_router_topk(const float* logits, const float* bias, const uint8_t* allowed, const RouteParams& rp,
-                               int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream) {
+cudaError_t launch_router_topk(float* logits, const double* part, int splits, const float* bias,
+                               const uint8_t* allowed, const RouteParams& rp, int T, int E, int k, int32_t* idx,
+                               float* w, cudaStream_t stream) {
   const int nv = (E + 31) / 32;
-  if (nv <= 1) return launch_topk_nv<1>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
-  if (nv <= 2) return launch_topk_nv<2>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
-  if (nv <= 4) return launch_topk_nv<4>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
-  if (nv <= 8) return launch_topk_nv<8>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
-  if (nv <= 16) return launch_topk_nv<16>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
-  if (nv <= 32) return launch_topk_nv<32>(logits, bias, allowed, rp, T, E, k, idx, w, stream);
+  if (splits <= 1) part = nullptr;
+#define MOE_TOPK(N) return launch_topk_nv<N>(logits, part, splits, bias, allowed, rp, T, E, k, idx, w, stream)
+  if (nv <= 1) MOE_TOPK(1);
+  if (nv <= 2) MOE_TOPK(2);
+  if (nv <= 4) MOE_TOPK(4);
+  if (nv <= 8) MOE_TOPK(8);
+  if (nv <= 16) MOE_TOPK(16);
+  if (nv <= 32) MOE_TOPK(32);
+#undef MOE_TOPK
   return cudaErrorInvalidValue;
 }
 

@@ -34,8 +34,14 @@ def _medium(**kw):
     return to_device(workloads.make_small("prefill", **shape))
 
 
+def _wide():
+    # 32 token tiles x 4 expert blocks: enough CTAs that the gate GEMM runs
+    # without a K split (tiny and medium split K into 8 and 16 parts)
+    return to_device(workloads.make_small("prefill", T=4096, d=512, E=256, k=8, inter=128, shared_inter=0))
+
+
 # --------------------------------------------------------------- router
-@pytest.mark.parametrize("make", [_tiny, _medium])
+@pytest.mark.parametrize("make", [_tiny, _medium, _wide])
 def test_router_matches_oracle(make):
     w = make()
     cfg = w.cfg
