@@ -25,6 +25,7 @@ __global__ void __launch_bounds__(128)
   __shared__ int32_t rows[32];
   __shared__ float ws[32];
   const int64_t t = blockIdx.x;
+  grid_dependency_wait();
   if (threadIdx.x < k) {
     rows[threadIdx.x] = row_of[t * k + threadIdx.x];
     ws[threadIdx.x] = topk_w[t * k + threadIdx.x];
@@ -75,11 +76,12 @@ cudaError_t launch_combine(const void* Y_perm, const float* Y_shared, const int3
   if (T == 0) return cudaSuccess;
   const uint4* yp = static_cast<const uint4*>(Y_perm);
   const float4* ys = reinterpret_cast<const float4*>(Y_shared);
-  if (y_bf16)
-    combine_kernel<true><<<(unsigned)T, 128, 0, stream>>>(yp, ys, row_of, topk_w, k, d, y);
-  else
-    combine_kernel<false><<<(unsigned)T, 128, 0, stream>>>(yp, ys, row_of, topk_w, k, d, y);
-  return cudaGetLastError();
+  const cudaError_t err =
+      y_bf16 ? launch_chained(combine_kernel<true>, dim3((unsigned)T), dim3(128), 0, stream, yp, ys, row_of, topk_w, k,
+                              d, y)
+             : launch_chained(combine_kernel<false>, dim3((unsigned)T), dim3(128), 0, stream, yp, ys, row_of, topk_w,
+                              k, d, y);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -257,6 +257,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();  // tile list, counters and A rows come from earlier kernels
 
   const TileSpan span = tile_span(p);
   const int total = span.count * p.n_nb;
@@ -613,7 +614,9 @@ cudaError_t launch(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtenso
       cudaFuncSetAttribute(grouped_gemm_kernel<M, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   if (grid <= 0) return cudaSuccess;
-  grouped_gemm_kernel<M, F8><<<grid, kernel_threads<F8>(), smem, stream>>>(a_r, a_s, b_r, b_s, c_r, c_s, p);
+  cudaError_t e = launch_chained(grouped_gemm_kernel<M, F8>, grid, dim3(kernel_threads<F8>()), smem, stream, a_r, a_s,
+                                 b_r, b_s, c_r, c_s, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -22,6 +22,7 @@ __global__ void expert_utilisation_kernel(const int32_t* __restrict__ counts, in
                                           int32_t* __restrict__ flags) {
   __shared__ long long partial[32];
   long long mine = 0;
+  grid_dependency_wait();
   for (int e = threadIdx.x; e < E; e += blockDim.x) mine += counts[e];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
@@ -40,8 +41,9 @@ __global__ void expert_utilisation_kernel(const int32_t* __restrict__ counts, in
 
 cudaError_t launch_expert_utilisation(const int32_t* counts, int E, float* util, int32_t* flags,
                                       cudaStream_t stream) {
-  expert_utilisation_kernel<<<1, 256, 0, stream>>>(counts, E, util, flags);
-  return cudaGetLastError();
+  const cudaError_t err =
+      launch_chained(expert_utilisation_kernel, dim3(1), dim3(256), 0, stream, counts, E, util, flags);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -35,6 +35,7 @@ __global__ void __launch_bounds__(kPermThreads)
   extern __shared__ int32_t h[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
   __syncthreads();
+  grid_dependency_wait();
   const int64_t begin = (int64_t)blockIdx.x * kPermTokens * k;
   const int64_t end = ::min((long long)T * k, (long long)(begin + (int64_t)kPermTokens * k));
   for (int64_t i = begin + threadIdx.x; i < end; i += blockDim.x) {
@@ -55,6 +56,7 @@ __global__ void scan_kernel(const int32_t* __restrict__ hist, int nb, int E, int
   __shared__ int32_t warp_sums[32];
   const int e = threadIdx.x;
   int32_t run = 0;
+  grid_dependency_wait();
   if (e < E)
     for (int b = 0; b < nb; ++b) {
       const int32_t v = hist[(size_t)b * E + e];
@@ -102,6 +104,7 @@ __global__ void __launch_bounds__(kPermThreads)
   const int nwarps = kPermThreads / 32;
   for (int i = threadIdx.x; i < nwarps * E; i += blockDim.x) wh[i] = 0;
   __syncthreads();
+  grid_dependency_wait();
 
   const int64_t tok0 = (int64_t)blockIdx.x * kPermTokens + warp * 32;
   const int64_t ent0 = tok0 * k;
@@ -158,15 +161,37 @@ __global__ void __launch_bounds__(kPermThreads)
 }
 
 // x_perm[r, :] = x[perm_token[r], :]; rows of d bf16 (d % 8 == 0), 16-byte
-// vectors, one CTA per row at a time.
+// vectors, one CTA per row at a time.  Each thread issues kGatherUnroll loads
+// before its stores, so an SM keeps enough bytes in flight to cover HBM
+// latency; the next row's token index is fetched while this row is copied.
+constexpr int kGatherUnroll = 4;
+
 __global__ void __launch_bounds__(256)
     gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_token, int64_t rows,
                        int vec_per_row, uint4* __restrict__ x_perm) {
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const int32_t t = perm_token[r];
+  grid_dependency_wait();
+  int64_t r = blockIdx.x;
+  if (r >= rows) return;
+  int32_t t = perm_token[r];
+  for (; r < rows; r += gridDim.x) {
+    const int64_t rn = r + gridDim.x;
+    const int32_t tn = rn < rows ? perm_token[rn] : 0;
     const uint4* src = x + (size_t)t * vec_per_row;
     uint4* dst = x_perm + (size_t)r * vec_per_row;
-    for (int v = threadIdx.x; v < vec_per_row; v += blockDim.x) dst[v] = __ldg(src + v);
+    for (int v0 = threadIdx.x; v0 < vec_per_row; v0 += kGatherUnroll * blockDim.x) {
+      uint4 buf[kGatherUnroll];
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        const int v = v0 + u * blockDim.x;
+        if (v < vec_per_row) buf[u] = __ldg(src + v);
+      }
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        const int v = v0 + u * blockDim.x;
+        if (v < vec_per_row) dst[v] = buf[u];
+      }
+    }
+    t = tn;
   }
 }
 
@@ -182,6 +207,7 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
   const int e = threadIdx.x;
   const int lane = e & 31, warp = e >> 5;
   int32_t start = 0, cnt = 0, mt = 0;
+  grid_dependency_wait();
   if (e < E) {
     start = offsets[e];
     cnt = offsets[e + 1] - start;
@@ -234,36 +260,38 @@ cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int32_t*
                            int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* row_of,
                            uint32_t* status, cudaStream_t stream) {
   const int nb = permute_blocks(T);
-  hist_kernel<<<nb, kPermThreads, E * sizeof(int32_t), stream>>>(idx, (int)T, k, E, hist, status);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_chained(hist_kernel, dim3(nb), dim3(kPermThreads), E * sizeof(int32_t), stream, idx,
+                                   (int)T, k, E, hist, status);
   if (err != cudaSuccess) return err;
   const int st = ((E + 31) / 32) * 32;
-  scan_kernel<<<1, st, 0, stream>>>(hist, nb, E, base, counts, offsets);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  err = launch_chained(scan_kernel, dim3(1), dim3(st), 0, stream, hist, nb, E, base, counts, offsets);
+  if (err != cudaSuccess) return err;
   const size_t sm = (size_t)(kPermThreads / 32) * E * sizeof(int32_t);
   if (sm > 48 * 1024) {
     err = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (err != cudaSuccess) return err;
   }
-  scatter_kernel<<<nb, kPermThreads, sm, stream>>>(idx, (int)T, k, E, base, perm_token, row_of);
-  return cudaGetLastError();
+  err = launch_chained(scatter_kernel, dim3(nb), dim3(kPermThreads), sm, stream, idx, (int)T, k, E, base, perm_token,
+                       row_of);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t rows, int d, void* x_perm,
                                int num_sms, cudaStream_t stream) {
   if (rows == 0) return cudaSuccess;
   const int64_t g = std::min<int64_t>(rows, (int64_t)num_sms * 16);
-  gather_rows_kernel<<<(unsigned)g, 256, 0, stream>>>(static_cast<const uint4*>(x), perm_token, rows, d / 8,
-                                                      static_cast<uint4*>(x_perm));
-  return cudaGetLastError();
+  const cudaError_t err = launch_chained(gather_rows_kernel, dim3((unsigned)g), dim3(256), 0, stream,
+                                         static_cast<const uint4*>(x), perm_token, rows, d / 8,
+                                         static_cast<uint4*>(x_perm));
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, bool with_shared, int4* tiles,
                                int32_t* ntiles, int* sched_counters, cudaStream_t stream) {
   const int threads = ((E + 31) / 32) * 32;
-  build_tiles_kernel<<<1, threads < 32 ? 32 : threads, 0, stream>>>(offsets, E, (int)T, with_shared ? 1 : 0,
-                                                                    tiles, ntiles, sched_counters);
-  return cudaGetLastError();
+  const cudaError_t err = launch_chained(build_tiles_kernel, dim3(1), dim3(threads < 32 ? 32 : threads), 0, stream,
+                                         offsets, E, (int)T, with_shared ? 1 : 0, tiles, ntiles, sched_counters);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

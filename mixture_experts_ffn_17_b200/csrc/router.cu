@@ -101,6 +101,7 @@ __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -229,6 +230,7 @@ __global__ void __launch_bounds__(128)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 4 + warp;
+  grid_dependency_wait();
   if (t >= T) return;
   const float NEG = -__int_as_float(0x7f800000);  // -inf
 
@@ -355,18 +357,18 @@ cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_
   const int cps = (nk + splits - 1) / splits;
   if ((nk + cps - 1) / cps != splits) return cudaErrorInvalidValue;  // a split would get no chunk
   dim3 grid((T + kRouterBM - 1) / kRouterBM, E / EB, splits);
-  router_logits_kernel<EB><<<grid, RouterSmem<EB>::kThreads, smem, stream>>>(
-      tm_x, tm_wg, T, d, E, cps, logits, splits > 1 ? part : nullptr, status);
-  return cudaGetLastError();
+  err = launch_chained(router_logits_kernel<EB>, grid, dim3(RouterSmem<EB>::kThreads), smem, stream, tm_x, tm_wg, T,
+                       d, E, cps, logits, splits > 1 ? part : nullptr, status);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 template <int NV>
 cudaError_t launch_topk_nv(float* logits, const double* part, int splits, const float* bias, const uint8_t* allowed,
                            const RouteParams& rp, int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream) {
-  router_topk_kernel<NV><<<(T + 3) / 4, 128, 0, stream>>>(logits, part, splits, bias, allowed, T, E, k, rp.route,
-                                                          rp.n_group, rp.topk_group, rp.group_topn, rp.route_scale,
-                                                          idx, w);
-  return cudaGetLastError();
+  const cudaError_t err =
+      launch_chained(router_topk_kernel<NV>, dim3((T + 3) / 4), dim3(128), 0, stream, logits, part, splits, bias,
+                     allowed, T, E, k, rp.route, rp.n_group, rp.topk_group, rp.group_topn, rp.route_scale, idx, w);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace
