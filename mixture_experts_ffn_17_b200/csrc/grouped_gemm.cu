@@ -104,6 +104,11 @@ struct TileInfo {
   bool shared;
 };
 
+// A half with at most 64 rows runs as an M=64 MMA (half the tensor work of
+// M=128).  Its accumulator holds row 16q + i in TMEM lane 32q + i (i < 16) of
+// the slot: the half-subpartition layout of the 64-row tcgen05.mma.
+__device__ __forceinline__ bool narrow_half(const TileInfo& ti, int h) { return ti.rows - h * kTileM <= kTileM / 2; }
+
 // The part of the tile list this launch walks: `count` tile-list rows.  A
 // launch over the whole list interleaves the shared expert's rows evenly among
 // the routed ones (the shared weights stay in L2 while routed tiles keep HBM
@@ -384,6 +389,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
       // 0-127 of the accumulator are g = x W1 and 128-255 are u = x W3 (A is
       // read once for both).  Down: 256 columns of W2.
       constexpr uint32_t idesc = ptx::idesc_bf16(kTileM, 256, false, true);
+      constexpr uint32_t idesc_narrow = ptx::idesc_bf16(kTileM / 2, 256, false, true);
       int kg = 0, ns = 0;
       SlotRing ring;
       bool ok = true;
@@ -421,7 +427,8 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
             const uint64_t bd = ptx::sdesc_sw128(b0 + kk * 2048, BoxBytes, 1024);
             for (int h = 0; h < ti.halves; ++h) {
               const uint64_t ad = ptx::sdesc(a0 + h * ABytes + kk * 32, 16, ASBO, ASwz);
-              ptx::mma_bf16(tmem + ((ring.next + h) & 1) * kSlotCols, ad, bd, idesc, acc);
+              ptx::mma_bf16(tmem + ((ring.next + h) & 1) * kSlotCols, ad, bd, narrow_half(ti, h) ? idesc_narrow : idesc,
+                            acc);
             }
           }
           ptx::mma_commit(&empty[s]);
@@ -462,8 +469,9 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         }
         ptx::tc_fence_after();
         const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + sl * kSlotCols;
-        const int r = h * kTileM + row;  // row within the tile
-        const bool valid = r < ti.rows;
+        const bool narrow = narrow_half(ti, h);
+        const int r = h * kTileM + (narrow ? (lane < 16 ? q * 16 + lane : kTileM) : row);  // row within the tile
+        const bool valid = r < ti.rows && (!narrow || lane < 16);
         if (M == Mode::kSwiGLU) {
           const int64_t hrow = (int64_t)ti.row0 + r + (ti.shared ? p.out_shared_row_offset : 0);
           uint16_t* base = static_cast<uint16_t*>(ti.shared ? p.out_shared : p.out_routed);
