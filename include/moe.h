@@ -12,7 +12,7 @@
  *   expert(x) = W2^T (silu(x W1) * (x W3))   SwiGLU, "All 5 steps" of
  *       "DeepSeek-V3.2-Exp / Mixture of experts / Shared expert" (atlas page)
  *   y[t] = sum_j w[t,j] expert_{idx[t,j]}(x[t]) + shared(x[t])
- *       (atlas page, MoE forward excerpt model.py 790-803: per-expert token
+ *       (atlas page, "Code" section, MoE forward block: per-expert token
  *        lists from bincount/where, an fp32 accumulator, then the shared
  *        expert added to every token)
  *
@@ -128,7 +128,7 @@ moe_status moe_expert_utilisation(const moe_shape* shape, const int32_t* counts,
 /* Dispatch: counts = bincount(topk_idx, minlength=E); offsets = exclusive
  * prefix sum (E+1 entries); the permuted order lists experts ascending and,
  * within an expert, its (token, slot) entries ascending -- the order of the
- * atlas page's torch.where(indices == i) (model.py 790-803 excerpt).
+ * atlas page's torch.where(indices == i) ("Code" section, MoE forward block).
  *   perm_token [T*k] int32 out: token at permuted position r
  *   row_of     [T*k] int32 out: permuted position of entry (t, j) at t*k + j
  *   x, x_perm  optional pair: when both are non-NULL, x_perm [T*k, d] bf16
@@ -171,7 +171,8 @@ moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t* topk_idx, 
  *     and s2 [E, inter/128, d/128] (dequantised value = code * scale)
  *   W1s, W3s [d, shared_inter], W2s [shared_inter, d] bf16 (NULL when none)
  *   Y_perm [T*k, d] bf16 out; Y_shared [T, d] fp32 out (NULL when none)
- * Source: atlas page "All 5 steps" and the model.py 643 excerpt (silu and
+ * Source: atlas page "All 5 steps" and the expert forward block of its "Code"
+ * section (silu and
  * product in fp32, h cast to the activation dtype before W2). */
 moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const void* x_perm, const int32_t* offsets,
                               const void* W1, const void* W3, const void* W2, const float* s1, const float* s3,
@@ -180,7 +181,8 @@ moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const void*
 
 /* Combine: y[t] = Y_shared[t] + sum_j topk_w[t,j] * Y_perm[row_of[t*k+j]],
  * summed in fp32 in slot order, written as shape->y_dtype.  Y_shared may be
- * NULL (no shared expert).  Source: atlas page model.py 790-803 excerpt. */
+ * NULL (no shared expert).  Source: atlas page, "Code" section, MoE forward
+ * block. */
 moe_status moe_combine(const moe_shape* shape, const void* Y_perm, const float* Y_shared, const int32_t* row_of,
                        const float* topk_w, void* y, void* stream);
 
@@ -193,6 +195,35 @@ moe_status moe_forward(const moe_shape* shape, const void* x, const void* Wg, co
                        const void* W3, const void* W2, const float* s1, const float* s3, const float* s2,
                        const void* W1s, const void* W3s, const void* W2s, void* y, int32_t* topk_idx_out,
                        float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes, void* stream);
+
+/* One rank's share of the expert-parallel layer (atlas page, "Code" section:
+ * the MoE constructor block gives rank r the experts
+ * [r*E/ep_size, (r+1)*E/ep_size) and a tensor-parallel shared expert; the MoE
+ * forward block adds the local experts' weighted outputs and this rank's
+ * shared-expert partial into y, then all-reduces y over the ranks):
+ *   y[t] = sum over slots j with e = topk_idx[t,j] local of topk_w[t,j] * expert_e(x[t])
+ *        + shared_r(x[t]),
+ *   shared_r = the shared expert restricted to hidden features
+ *              [r*Is/ep_size, (r+1)*Is/ep_size) (Is = shape->shared_inter).
+ * Summing y over ep_rank = 0..ep_size-1 gives moe_forward's y; the caller does
+ * that sum (the all-reduce, e.g. NCCL).  Routing runs over all E experts on
+ * every rank (same inputs, same indices).
+ *   shape: the whole layer's shape (E experts, shared_inter Is).
+ *   W1, W3 [E/ep_size, d, inter], W2 [E/ep_size, inter, d] (and s1, s3, s2
+ *     [E/ep_size, ...] for MOE_E4M3): this rank's experts only, slice 0 =
+ *     expert r*E/ep_size.
+ *   W1s, W3s [d, Is/ep_size], W2s [Is/ep_size, d]: this rank's columns of the
+ *     shared W1/W3 and rows of W2 (NULL when Is = 0).
+ *   Other arguments as moe_forward; topk_idx_out / topk_w_out / counts_out
+ *   report the full routing.
+ * Errors: MOE_ERR_INVALID_ARG for ep_size < 1 or ep_rank outside
+ * [0, ep_size); MOE_ERR_UNSUPPORTED unless E and Is divide by ep_size and
+ * Is/ep_size is a multiple of 128.  ep_size = 1 is moe_forward. */
+moe_status moe_forward_ep(const moe_shape* shape, int ep_rank, int ep_size, const void* x, const void* Wg,
+                          const float* bias, const void* W1, const void* W3, const void* W2, const float* s1,
+                          const float* s3, const float* s2, const void* W1s, const void* W3s, const void* W2s, void* y,
+                          int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes,
+                          void* stream);
 
 /* moe_forward plus per-stage timing: records the caller's CUDA events
  * (cudaEvent_t handles, created with timing enabled) on `stream` at the stage

@@ -23,7 +23,7 @@ MOE_ROUTE_TOPK_SOFTMAX, MOE_ROUTE_SIGMOID_GROUP = 0, 1
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
             "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version",
-            "moe_permute_noalloc", "moe_router_topk_limited", "moe_expert_utilisation")
+            "moe_permute_noalloc", "moe_router_topk_limited", "moe_expert_utilisation", "moe_forward_ep")
 NUM_STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "experts_up", "experts_down", "combine")
 
@@ -78,9 +78,11 @@ def lib() -> ctypes.CDLL:
         L.moe_combine.argtypes = [S, P, P, P, P, P, P]
         L.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P, P]
+        I = ctypes.c_int
+        L.moe_forward_ep.argtypes = [S, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         for fn in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward",
-                   "moe_forward_profiled", "moe_check_device_status"):
+                   "moe_forward_profiled", "moe_forward_ep", "moe_check_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -166,6 +168,18 @@ def forward(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, ws, to
                              _ptr(s1), _ptr(s3), _ptr(s2), _ptr(W1s), _ptr(W3s), _ptr(W2s), _ptr(y), _ptr(topk_idx),
                              _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel() if ws is not None else 0,
                              _stream(stream)), "moe_forward")
+
+
+def forward_ep(shape, ep_rank, ep_size, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, ws, topk_idx=None,
+               topk_w=None, counts=None, stream=None):
+    """This rank's share of the expert-parallel layer (moe_forward_ep): W1/W3/W2
+    (and scales) hold the rank's E/ep_size experts, W1s/W3s/W2s its slice of
+    the shared expert's hidden features; y receives the partial sum that
+    all_reduce_partial (or any sum over ranks) completes."""
+    _check(lib().moe_forward_ep(ctypes.byref(shape), int(ep_rank), int(ep_size), _ptr(x), _ptr(Wg), _ptr(bias),
+                                _ptr(W1), _ptr(W3), _ptr(W2), _ptr(s1), _ptr(s3), _ptr(s2), _ptr(W1s), _ptr(W3s),
+                                _ptr(W2s), _ptr(y), _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(ws),
+                                ws.numel() if ws is not None else 0, _stream(stream)), "moe_forward_ep")
 
 
 def forward_profiled(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, ws, events, topk_idx=None,

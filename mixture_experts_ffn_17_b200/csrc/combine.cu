@@ -1,6 +1,6 @@
 // combine.cu -- weighted sum of each token's expert outputs back in token order.
 //
-// The atlas page's MoE forward (model.py 790-803 excerpt) accumulates
+// The atlas page's MoE forward ("Code" section, MoE forward block) accumulates
 // y[idx] += expert(x[idx]) * weights[idx, top] into an fp32 buffer, then adds
 // the shared expert.  Here every token gathers its k routed rows (bf16, in
 // permuted order, located through row_of) and its shared-expert row (fp32),
@@ -21,13 +21,16 @@ template <bool OUT_BF16>
 __global__ void __launch_bounds__(128)
     combine_kernel(const uint4* __restrict__ Y_perm, const float4* __restrict__ Y_shared,
                    const int32_t* __restrict__ row_of, const float* __restrict__ topk_w, int k, int d,
-                   void* __restrict__ y) {
+                   void* __restrict__ y, const int32_t* __restrict__ offsets, int e_lo, int e_hi) {
   __shared__ int32_t rows[32];
   __shared__ float ws[32];
   const int64_t t = blockIdx.x;
   grid_dependency_wait();
   if (threadIdx.x < k) {
-    rows[threadIdx.x] = row_of[t * k + threadIdx.x];
+    int32_t r = row_of[t * k + threadIdx.x];
+    // a shard adds only the rows of its own experts
+    if (offsets && (r < offsets[e_lo] || r >= offsets[e_hi])) r = -1;
+    rows[threadIdx.x] = r;
     ws[threadIdx.x] = topk_w[t * k + threadIdx.x];
   }
   __syncthreads();
@@ -72,15 +75,18 @@ __global__ void __launch_bounds__(128)
 }  // namespace
 
 cudaError_t launch_combine(const void* Y_perm, const float* Y_shared, const int32_t* row_of, const float* topk_w,
-                           int64_t T, int k, int d, void* y, bool y_bf16, cudaStream_t stream) {
+                           int64_t T, int k, int d, void* y, bool y_bf16, cudaStream_t stream,
+                           const int32_t* offsets, const Shard* shard) {
   if (T == 0) return cudaSuccess;
   const uint4* yp = static_cast<const uint4*>(Y_perm);
   const float4* ys = reinterpret_cast<const float4*>(Y_shared);
+  const int e_lo = shard ? shard->e_lo : 0, e_hi = shard ? shard->e_hi : 0;
+  if (!shard) offsets = nullptr;
   const cudaError_t err =
       y_bf16 ? launch_chained(combine_kernel<true>, dim3((unsigned)T), dim3(128), 0, stream, yp, ys, row_of, topk_w, k,
-                              d, y)
+                              d, y, offsets, e_lo, e_hi)
              : launch_chained(combine_kernel<false>, dim3((unsigned)T), dim3(128), 0, stream, yp, ys, row_of, topk_w,
-                              k, d, y);
+                              k, d, y, offsets, e_lo, e_hi);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

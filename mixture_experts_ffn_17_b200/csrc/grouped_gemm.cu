@@ -3,7 +3,7 @@
 // SwiGLU expert ("DeepSeek-V3.2-Exp / Mixture of experts / Shared expert",
 // "All 5 steps"): g = x W1, u = x W3, a = g sigmoid(g), h = a * u, y = h W2.
 // The page's code applies silu and the product in fp32 and casts h to the
-// activation dtype before W2 (model.py 643 excerpt); here h is stored bf16.
+// activation dtype before W2 (the expert forward block of its "Code" section); h is stored bf16.
 //
 // Both kernels are persistent (one CTA per SM) and walk a device-side tile
 // list: one entry per 256-row slice of an expert's segment of permuted rows,
@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         const CUtensorMap* mB = ti.shared ? &tmB_s : &tmB_r;
         const CUtensorMap* mC = ti.shared ? &tmC_s : &tmC_r;
         const int arow = ti.row0 + (ti.shared ? p.a_shared_row_offset : 0);
-        const int e3 = ti.shared ? 0 : ti.group;
+        const int e3 = ti.shared ? 0 : ti.group - p.group_base;
         const int nk = (ti.shared ? p.K_shared : p.K_routed) / BK;
         const int n0 = ti.nb * BN;
         const uint32_t bytes = ti.halves * ABytes + (F8 ? 2 * kF8RawBox : kBBytes);
@@ -574,7 +574,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         const uint8_t* raw = stage0 + s * kF8StageBytes + 2 * kF8ABytes;
         uint8_t* conv = conv0 + c * kF8ConvBytes;
         const int kblk = (kb * BK) / 128;
-        const int64_t sbase = ((int64_t)ti.group * ksb + kblk) * nsb;
+        const int64_t sbase = ((int64_t)(ti.group - p.group_base) * ksb + kblk) * nsb;
         float sc[2];
         if (M == Mode::kSwiGLU) {
           sc[0] = p.scale_b[sbase + n0 / 128];

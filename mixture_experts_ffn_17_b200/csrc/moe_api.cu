@@ -186,10 +186,14 @@ moe_status run_router(const moe_shape& s, const void* x, const void* Wg, const f
   return MOE_OK;
 }
 
+Shard whole_layer(const moe_shape& s) { return Shard{0, s.E}; }
+
+// Routed weights (and FP8 scales) hold the experts [shard.e_lo, shard.e_hi)
+// only: slice 0 is expert shard.e_lo.
 moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void* x, const void* x_perm,
                        const int32_t* offsets, const void* W1, const void* W3, const void* W2, const float* s1,
                        const float* s3, const float* s2, const void* W1s, const void* W3s, const void* W2s,
-                       void* Y_perm, float* Y_shared, uint32_t* status, cudaStream_t st,
+                       void* Y_perm, float* Y_shared, uint32_t* status, cudaStream_t st, const Shard& shard,
                        const cudaEvent_t* ev = nullptr) {
   const bool f8 = s.w_dtype == MOE_E4M3;
   const bool sh = s.shared_inter > 0;
@@ -198,7 +202,8 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   int32_t* ntiles = at<int32_t>(ws, L.ntiles);
   uint16_t* H = at<uint16_t>(ws, L.H);
   int* sched = at<int>(ws, L.sched);
-  MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, sh, tiles, ntiles, sched, st));
+  MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, shard, sh, tiles, ntiles, sched, st));
+  const int E_w = shard.e_hi - shard.e_lo;  // expert slices held by the weight tensors
   if (ev) MOE_CUDA(cudaEventRecord(ev[0], st));
 
   const int sms = num_sms();
@@ -208,12 +213,12 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
     return MOE_ERR_CUDA;
   if (f8) {
     // FP8 launches use a 64-deep K stage whatever the bf16 kernel's depth
-    if (!map_2d(&a8_r, x_perm, s.d, Tk, 64, kTileM) || !map_3d_u8(&w18_r, W1, s.inter, s.d, s.E) ||
-        !map_3d_u8(&w38_r, W3, s.inter, s.d, s.E))
+    if (!map_2d(&a8_r, x_perm, s.d, Tk, 64, kTileM) || !map_3d_u8(&w18_r, W1, s.inter, s.d, E_w) ||
+        !map_3d_u8(&w38_r, W3, s.inter, s.d, E_w))
       return MOE_ERR_CUDA;
     w1_r = a_r;  // placeholders: the bf16 launch below only walks the shared expert's tiles
     w3_r = a_r;
-  } else if (!map_3d(&w1_r, W1, s.inter, s.d, s.E, kGemmBK) || !map_3d(&w3_r, W3, s.inter, s.d, s.E, kGemmBK)) {
+  } else if (!map_3d(&w1_r, W1, s.inter, s.d, E_w, kGemmBK) || !map_3d(&w3_r, W3, s.inter, s.d, E_w, kGemmBK)) {
     return MOE_ERR_CUDA;
   }
   if (sh) {
@@ -228,6 +233,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   p1.ntiles = ntiles;
   p1.max_mtiles = L.max_mtiles;
   p1.E = s.E;
+  p1.group_base = shard.e_lo;
   const int bn1 = gemm_block_n_swiglu();
   p1.n_nb = (L.Hld + bn1 - 1) / bn1;
   p1.K_routed = s.d;
@@ -265,10 +271,10 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   CUtensorMap h_map, w2_r, w2_s, h8_map, w28_r;
   if (!map_2d(&h_map, H, L.Hld, L.Hrows, kGemmBK, kTileM)) return MOE_ERR_CUDA;
   if (f8) {
-    if (!map_2d(&h8_map, H, L.Hld, L.Hrows, 64, kTileM) || !map_3d_u8(&w28_r, W2, s.d, s.inter, s.E))
+    if (!map_2d(&h8_map, H, L.Hld, L.Hrows, 64, kTileM) || !map_3d_u8(&w28_r, W2, s.d, s.inter, E_w))
       return MOE_ERR_CUDA;
     w2_r = h_map;  // placeholder: the bf16 launch below only walks the shared expert's tiles
-  } else if (!map_3d(&w2_r, W2, s.d, s.inter, s.E, kGemmBK)) {
+  } else if (!map_3d(&w2_r, W2, s.d, s.inter, E_w, kGemmBK)) {
     return MOE_ERR_CUDA;
   }
   if (sh) {
@@ -317,10 +323,22 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
                         const void* W3, const void* W2, const float* s1, const float* s3, const float* s2,
                         const void* W1s, const void* W3s, const void* W2s, void* y, int32_t* topk_idx_out,
                         float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes, void* stream,
-                        const cudaEvent_t* ev) {
+                        const cudaEvent_t* ev, int ep_rank = 0, int ep_size = 1) {
   moe_status v = validate_shape(shape);
   if (v != MOE_OK) return v;
   const moe_shape& s = *shape;
+  if (ep_size < 1 || ep_rank < 0 || ep_rank >= ep_size) return MOE_ERR_INVALID_ARG;
+  // expert-parallel share (atlas page, "Code" section, the MoE constructor and
+  // forward blocks): an even slice of the routed experts, and the shared
+  // expert's slice of hidden features (its W1/W3 columns, W2 rows), so that
+  // the sum over ranks is the layer
+  if (s.E % ep_size != 0 || s.shared_inter % ep_size != 0 || (s.shared_inter / ep_size) % 128 != 0)
+    return MOE_ERR_UNSUPPORTED;
+  const int e_per = s.E / ep_size;
+  const Shard shard{ep_rank * e_per, (ep_rank + 1) * e_per};
+  const bool whole = ep_size == 1;
+  moe_shape sl = s;  // this rank's experts: shared expert of shared_inter / ep_size features
+  sl.shared_inter = s.shared_inter / ep_size;
   const bool sh = s.shared_inter > 0;
   if (!x || !Wg || !W1 || !W3 || !W2 || !y) return MOE_ERR_INVALID_ARG;
   if (sh && (!W1s || !W3s || !W2s)) return MOE_ERR_INVALID_ARG;
@@ -351,11 +369,13 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   if (ev) MOE_CUDA(cudaEventRecord(ev[1], st));
   MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
                           perm, row_of, status, st));
-  MOE_CUDA(launch_gather_rows(x, perm, s.T * s.k, s.d, x_perm, num_sms(), st));
-  r = run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared, status, st,
-                  ev ? ev + 2 : nullptr);
+  MOE_CUDA(launch_gather_rows(x, perm, s.T * s.k, s.d, x_perm, num_sms(), st, whole ? nullptr : offsets, shard.e_lo,
+                              shard.e_hi));
+  r = run_experts(sl, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared, status, st,
+                  shard, ev ? ev + 2 : nullptr);
   if (r != MOE_OK) return r;
-  MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16, st));
+  MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16, st,
+                          whole ? nullptr : offsets, whole ? nullptr : &shard));
   if (ev) MOE_CUDA(cudaEventRecord(ev[5], st));
   return MOE_OK;
 }
@@ -470,7 +490,7 @@ moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const void*
   MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
   if (s.T == 0) return MOE_OK;
   return run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm,
-                     sh ? Y_shared : nullptr, status, st);
+                     sh ? Y_shared : nullptr, status, st, whole_layer(s));
 }
 
 moe_status moe_combine(const moe_shape* shape, const void* Y_perm, const float* Y_shared, const int32_t* row_of,
@@ -506,6 +526,15 @@ moe_status moe_forward_profiled(const moe_shape* shape, const void* x, const voi
     if (!stage_events[i]) return MOE_ERR_INVALID_ARG;
   return forward_impl(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out,
                       counts_out, ws, ws_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events));
+}
+
+moe_status moe_forward_ep(const moe_shape* shape, int ep_rank, int ep_size, const void* x, const void* Wg,
+                          const float* bias, const void* W1, const void* W3, const void* W2, const float* s1,
+                          const float* s3, const float* s2, const void* W1s, const void* W3s, const void* W2s, void* y,
+                          int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes,
+                          void* stream) {
+  return forward_impl(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out,
+                      counts_out, ws, ws_bytes, stream, nullptr, ep_rank, ep_size);
 }
 
 moe_status moe_check_device_status(const void* ws, void* stream, uint32_t* raw) {

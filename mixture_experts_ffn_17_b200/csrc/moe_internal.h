@@ -67,17 +67,25 @@ cudaError_t launch_router_topk(float* logits, const double* part, int splits, co
 cudaError_t launch_expert_utilisation(const int32_t* counts, int E, float* util, int32_t* flags,
                                       cudaStream_t stream);
 
+// The routed experts one call computes: [e_lo, e_hi), on every token routed
+// to them.  The whole layer is {0, E}; an expert-parallel rank takes its slice.
+struct Shard {
+  int e_lo, e_hi;
+};
+
 // permute.cu
 int permute_blocks(int64_t T);
 cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int32_t* hist, int32_t* base,
                            int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* row_of,
                            uint32_t* status, cudaStream_t stream);
+// offsets != nullptr: only permuted rows of experts [e_lo, e_hi) are copied.
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t rows, int d, void* x_perm,
-                               int num_sms, cudaStream_t stream);
+                               int num_sms, cudaStream_t stream, const int32_t* offsets = nullptr, int e_lo = 0,
+                               int e_hi = 0);
 // Also zeroes the grouped GEMMs' tile counters (kNumSchedCounters ints).
 constexpr int kNumSchedCounters = 4;
-cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, bool with_shared, int4* tiles,
-                               int32_t* ntiles, int* sched_counters, cudaStream_t stream);
+cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, const Shard& shard, bool with_shared,
+                               int4* tiles, int32_t* ntiles, int* sched_counters, cudaStream_t stream);
 
 // grouped_gemm.cu
 // Which part of the tile list a grouped-GEMM launch walks.
@@ -89,6 +97,7 @@ struct GemmParams {
   int max_mtiles;         // capacity of the tile list (clamps the device counts)
   int tile_set;           // TileSet
   int E;                  // group index E = shared expert
+  int group_base;         // routed group g uses weight (and scale) slice g - group_base
   int n_nb;               // N blocks per tile row (max over routed / shared)
   int K_routed, K_shared;
   int N_routed, N_shared;
@@ -124,7 +133,10 @@ cudaError_t launch_grouped_down_fp8(const CUtensorMap& tmA, const CUtensorMap& t
                                     cudaStream_t stream);
 
 // combine.cu
+// offsets != nullptr: only permuted rows of experts [shard.e_lo, shard.e_hi)
+// are added.
 cudaError_t launch_combine(const void* Y_perm, const float* Y_shared, const int32_t* row_of, const float* topk_w,
-                           int64_t T, int k, int d, void* y, bool y_bf16, cudaStream_t stream);
+                           int64_t T, int k, int d, void* y, bool y_bf16, cudaStream_t stream,
+                           const int32_t* offsets = nullptr, const Shard* shard = nullptr);
 
 }  // namespace moe

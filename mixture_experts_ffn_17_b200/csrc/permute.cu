@@ -1,7 +1,7 @@
 // permute.cu -- token-to-expert dispatch without a host round trip.
 //
 // The atlas page's MoE forward ("DeepSeek-V3.2-Exp / Mixture of experts",
-// model.py 790-803 excerpt) counts assignments with bincount(indices,
+// "Code" section, MoE forward block) counts assignments with bincount(indices,
 // minlength=E), copies the counts to the host and, for each expert, gathers
 // the tokens that chose it with torch.where(indices == e), i.e. in ascending
 // (token, slot) order.  Here the same order is built on the device as a stable
@@ -168,9 +168,13 @@ constexpr int kGatherUnroll = 4;
 
 __global__ void __launch_bounds__(256)
     gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ perm_token, int64_t rows,
-                       int vec_per_row, uint4* __restrict__ x_perm) {
+                       int vec_per_row, uint4* __restrict__ x_perm, const int32_t* __restrict__ offsets, int e_lo,
+                       int e_hi) {
   grid_dependency_wait();
-  int64_t r = blockIdx.x;
+  // rows [r_lo, r_hi) of the permuted order: all of them, or one expert slice
+  const int64_t r_lo = offsets ? offsets[e_lo] : 0;
+  if (offsets) rows = offsets[e_hi];
+  int64_t r = r_lo + blockIdx.x;
   if (r >= rows) return;
   int32_t t = perm_token[r];
   for (; r < rows; r += gridDim.x) {
@@ -196,11 +200,11 @@ __global__ void __launch_bounds__(256)
 }
 
 // Tile list for the grouped GEMMs: one int4 {group, row_start, rows, 0} per
-// 256-row tile of each expert segment (group e, rows in permuted order), then
-// the shared expert's tiles (group E, rows in token order).  ntiles[0] = all
-// tiles, ntiles[1] = routed tiles.
-__global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, int T, int with_shared,
-                                   int4* __restrict__ tiles, int32_t* __restrict__ ntiles,
+// 256-row tile of each expert segment of [e_lo, e_hi) (group e, rows in
+// permuted order), then the shared expert's tiles (group E, rows in token
+// order).  ntiles[0] = all tiles, ntiles[1] = routed tiles.
+__global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, int e_lo, int e_hi, int T,
+                                   int with_shared, int4* __restrict__ tiles, int32_t* __restrict__ ntiles,
                                    int* __restrict__ sched_counters) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t total;
@@ -208,7 +212,7 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
   const int lane = e & 31, warp = e >> 5;
   int32_t start = 0, cnt = 0, mt = 0;
   grid_dependency_wait();
-  if (e < E) {
+  if (e >= e_lo && e < e_hi) {
     start = offsets[e];
     cnt = offsets[e + 1] - start;
     mt = (cnt + kTileRows - 1) / kTileRows;
@@ -277,20 +281,21 @@ cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int32_t*
 }
 
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t rows, int d, void* x_perm,
-                               int num_sms, cudaStream_t stream) {
+                               int num_sms, cudaStream_t stream, const int32_t* offsets, int e_lo, int e_hi) {
   if (rows == 0) return cudaSuccess;
   const int64_t g = std::min<int64_t>(rows, (int64_t)num_sms * 16);
   const cudaError_t err = launch_chained(gather_rows_kernel, dim3((unsigned)g), dim3(256), 0, stream,
                                          static_cast<const uint4*>(x), perm_token, rows, d / 8,
-                                         static_cast<uint4*>(x_perm));
+                                         static_cast<uint4*>(x_perm), offsets, e_lo, e_hi);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
-cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, bool with_shared, int4* tiles,
-                               int32_t* ntiles, int* sched_counters, cudaStream_t stream) {
+cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, const Shard& shard, bool with_shared,
+                               int4* tiles, int32_t* ntiles, int* sched_counters, cudaStream_t stream) {
   const int threads = ((E + 31) / 32) * 32;
-  const cudaError_t err = launch_chained(build_tiles_kernel, dim3(1), dim3(threads < 32 ? 32 : threads), 0, stream,
-                                         offsets, E, (int)T, with_shared ? 1 : 0, tiles, ntiles, sched_counters);
+  const cudaError_t err =
+      launch_chained(build_tiles_kernel, dim3(1), dim3(threads < 32 ? 32 : threads), 0, stream, offsets, E, shard.e_lo,
+                     shard.e_hi, (int)T, with_shared ? 1 : 0, tiles, ntiles, sched_counters);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

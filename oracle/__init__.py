@@ -13,7 +13,7 @@ helpers written in the order of the pages' definitions:
   in one diagram", simplified block pseudocode);
 * bincount + per-expert token lists in token order, y += w * expert(x),
   y += shared(x) (atlas page "DeepSeek-V3.2-Exp / Mixture of experts / Shared
-  expert", model.py 790-803 excerpt);
+  expert", "Code" section, MoE forward block);
 * SwiGLU g=xW1, u=xW3, a=g*sigmoid(g), h=a*u, y=hW2 (same atlas page, "All 5
   steps");
 * sigmoid group-limited routing with selection bias (the FP8 group-routing
@@ -69,11 +69,14 @@ def lib():
             "oracle_expert_utilisation": [i32, P, P, P],
             "oracle_moe_forward": [i64, i64, i32, i32, i64, i64, i32, i32, i32, i32, f64,
                                    P, P, P, P, P, P, P, P, P, P, P, P, P, P],
+            "oracle_moe_forward_ep_rank": [i64, i64, i32, i32, i64, i64, i32, i32, i32, i32, f64,
+                                           P, P, P, i32, i32, P, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
             fn.argtypes = args
-            fn.restype = ctypes.c_int if name in ("oracle_dispatch", "oracle_moe_forward") else None
+            fn.restype = ctypes.c_int if name in ("oracle_dispatch", "oracle_moe_forward",
+                                                  "oracle_moe_forward_ep_rank") else None
         L.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_value.restype = ctypes.c_double
         _lib = L
@@ -274,3 +277,42 @@ def moe_forward(x, Wg, W1, W3, W2, W1s=None, W3s=None, W2s=None, *, k: int, rout
     if rc != 0:
         raise MemoryError("oracle_moe_forward: allocation failed")
     return y, idx, w, lg
+
+
+# ------------------------------------------------------- expert parallelism
+def ep_partition(E: int, Is: int, rank: int, size: int):
+    """Rank `rank` of `size` holds experts [e_lo, e_hi) and the shared expert's
+    hidden features [i_lo, i_hi) (atlas page, "Code" section, MoE constructor
+    block: n_local_experts = E // world_size, experts_start_idx = rank *
+    n_local_experts; the shared MLP's W1/W3 are column-parallel and its W2
+    row-parallel, so each rank holds an even slice of its hidden features)."""
+    el, il = E // size, Is // size
+    return rank * el, (rank + 1) * el, rank * il, (rank + 1) * il
+
+
+def moe_forward_ep_rank(x, Wg, W1l, W3l, W2l, W1sl=None, W3sl=None, W2sl=None, *, e_lo: int, k: int,
+                        route: int = 0, bias=None, n_group: int = 1, topk_group: int = 1, group_topn: int = 2,
+                        route_scale: float = 2.5) -> np.ndarray:
+    """One rank's partial y of the expert-parallel layer: its experts' weighted
+    outputs (W1l/W3l/W2l hold experts e_lo, e_lo+1, ...) plus its slice of the
+    shared expert (W1sl [d, Isl], W3sl [d, Isl], W2sl [Isl, d]); the all-reduce
+    of these over the ranks is the layer (atlas page, "Code" section, MoE
+    forward block)."""
+    x, Wg, W1l, W3l, W2l = (_c(a, np.float64) for a in (x, Wg, W1l, W3l, W2l))
+    T, d = x.shape
+    E = Wg.shape[0]
+    El, _, I = W1l.shape
+    if W1sl is None or W1sl.shape[1] == 0:
+        Isl = 0
+        W1sl = W3sl = W2sl = np.zeros(1)
+    else:
+        Isl = W1sl.shape[1]
+    W1sl, W3sl, W2sl = (_c(a, np.float64) for a in (W1sl, W3sl, W2sl))
+    b = None if bias is None else _c(bias, np.float64)
+    y = np.empty((T, d), dtype=np.float64)
+    rc = lib().oracle_moe_forward_ep_rank(T, d, E, k, I, Isl, route, n_group, topk_group, group_topn, route_scale,
+                                          _p(x), _p(Wg), _p(b), e_lo, El, _p(W1l), _p(W3l), _p(W2l), _p(W1sl),
+                                          _p(W3sl), _p(W2sl), _p(y))
+    if rc != 0:
+        raise MemoryError("oracle_moe_forward_ep_rank: allocation failed")
+    return y

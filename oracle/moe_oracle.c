@@ -22,7 +22,7 @@
  *  - "DeepSeek-V3.2-Exp / Mixture of experts / Shared expert" (atlas page),
  *    the five SwiGLU steps g=xW1, u=xW3, a=g*sigmoid(g), h=a*u, y=hW2, the
  *    per-instance parameter table (3 x 7168 x 2048 = 44,040,192), and the
- *    MoE forward excerpt (model.py 790-803): bincount of indices, a per-expert
+ *    MoE forward block of its "Code" section: bincount of indices, a per-expert
  *    gather of the tokens that chose it in token order, y[idx] += expert(x)
  *    * weight in an fp32 accumulator, then y += shared_experts(x).
  *  - The group-limited sigmoid routing with a selection bias (config "group
@@ -409,8 +409,8 @@ ORACLE_EXPORT int oracle_moe_forward(int64_t T, int64_t d, int E, int k, int64_t
 /* ------------------------------------------------------------------------ */
 /* Combine step alone: y[t] = sum_j w[t,j] * Yp[row_of[t*k+j]] + Ys[t]        */
 /* (the y[idx] += expert_out * weight accumulation of the atlas page's       */
-/* model.py 790-803 excerpt, then y += shared).  Ys may be NULL.  Rows with   */
-/* row_of < 0 are skipped.                                                    */
+/* "Code" section, MoE forward block, then y += shared).  Ys may be NULL.    */
+/* Rows with row_of < 0 are skipped.                                          */
 /* ------------------------------------------------------------------------ */
 ORACLE_EXPORT void oracle_combine(int64_t T, int k, int64_t d, const double *Yp, const double *Ys,
                                   const int32_t *row_of, const double *w, double *y)
@@ -463,4 +463,58 @@ ORACLE_EXPORT void oracle_expert_utilisation(int E, const int32_t *counts, doubl
         util[e] = total > 0 ? (double)c / (double)total : 0.0;
         flag[e] = (c * E > 2 * total) ? 1 : ((10 * c * E < total) ? -1 : 0);
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* One rank's share of the expert-parallel layer (atlas page, "Code"         */
+/* section: the MoE constructor block gives rank r the experts                */
+/* [r*E/size, (r+1)*E/size) and a shared-expert MLP whose W1/W3 are column-  */
+/* parallel and whose W2 is row-parallel without an output reduction; the    */
+/* MoE forward block adds the local experts' weighted outputs and the shared  */
+/* MLP's output into y, then all-reduces y over the ranks).                   */
+/*   W1l, W3l [El, d, I], W2l [El, I, d]: the rank's experts, slice 0 is     */
+/*     expert e_lo;                                                          */
+/*   W1sl, W3sl [d, Isl], W2sl [Isl, d]: the rank's hidden features of the   */
+/*     shared expert (Isl may be 0);                                         */
+/*   y[t] = sum_{j: e_lo <= idx[t,j] < e_lo+El} w[t,j] expert(x[t])           */
+/*        + W2sl(silu(x[t] W1sl) * (x[t] W3sl)).                             */
+/* Routing is over all E experts, as every rank routes every token.          */
+/* ------------------------------------------------------------------------ */
+ORACLE_EXPORT int oracle_moe_forward_ep_rank(int64_t T, int64_t d, int E, int k, int64_t I, int64_t Isl,
+                                             int route, int n_group, int topk_group, int group_topn,
+                                             double route_scale, const double *x, const double *Wg,
+                                             const double *bias, int e_lo, int El, const double *W1l,
+                                             const double *W3l, const double *W2l, const double *W1sl,
+                                             const double *W3sl, const double *W2sl, double *y)
+{
+    double *logits = (double *)malloc(sizeof(double) * T * E);
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * T * k);
+    double *w = (double *)malloc(sizeof(double) * T * k);
+    double *o = (double *)malloc(sizeof(double) * d);
+    if (!logits || !idx || !w || !o) { free(logits); free(idx); free(w); free(o); return -1; }
+
+    oracle_logits(T, d, E, x, Wg, logits);
+    if (route == 0)
+        oracle_route_topk_softmax(T, E, k, logits, idx, w, NULL);
+    else
+        oracle_route_sigmoid_group(T, E, k, n_group, topk_group, group_topn, route_scale,
+                                   logits, bias, idx, w, NULL, NULL);
+
+    for (int64_t i = 0; i < T * d; ++i) y[i] = 0.0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[t * k + j];
+            if (e < e_lo || e >= e_lo + El) continue;  /* another rank's expert */
+            const int64_t el = e - e_lo;
+            const double wj = w[t * k + j];
+            oracle_swiglu_rows(1, d, I, x + t * d, W1l + el * d * I, W3l + el * d * I, W2l + el * I * d, o);
+            for (int64_t c = 0; c < d; ++c) y[t * d + c] += wj * o[c];
+        }
+    if (Isl > 0)
+        for (int64_t t = 0; t < T; ++t) {
+            oracle_swiglu_rows(1, d, Isl, x + t * d, W1sl, W3sl, W2sl, o);
+            for (int64_t c = 0; c < d; ++c) y[t * d + c] += o[c];
+        }
+    free(logits); free(idx); free(w); free(o);
+    return 0;
 }

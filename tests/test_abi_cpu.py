@@ -157,3 +157,19 @@ def test_binding_refuses_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         B.lib()
+
+
+def test_forward_ep_validation_without_gpu():
+    L = B.lib()
+    s = B.make_shape(T=128, d=512, E=32, k=4, inter=256, shared_inter=256)
+    keep, p = _fake()
+    n = B.workspace_size(s)
+    nul = None
+    args = [p, p, nul, p, p, p, nul, nul, nul, p, p, p, p, nul, nul, nul, p, n, nul]
+    assert L.moe_forward_ep(ctypes.byref(s), 0, 0, *args) == B.MOE_ERR_INVALID_ARG     # no ranks
+    assert L.moe_forward_ep(ctypes.byref(s), 2, 2, *args) == B.MOE_ERR_INVALID_ARG     # rank out of range
+    assert L.moe_forward_ep(ctypes.byref(s), -1, 2, *args) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_forward_ep(ctypes.byref(s), 0, 3, *args) == B.MOE_ERR_UNSUPPORTED     # 32 experts over 3 ranks
+    assert L.moe_forward_ep(ctypes.byref(s), 0, 4, *args) == B.MOE_ERR_UNSUPPORTED     # shared slice of 64 features
+    s0 = B.make_shape(T=0, d=512, E=32, k=4, inter=256, shared_inter=256)
+    assert L.moe_forward_ep(ctypes.byref(s0), 1, 2, *args) == B.MOE_OK                 # empty batch

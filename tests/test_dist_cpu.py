@@ -89,3 +89,48 @@ def test_single_process_dist_is_a_no_op():
         for k, v in env_keep.items():
             if v is not None:
                 os.environ[k] = v
+
+
+def test_expert_parallel_split_and_all_reduce_gloo():
+    # each rank slices the full weights with the package's shard_weights, runs
+    # its share of the layer (here the oracle's per-rank forward stands in for
+    # the GPU kernels), and all_reduce_partial sums the shares: every rank then
+    # holds the whole layer's output
+    outs = _run_ranks("""
+        import datetime
+        import numpy as np, torch, torch.distributed as dist
+        import oracle
+        from mixture_experts_ffn_17_b200 import expert_parallel as ep
+        dist.init_process_group("gloo", init_method="env://", timeout=datetime.timedelta(seconds=60))
+        r, W = dist.get_rank(), dist.get_world_size()
+        rng = np.random.default_rng(7)            # same draws on every rank
+        T, d, E, k, I, Is = 20, 16, 8, 3, 12, 8
+        x = rng.standard_normal((T, d)); Wg = rng.standard_normal((E, d))
+        W1, W3 = rng.standard_normal((E, d, I)) * .3, rng.standard_normal((E, d, I)) * .3
+        W2 = rng.standard_normal((E, I, d)) * .3
+        W1s, W3s, W2s = rng.standard_normal((d, Is)) * .3, rng.standard_normal((d, Is)) * .3, rng.standard_normal((Is, d)) * .3
+        t = torch.from_numpy
+        w = ep.shard_weights(t(W1), t(W3), t(W2), None, None, None, t(W1s), t(W3s), t(W2s), r, W)
+        sl = ep.ep_slice(E, Is, r, W)
+        y = t(oracle.moe_forward_ep_rank(x, Wg, w.W1.numpy(), w.W3.numpy(), w.W2.numpy(), w.W1s.numpy(),
+                                         w.W3s.numpy(), w.W2s.numpy(), e_lo=sl.e_lo, k=k))
+        ep.all_reduce_partial(y)
+        y_full, *_ = oracle.moe_forward(x, Wg, W1, W3, W2, W1s, W3s, W2s, k=k)
+        err = float(np.abs(y.numpy() - y_full).max() / np.sqrt(np.mean(y_full ** 2)))
+        print("RESULT", r, sl.e_lo, sl.e_hi, sl.i_lo, sl.i_hi, err)
+        dist.destroy_process_group()
+    """)
+    for rc, o, e in outs:
+        assert rc == 0, e
+    res = sorted(l.split()[1:] for _, o, _ in outs for l in o.splitlines() if l.startswith("RESULT"))
+    assert [v[:5] for v in res] == [["0", "0", "4", "0", "4"], ["1", "4", "8", "4", "8"]]
+    assert all(float(v[5]) <= 1e-12 for v in res)
+
+
+def test_ep_slice_rejects_uneven_splits():
+    from mixture_experts_ffn_17_b200 import expert_parallel as ep
+    with pytest.raises(ValueError):
+        ep.ep_slice(256, 2048, 0, 3)
+    with pytest.raises(ValueError):
+        ep.ep_slice(256, 2048, 2, 2)
+    assert ep.ep_slice(256, 2048, 7, 8) == ep.EpSlice(224, 256, 1792, 2048)

@@ -186,6 +186,30 @@ def test_grouped_swiglu_oversize_and_empty_segments():
     _experts_case(w, idx)
 
 
+# segment sizes around the tile-half boundaries: <= 64 rows runs as an M=64
+# MMA, 65-128 as one M=128 half, 129-192 as a full half plus an M=64 half,
+# 193-256 as two full halves, more as several tiles; 0 = empty expert
+HALF_BOUNDARY_COUNTS = [1, 63, 64, 65, 127, 128, 129, 191, 192, 193, 255, 256, 257, 320, 385, 0, 2]
+
+
+def _boundary_idx(E):
+    counts = HALF_BOUNDARY_COUNTS + [0] * (E - len(HALF_BOUNDARY_COUNTS))
+    idx = np.repeat(np.arange(E, dtype=np.int32), counts)
+    np.random.default_rng(5).shuffle(idx)  # tokens of one expert are not contiguous
+    return idx[:, None]
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_grouped_swiglu_tile_half_boundaries(fp8):
+    T = sum(HALF_BOUNDARY_COUNTS)
+    if fp8:
+        w = to_device(workloads.make_small("fp8", T=T, d=256, E=32, k=1, inter=128, shared_inter=128, n_group=4,
+                                           topk_group=2))
+    else:
+        w = to_device(workloads.make_small("prefill", T=T, d=256, E=32, k=1, inter=128, shared_inter=128))
+    _experts_case(w, _boundary_idx(32))
+
+
 def test_grouped_swiglu_no_shared_expert():
     w = _medium(T=300, shared_inter=0)
     lg = oracle.logits(dec(w.x), dec(w.Wg))
@@ -378,3 +402,44 @@ def test_expert_utilisation_of_a_forward_pass():
     c, _, _, _ = oracle.dispatch(to_np(idx), w.cfg.E)
     u_o, _ = oracle.expert_utilisation(c)
     assert np.allclose(to_np(util), u_o, rtol=1e-6) and abs(float(util.sum()) - 1.0) < 1e-5
+
+
+# ------------------------------------------------- expert parallelism (next row)
+@pytest.mark.parametrize("fp8,world", [(False, 2), (False, 4), (True, 2)])
+def test_forward_expert_parallel_shares_sum_to_the_layer(fp8, world):
+    # every rank's share on this one GPU in turn (the all-reduce is the sum):
+    # the sum matches the whole-layer launch up to fp32 summation order and
+    # the oracle within the layer's tolerance
+    from mixture_experts_ffn_17_b200 import expert_parallel as ep
+    w = _fp8() if fp8 else _medium(shared_inter=512)
+    cfg = w.cfg
+    y_full, idx, tw, counts, ws = run_forward(w)
+    shape = B.shape_of(cfg)
+    acc = torch.zeros_like(y_full)
+    for r in range(world):
+        wr = ep.shard_weights(w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s, r, world)
+        y_r = torch.empty_like(y_full)
+        idx_r = torch.empty_like(idx)
+        B.forward_ep(shape, r, world, w.x, w.Wg, w.bias, wr.W1, wr.W3, wr.W2, wr.s1, wr.s3, wr.s2, wr.W1s, wr.W3s,
+                     wr.W2s, y_r, ws, topk_idx=idx_r)
+        rc, raw = B.check_device_status(ws)
+        assert rc == B.MOE_OK, raw
+        assert torch.equal(idx_r, idx)  # every rank routes every token the same way
+        acc += y_r
+    rms = float(y_full.double().pow(2).mean().sqrt())
+    assert float((acc - y_full).abs().max()) <= 1e-4 * rms
+    y_o, _, _, lg = oracle_full(w)
+    _, _, merged, report = route_with_exemptions(w, lg, to_np(idx))
+    if report:
+        y_o, *_ = oracle_full(w, force_idx=merged)
+    assert max_rel_err(to_np(acc).astype(np.float64), y_o) <= (TOL_FP8 if fp8 else TOL_BF16)
+
+
+def test_forward_expert_parallel_one_rank_is_the_layer():
+    w = _tiny()
+    y_full, idx, tw, counts, ws = run_forward(w)
+    y1 = torch.empty_like(y_full)
+    B.forward_ep(B.shape_of(w.cfg), 0, 1, w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s,
+                 w.W2s, y1, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y_full)

@@ -33,6 +33,9 @@ MUTANTS = {
     "group score top-1": ("for (int i = 0; i < group_topn; ++i) acc += sel[inner[i]];",
                           "for (int i = 0; i < group_topn; ++i) acc = sel[inner[i]];"),
     "softmax not shifted by max": ("den += exp(l[top[j]] - l[top[0]]);", "den += exp(l[top[j]] - l[top[1 % k]]);"),
+    "expert-parallel rank skips its first expert": ("if (e < e_lo || e >= e_lo + El) continue;",
+                                                    "if (e <= e_lo || e >= e_lo + El) continue;"),
+    "expert-parallel rank drops its shared slice": ("    if (Isl > 0)\n", "    if (0)\n"),
     "combine drops shared": ("        if (Ys)\n            for (int64_t c = 0; c < d; ++c) yt[c] += Ys[t * d + c];",
                              "        if (0)\n            for (int64_t c = 0; c < d; ++c) yt[c] += Ys[t * d + c];"),
 }

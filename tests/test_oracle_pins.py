@@ -445,3 +445,68 @@ def test_expert_utilisation_definition_cases():
     # uniform load: nothing flagged, utilisation 1/E
     u, f = oracle.expert_utilisation(np.full(16, 7, dtype=np.int32))
     assert np.allclose(u, 1 / 16) and np.all(f == 0)
+
+
+# ------------------------------------------------------- expert parallelism
+def _ep_problem(seed, T=24, d=16, E=8, k=3, I=12, Is=8):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, d))
+    Wg = rng.standard_normal((E, d))
+    W1, W3 = rng.standard_normal((E, d, I)) * 0.3, rng.standard_normal((E, d, I)) * 0.3
+    W2 = rng.standard_normal((E, I, d)) * 0.3
+    W1s, W3s, W2s = rng.standard_normal((d, Is)) * 0.3, rng.standard_normal((d, Is)) * 0.3, \
+        rng.standard_normal((Is, d)) * 0.3
+    return x, Wg, W1, W3, W2, W1s, W3s, W2s
+
+
+def _ep_sum(x, Wg, W1, W3, W2, W1s, W3s, W2s, size, **kw):
+    E, Is = W1.shape[0], W1s.shape[1]
+    acc = np.zeros_like(x)
+    for r in range(size):
+        a, b, i0, i1 = oracle.ep_partition(E, Is, r, size)
+        acc += oracle.moe_forward_ep_rank(x, Wg, W1[a:b], W3[a:b], W2[a:b], W1s[:, i0:i1], W3s[:, i0:i1],
+                                          W2s[i0:i1], e_lo=a, **kw)
+    return acc
+
+
+@pytest.mark.parametrize("route", [0, 1])
+def test_expert_parallel_ranks_sum_to_the_layer(route):
+    # the all-reduce of the ranks' partial outputs is the layer: every routed
+    # slot is owned by exactly one rank and the shared expert's hidden
+    # features are split without overlap (SwiGLU is a sum over them)
+    p = _ep_problem(3)
+    kw = dict(k=3, route=route)
+    if route == 1:
+        kw.update(bias=np.random.default_rng(4).standard_normal(8) * 0.1, n_group=4, topk_group=2, group_topn=2,
+                  route_scale=2.5)
+    y_full, *_ = oracle.moe_forward(*p, **kw)
+    rms = np.sqrt(np.mean(y_full ** 2))
+    for size in (2, 4, 8):
+        assert np.abs(_ep_sum(*p, size, **kw) - y_full).max() <= 1e-12 * rms
+    # one rank is the layer itself, bit for bit
+    assert np.array_equal(_ep_sum(*p, 1, **kw), y_full)
+
+
+def test_expert_parallel_partition_covers_each_expert_once():
+    for E, Is, size in ((256, 2048, 8), (8, 8, 4), (32, 0, 2)):
+        seen_e, seen_i = [], []
+        for r in range(size):
+            a, b, i0, i1 = oracle.ep_partition(E, Is, r, size)
+            seen_e += list(range(a, b))
+            seen_i += list(range(i0, i1))
+        assert seen_e == list(range(E)) and seen_i == list(range(Is))
+
+
+def test_expert_parallel_rank_without_routed_tokens_is_its_shared_slice():
+    # experts 4..7 (rank 1 of 2) get logit -500 on every token, so no slot is
+    # theirs and rank 1's partial is exactly its slice of the shared expert
+    x, Wg, W1, W3, W2, W1s, W3s, W2s = _ep_problem(5)
+    x[:, 0] = 5.0
+    Wg[4:] = 0.0
+    Wg[4:, 0] = -100.0
+    idx, _, _ = oracle.route_topk_softmax(oracle.logits(x, Wg), 3)
+    assert (idx < 4).all()
+    a, b, i0, i1 = oracle.ep_partition(8, 8, 1, 2)
+    y1 = oracle.moe_forward_ep_rank(x, Wg, W1[a:b], W3[a:b], W2[a:b], W1s[:, i0:i1], W3s[:, i0:i1], W2s[i0:i1],
+                                    e_lo=a, k=3)
+    assert np.array_equal(y1, oracle.swiglu_rows(x, W1s[:, i0:i1], W3s[:, i0:i1], W2s[i0:i1]))
