@@ -51,6 +51,10 @@ def parse_args():
     p.add_argument("--cpu-sample", type=int, default=16, help="tokens the CPU baseline runs through the oracle")
     p.add_argument("--ref-sample", type=int, default=2, help="tokens per step of the reference arm")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--ep-size", type=int, default=1,
+                   help="expert-parallel layer over this many ranks (moe_forward_ep + an all-reduce of y)")
+    p.add_argument("--ep-rank", type=int, default=0,
+                   help="with one process and --ep-size > 1: the rank whose share is timed")
     return p.parse_args()
 
 
@@ -417,6 +421,102 @@ def run_ours(args, dist):
         print(json.dumps(line), flush=True)
 
 
+def run_ep(args, dist):
+    """Expert-parallel layer (moe_forward_ep): rank r of --ep-size holds E/n
+    experts and its slice of the shared expert's hidden features; every step
+    runs the rank's share and all-reduces y over the ranks (NCCL), both inside
+    the timed region.  With one process only one share can run: --ep-rank picks
+    it, there is no all-reduce, and the value is that share's tokens/s."""
+    from mixture_experts_ffn_17_b200 import binding as B
+    from mixture_experts_ffn_17_b200 import expert_parallel as ep
+    from mixture_experts_ffn_17_b200 import workloads
+
+    n = args.ep_size
+    if dist.world not in (1, n):
+        raise SystemExit(f"--ep-size {n} needs {n} ranks (or one process timing one share)")
+    rank = dist.rank if dist.world == n else args.ep_rank
+    dev = torch.device("cuda", dist.local)
+    torch.cuda.set_device(dev)
+    cfg = workloads.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = cfg.replace(T=args.tokens)
+    if args.experts:
+        cfg = cfg.replace(E=args.experts)
+    w = workloads.make(cfg, device=dev)
+    wr = ep.shard_weights(w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s, rank, n)
+    sl = ep.ep_slice(cfg.E, cfg.shared_inter, rank, n)
+    w.W1 = w.W3 = w.W2 = w.s1 = w.s3 = w.s2 = None  # only the rank's share stays resident
+    torch.cuda.empty_cache()
+    shape = B.shape_of(cfg, B.MOE_F32)
+    ws = B.alloc_workspace(shape, dev)
+    y = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device=dev)
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ep.forward(shape, rank, n, w.x, w.Wg, w.bias, wr, y, ws, counts=counts)
+
+    for _ in range(args.warmup):
+        step()
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"device status after warm-up (raw {raw})")
+    K = args.steps
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        start.record(stream)
+        for _ in range(K):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier()
+    ms_max = dist.max(start.elapsed_time(end) / K)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"device status after the timed steps (raw {raw})")
+
+    # the share's algorithmic work: router on every token, the rank's touched
+    # experts on their rows, its shared-expert slice on every token
+    c = counts.cpu().numpy()
+    local_rows = int(c[sl.e_lo:sl.e_hi].sum())
+    local_touched = int((c[sl.e_lo:sl.e_hi] > 0).sum())
+    wb = 1 if cfg.fp8 else 2
+    isl = sl.i_hi - sl.i_lo
+    flops = 2 * cfg.T * cfg.d * cfg.E + local_rows * 6 * cfg.d * cfg.inter + cfg.T * 6 * cfg.d * isl
+    nbytes = (local_touched * 3 * cfg.d * cfg.inter * wb + 3 * cfg.d * isl * 2 + cfg.E * cfg.d * 2
+              + cfg.T * cfg.d * 2 + cfg.T * cfg.d * 4)
+    if cfg.fp8:
+        nbytes += local_touched * 3 * (cfg.d // 128) * (cfg.inter // 128) * 4
+    peaks, peak_src = load_peaks()
+    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": nbytes / (ms_max / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / (ms_max / 1e3) / 1e12, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "whole step of the rank's share (moe_forward_ep" + (" + all-reduce)" if dist.world > 1 else ")")
+    roof["peak_source"] = peak_src
+    conf = config_of(cfg, args)
+    conf["parallelism"] = f"ep{n}"
+    conf["ep"] = {"size": n, "rank_timed": rank if dist.world == 1 else "all", "experts": [sl.e_lo, sl.e_hi],
+                  "shared_features": [sl.i_lo, sl.i_hi], "all_reduce": dist.world > 1,
+                  "note": ("one share on one GPU; the other ranks and the all-reduce are not run"
+                           if dist.world == 1 else "all ranks, NCCL all-reduce of y every step")}
+    line = {"metric": METRIC, "value": cfg.T / (ms_max / 1e3), "unit": "tokens/s", "n_gpus": dist.world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": conf,
+            "tflops": flops / (ms_max / 1e3) / 1e12, "roofline": roof, "clocks": sampler.summary(),
+            "gpu_launches": KERNELS_PER_STEP * K}
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_e2e(args, B, fwd_args, w, cfg, y, dev, stream, dist):
     """Same metric through the public call with host buffers.  Every step
     copies its own tokens from pinned host memory, runs the layer and copies
@@ -491,6 +591,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, dist)
+        elif args.ep_size > 1:
+            run_ep(args, dist)
         else:
             run_ours(args, dist)
     finally:
