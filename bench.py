@@ -35,7 +35,6 @@ import torch  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and TFLOPS at V3 shapes (T=4096 bf16); % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 10  # router logits, top-k, hist, scan, scatter, gather, tile list, up, down, combine
 
 
 def parse_args():
@@ -412,7 +411,7 @@ def run_ours(args, dist):
                                "peaks": f"{peak_src}: hbm {peaks['hbm_gbs']} GB/s, bf16 "
                                         f"{peaks['bf16_tflops_sustained']} TF/s sustained"},
             "roofline": roof, "stage_ms": stage_ms, "clocks": sampler.summary(),
-            "gpu_launches": KERNELS_PER_STEP * K}
+            "gpu_launches": B.forward_launches(shape) * K}
     if e2e:
         line["e2e"] = e2e
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
@@ -512,7 +511,7 @@ def run_ep(args, dist):
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": conf,
             "tflops": flops / (ms_max / 1e3) / 1e12, "roofline": roof, "clocks": sampler.summary(),
-            "gpu_launches": KERNELS_PER_STEP * K}
+            "gpu_launches": B.forward_launches(shape) * K}
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
 

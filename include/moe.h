@@ -225,6 +225,11 @@ moe_status moe_forward_ep(const moe_shape* shape, int ep_rank, int ep_size, cons
                           int32_t* topk_idx_out, float* topk_w_out, int32_t* counts_out, void* ws, size_t ws_bytes,
                           void* stream);
 
+/* Number of kernel launches moe_forward (and moe_forward_ep, moe_forward_profiled)
+ * issues for this shape on the current device; -1 for an invalid shape.
+ * Profiling aid; the pages have no counterpart. */
+int moe_forward_launches(const moe_shape* shape);
+
 /* moe_forward plus per-stage timing: records the caller's CUDA events
  * (cudaEvent_t handles, created with timing enabled) on `stream` at the stage
  * boundaries, without synchronising:

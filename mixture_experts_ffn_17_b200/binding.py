@@ -23,7 +23,8 @@ MOE_ROUTE_TOPK_SOFTMAX, MOE_ROUTE_SIGMOID_GROUP = 0, 1
 
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
             "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version",
-            "moe_permute_noalloc", "moe_router_topk_limited", "moe_expert_utilisation", "moe_forward_ep")
+            "moe_permute_noalloc", "moe_router_topk_limited", "moe_expert_utilisation", "moe_forward_ep",
+            "moe_forward_launches")
 NUM_STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "experts_up", "experts_down", "combine")
 
@@ -80,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P, P]
         I = ctypes.c_int
         L.moe_forward_ep.argtypes = [S, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.moe_forward_launches.argtypes = [S]
+        L.moe_forward_launches.restype = ctypes.c_int
         L.moe_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         for fn in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward",
                    "moe_forward_profiled", "moe_forward_ep", "moe_check_device_status"):
@@ -168,6 +171,14 @@ def forward(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, ws, to
                              _ptr(s1), _ptr(s3), _ptr(s2), _ptr(W1s), _ptr(W3s), _ptr(W2s), _ptr(y), _ptr(topk_idx),
                              _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel() if ws is not None else 0,
                              _stream(stream)), "moe_forward")
+
+
+def forward_launches(shape) -> int:
+    """Kernel launches one moe_forward call issues for this shape on the current device."""
+    n = int(lib().moe_forward_launches(ctypes.byref(shape)))
+    if n < 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_forward_launches")
+    return n
 
 
 def forward_ep(shape, ep_rank, ep_size, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, ws, topk_idx=None,

@@ -6,8 +6,11 @@
 // permuted order, located through row_of) and its shared-expert row (fp32),
 // and sums them in fp32 with no atomics, so the result is deterministic:
 //   y[t] = Y_shared[t] + sum_j w[t, j] * Y_perm[row_of[t*k + j]].
-// One CTA per token; each thread owns 8 consecutive features (one 16-byte
-// vector of each routed row), so every row read is coalesced.
+// One CTA per token (per token and slice of the features when there are
+// few tokens, so that small batches still spread over the SMs); each thread
+// owns 8 consecutive features (one 16-byte vector of each routed row), so
+// every row read is coalesced.
+#include <algorithm>
 #include <cstdint>
 
 #include "common.cuh"
@@ -35,7 +38,10 @@ __global__ void __launch_bounds__(128)
   }
   __syncthreads();
   const int nv = d / 8;
-  for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+  // this CTA's slice of the row's 16-byte vectors
+  const int per = (nv + gridDim.y - 1) / gridDim.y;
+  const int v_end = min(nv, (int)(blockIdx.y + 1) * per);
+  for (int v = blockIdx.y * per + threadIdx.x; v < v_end; v += blockDim.x) {
     float acc[8];
     if (Y_shared) {
       const float4 a = Y_shared[(t * d) / 4 + 2 * v];
@@ -82,11 +88,17 @@ cudaError_t launch_combine(const void* Y_perm, const float* Y_shared, const int3
   const float4* ys = reinterpret_cast<const float4*>(Y_shared);
   const int e_lo = shard ? shard->e_lo : 0, e_hi = shard ? shard->e_hi : 0;
   if (!shard) offsets = nullptr;
+  // feature slices per token: enough CTAs for about four per SM
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = ((int64_t)4 * sms + T - 1) / T;
+  const unsigned slices = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, std::max(1, d / 8 / 128)));
+  const dim3 grid((unsigned)T, slices);
   const cudaError_t err =
-      y_bf16 ? launch_chained(combine_kernel<true>, dim3((unsigned)T), dim3(128), 0, stream, yp, ys, row_of, topk_w, k,
-                              d, y, offsets, e_lo, e_hi)
-             : launch_chained(combine_kernel<false>, dim3((unsigned)T), dim3(128), 0, stream, yp, ys, row_of, topk_w,
-                              k, d, y, offsets, e_lo, e_hi);
+      y_bf16 ? launch_chained(combine_kernel<true>, grid, dim3(128), 0, stream, yp, ys, row_of, topk_w, k, d, y,
+                              offsets, e_lo, e_hi)
+             : launch_chained(combine_kernel<false>, grid, dim3(128), 0, stream, yp, ys, row_of, topk_w, k, d, y,
+                              offsets, e_lo, e_hi);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

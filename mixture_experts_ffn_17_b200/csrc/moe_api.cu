@@ -528,6 +528,16 @@ moe_status moe_forward_profiled(const moe_shape* shape, const void* x, const voi
                       counts_out, ws, ws_bytes, stream, reinterpret_cast<const cudaEvent_t*>(stage_events));
 }
 
+int moe_forward_launches(const moe_shape* shape) {
+  if (validate_shape(shape) != MOE_OK) return -1;
+  const moe_shape& s = *shape;
+  if (s.T == 0) return 0;
+  const int splits = router_splits(s.T, s.d, s.E, std::min(num_sms(), kRouterMaxSms));
+  const int gemm_launches = (s.w_dtype == MOE_E4M3 && s.shared_inter > 0) ? 2 : 1;  // FP8: routed + shared launch
+  // router (+ split sum) + top-k, hist + scan + scatter, gather, tile list, two grouped GEMMs, combine
+  return 1 + (splits > 1 ? 1 : 0) + 1 + 3 + 1 + 1 + 2 * gemm_launches + 1;
+}
+
 moe_status moe_forward_ep(const moe_shape* shape, int ep_rank, int ep_size, const void* x, const void* Wg,
                           const float* bias, const void* W1, const void* W3, const void* W2, const float* s1,
                           const float* s3, const float* s2, const void* W1s, const void* W3s, const void* W2s, void* y,

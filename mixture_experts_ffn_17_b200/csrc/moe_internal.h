@@ -57,8 +57,8 @@ constexpr int kRouterMaxSms = 256;  // workspace is sized for router_splits(.., 
 // `part`, summed in split order by the top-k launch.
 cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E, int splits,
                                  float* logits, double* part, uint32_t* status, cudaStream_t stream);
-// part != nullptr: logits[t][e] = (float) sum_s part[s][t][e] is computed
-// (and stored to `logits`) before the selection; otherwise logits are read.
+// splits > 1: logits[t][e] = (float) sum_s part[s][t][e] is computed (and
+// stored to `logits`) first, by one more launch; otherwise logits are read.
 cudaError_t launch_router_topk(float* logits, const double* part, int splits, const float* bias,
                                const uint8_t* allowed, const RouteParams& rp, int T, int E, int k, int32_t* idx,
                                float* w, cudaStream_t stream);

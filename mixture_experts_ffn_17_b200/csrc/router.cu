@@ -17,8 +17,8 @@
 //            finished chunk is read from TMEM and added into fp64 registers,
 //            so a logit carries one fp32 rounding per 64 terms.  Without a K
 //            split the fp32 logits [T, E] are written at the end; with one,
-//            the fp64 partial sums [split, T, E] are, and kernel 2 adds them
-//            in split order.  Small batches split K so that the grid still
+//            the fp64 partial sums [split, T, E] are, and a small kernel
+//            adds them in split order (one thread per logit).  Small batches split K so that the grid still
 //            covers the device.
 // Kernel 2 (router_topk_kernel): one warp per token, k rounds of a warp
 //   arg-max on (value desc, index asc), then the weights.
@@ -199,6 +199,20 @@ __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
   }
 }
 
+// K-split gate GEMM: logits[i] = (float) sum_s part[s][i] over the T*E
+// logits, the splits added in order; one thread per logit, loads issued
+// several splits ahead of the adds.
+__global__ void __launch_bounds__(256)
+    router_split_sum_kernel(const double* __restrict__ part, int splits, int64_t n, float* __restrict__ logits) {
+  grid_dependency_wait();
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  double a = 0.0;
+#pragma unroll 8
+  for (int sp = 0; sp < splits; ++sp) a += __ldg(part + sp * n + i);
+  logits[i] = (float)a;
+}
+
 // ---------------------------------------------------------------- top-k
 struct Cand {
   float key;   // selection score
@@ -221,8 +235,7 @@ __device__ __forceinline__ Cand warp_best(Cand c) {
 // NV = values per lane (expert e lives in lane e % 32, slot e / 32).
 template <int NV>
 __global__ void __launch_bounds__(128)
-    router_topk_kernel(float* __restrict__ logits, const double* __restrict__ part, int splits,
-                       const float* __restrict__ bias, const uint8_t* __restrict__ allowed, int T, int E, int k,
+    router_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, const uint8_t* __restrict__ allowed, int T, int E, int k,
                        int route, int n_group,
                        int topk_group, int group_topn, float route_scale, int32_t* __restrict__ topk_idx,
                        float* __restrict__ topk_w) {
@@ -236,23 +249,13 @@ __global__ void __launch_bounds__(128)
 
   float key[NV], aux[NV];
   uint32_t taken = 0;  // bit v: slot v of this lane is out of the running
-  float* lrow = logits + (size_t)t * E;
+  const float* lrow = logits + (size_t)t * E;
 #pragma unroll
   for (int v = 0; v < NV; ++v) {
     const int e = v * 32 + lane;
     if (e < E) {
-      float l0;
-      if (part) {
-        // K-split gate GEMM: add the fp64 partial sums in split order
-        double a = 0.0;
-        for (int sp = 0; sp < splits; ++sp) a += part[((size_t)sp * T + t) * E + e];
-        l0 = (float)a;
-        lrow[e] = l0;
-      } else {
-        l0 = lrow[e];
-      }
       // device-limited routing: experts this device does not hold get -inf
-      const float l = (allowed && !allowed[e]) ? NEG : l0;
+      const float l = (allowed && !allowed[e]) ? NEG : lrow[e];
       if (route == 0) {
         key[v] = l;
         aux[v] = l;
@@ -363,11 +366,11 @@ cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_
 }
 
 template <int NV>
-cudaError_t launch_topk_nv(float* logits, const double* part, int splits, const float* bias, const uint8_t* allowed,
-                           const RouteParams& rp, int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream) {
+cudaError_t launch_topk_nv(const float* logits, const float* bias, const uint8_t* allowed, const RouteParams& rp,
+                           int T, int E, int k, int32_t* idx, float* w, cudaStream_t stream) {
   const cudaError_t err =
-      launch_chained(router_topk_kernel<NV>, dim3((T + 3) / 4), dim3(128), 0, stream, logits, part, splits, bias,
-                     allowed, T, E, k, rp.route, rp.n_group, rp.topk_group, rp.group_topn, rp.route_scale, idx, w);
+      launch_chained(router_topk_kernel<NV>, dim3((T + 3) / 4), dim3(128), 0, stream, logits, bias, allowed, T, E, k,
+                     rp.route, rp.n_group, rp.topk_group, rp.group_topn, rp.route_scale, idx, w);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
@@ -404,8 +407,13 @@ cudaError_t launch_router_topk(float* logits, const double* part, int splits, co
                                const uint8_t* allowed, const RouteParams& rp, int T, int E, int k, int32_t* idx,
                                float* w, cudaStream_t stream) {
   const int nv = (E + 31) / 32;
-  if (splits <= 1) part = nullptr;
-#define MOE_TOPK(N) return launch_topk_nv<N>(logits, part, splits, bias, allowed, rp, T, E, k, idx, w, stream)
+  if (splits > 1) {
+    const int64_t n = (int64_t)T * E;
+    const cudaError_t err = launch_chained(router_split_sum_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0,
+                                           stream, part, splits, n, logits);
+    if (err != cudaSuccess) return err;
+  }
+#define MOE_TOPK(N) return launch_topk_nv<N>(logits, bias, allowed, rp, T, E, k, idx, w, stream)
   if (nv <= 1) MOE_TOPK(1);
   if (nv <= 2) MOE_TOPK(2);
   if (nv <= 4) MOE_TOPK(4);
