@@ -472,7 +472,77 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         const bool narrow = narrow_half(ti, h);
         const int r = h * kTileM + (narrow ? (lane < 16 ? q * 16 + lane : kTileM) : row);  // row within the tile
         const bool valid = r < ti.rows && (!narrow || lane < 16);
-        if (M == Mode::kSwiGLU) {
+        if constexpr (!F8) {
+          // Drain first: this warp's whole share of the slot (128 fp32 per
+          // lane: g and u of two 32-column chunks, or four W2 chunks) is read
+          // before the slot is released, so the MMA can reuse it while the
+          // stores below are still in flight.
+          static_assert(kChunks * 32 * (M == Mode::kSwiGLU ? 2 : 1) == 128, "drain-first share is 128 columns");
+          uint32_t buf[4][32];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int col = M == Mode::kSwiGLU ? (i >= 2 ? 128 : 0) + (part * kChunks + (i & 1)) * 32
+                                               : (part * kChunks + i) * 32;
+            ptx::tmem_ld32(tbase + col, buf[i]);
+          }
+          ptx::tmem_ld_wait(buf[0]);
+          ptx::tmem_ld_keep(buf[1]);
+          ptx::tmem_ld_keep(buf[2]);
+          ptx::tmem_ld_keep(buf[3]);
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&tempty[sl]);
+          if (valid) {
+            if (M == Mode::kSwiGLU) {
+              const int64_t hrow = (int64_t)ti.row0 + r + (ti.shared ? p.out_shared_row_offset : 0);
+              uint16_t* base = static_cast<uint16_t*>(ti.shared ? p.out_shared : p.out_routed);
+              uint4* out = reinterpret_cast<uint4*>(base + hrow * p.ld_out + n0);
+#pragma unroll
+              for (int cc = 0; cc < 2; ++cc) {
+                const uint32_t* g = buf[cc];
+                const uint32_t* u = buf[2 + cc];
+                uint32_t hp[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                  const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                  const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+                  const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+                  hp[i] = ptx::pack_bf16x2(h0, h1);
+                }
+                const int c = part * kChunks + cc;
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                  out[c * 4 + v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
+              }
+            } else {
+              const int64_t orow = (int64_t)ti.row0 + r + (ti.shared ? p.out_shared_row_offset : 0);
+              const int N = ti.shared ? p.N_shared : p.N_routed;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t* v32 = buf[i];
+                const int col = n0 + (part * kChunks + i) * 32;
+                if (col >= N) continue;
+                if (ti.shared) {
+                  float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.out_shared) + orow * p.ld_out + col);
+#pragma unroll
+                  for (int v = 0; v < 8; ++v)
+                    out[v] = make_float4(__uint_as_float(v32[4 * v]), __uint_as_float(v32[4 * v + 1]),
+                                         __uint_as_float(v32[4 * v + 2]), __uint_as_float(v32[4 * v + 3]));
+                } else {
+                  uint4* out =
+                      reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out_routed) + orow * p.ld_out + col);
+#pragma unroll
+                  for (int v = 0; v < 4; ++v)
+                    out[v] = make_uint4(
+                        ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 0]), __uint_as_float(v32[8 * v + 1])),
+                        ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 2]), __uint_as_float(v32[8 * v + 3])),
+                        ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 4]), __uint_as_float(v32[8 * v + 5])),
+                        ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 6]), __uint_as_float(v32[8 * v + 7])));
+                }
+              }
+            }
+          }
+        } else if (M == Mode::kSwiGLU) {
           const int64_t hrow = (int64_t)ti.row0 + r + (ti.shared ? p.out_shared_row_offset : 0);
           uint16_t* base = static_cast<uint16_t*>(ti.shared ? p.out_shared : p.out_routed);
           uint4* out = reinterpret_cast<uint4*>(base + hrow * p.ld_out + n0);

@@ -194,6 +194,16 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" : MOE_W8(0), MOE_W8(8), MOE_W8(16), MOE_W8(24)::"memory");
 }
 
+// Registers of another tcgen05.ld issued before the same wait: passed
+// through an empty asm so no use of them moves above that wait.
+__device__ __forceinline__ void tmem_ld_keep(uint32_t (&q)[32]) {
+  asm volatile("" : "+r"(q[0]), "+r"(q[1]), "+r"(q[2]), "+r"(q[3]), "+r"(q[4]), "+r"(q[5]), "+r"(q[6]),
+               "+r"(q[7]), "+r"(q[8]), "+r"(q[9]), "+r"(q[10]), "+r"(q[11]), "+r"(q[12]), "+r"(q[13]),
+               "+r"(q[14]), "+r"(q[15]), "+r"(q[16]), "+r"(q[17]), "+r"(q[18]), "+r"(q[19]), "+r"(q[20]),
+               "+r"(q[21]), "+r"(q[22]), "+r"(q[23]), "+r"(q[24]), "+r"(q[25]), "+r"(q[26]), "+r"(q[27]),
+               "+r"(q[28]), "+r"(q[29]), "+r"(q[30]), "+r"(q[31])::"memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait2(uint32_t (&r)[32], uint32_t (&q)[32]) {
   tmem_ld_wait(r);
   asm volatile("" : "+r"(q[0]), "+r"(q[1]), "+r"(q[2]), "+r"(q[3]), "+r"(q[4]), "+r"(q[5]), "+r"(q[6]),
