@@ -683,6 +683,289 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
   }
 }
 
+// ------------------------------------------------------------ CTA pairs
+// Full 256-row tiles (bf16 weights) on a 2-CTA cluster: CTA r holds rows
+// 128r..128r+127 of the tile (A) and half of its B columns (SwiGLU: CTA 0 the
+// 128 W1 columns, CTA 1 the same 128 W3 columns; down: 128 of the 256 W2
+// columns each).  CTA 0's thread issues tcgen05.mma.cta_group::2 with M=256,
+// N=256, so each weight byte is read from shared memory once per 256 rows
+// (the one-CTA kernel reads it once per 128-row half); each CTA's TMEM gets
+// its 128 rows x 256 columns, in the same column order as the one-CTA kernel
+// (SwiGLU: g then u), and each CTA's epilogue stores its own rows.  Tiles are
+// taken in a fixed order: cluster c takes tiles c, c + clusters, ...
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairABytes = kTileM * kBK * 2;  // this CTA's 128 rows
+constexpr uint32_t kPairBBytes = 2 * kBoxBytes;     // this CTA's 128 columns
+constexpr uint32_t kPairStageBytes = kPairABytes + kPairBBytes;
+constexpr int kPairEpiWarps = 8;
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
+static_assert(kBK == 64, "the pair kernel uses 64-deep K steps");
+static_assert(kPairStages * kPairStageBytes + 1024 + 256 <= 232448, "shared memory budget (pair)");
+
+constexpr size_t pair_smem_bytes() { return 1024 + kPairStages * kPairStageBytes + 256; }
+
+template <Mode M>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
+                             const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
+                             const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s,
+                             const GemmParams p) {
+  constexpr int S = kPairStages;
+  constexpr int BN = Cfg<M>::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* stage0 = align_1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(stage0 + S * kPairStageBytes);  // used on CTA 0
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* tempty = tfull + 2;  // used on CTA 0: both CTAs' epilogues arrive
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  __shared__ uint32_t never;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();  // 0: issues the MMA
+  const bool lead = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&tfull[b], 1);
+      ptx::mbar_init(&tempty[b], 2 * 32 * kPairEpiWarps);
+    }
+    ptx::mbar_init(done, 1);
+    *abort_flag = 0u;
+    never = 0u;
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // both CTAs' barriers exist before any cross-CTA arrival
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();
+
+  const TileSpan span = tile_span(p);
+  const int total = span.count * p.n_nb;
+  const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmA_r);
+      ptx::prefetch_tmap(&tmB_r);
+      ptx::prefetch_tmap(&tmA_s);
+      ptx::prefetch_tmap(&tmB_s);
+      if (M == Mode::kSwiGLU) {
+        ptx::prefetch_tmap(&tmC_r);
+        ptx::prefetch_tmap(&tmC_s);
+      }
+      const uint64_t pol_a = ptx::policy_evict_normal();
+      const uint64_t pol_w = ptx::policy_evict_first();
+      const uint64_t pol_ws = ptx::policy_evict_last();
+      int kg = 0;
+      bool ok = !p.debug_withhold_loads;
+      for (int tile = cluster; ok && tile < total; tile += clusters) {
+        TileInfo ti;
+        if (!tile_at(p, span, tile, BN, ti)) continue;
+        const uint64_t pol_b = ti.shared ? pol_ws : pol_w;
+        const CUtensorMap* mA = ti.shared ? &tmA_s : &tmA_r;
+        // SwiGLU: CTA 0 loads W1's columns, CTA 1 the same columns of W3
+        const CUtensorMap* mB = (M == Mode::kSwiGLU && rank == 1) ? (ti.shared ? &tmC_s : &tmC_r)
+                                                                   : (ti.shared ? &tmB_s : &tmB_r);
+        const int arow = ti.row0 + (ti.shared ? p.a_shared_row_offset : 0) + (int)rank * kTileM;
+        const int e3 = ti.shared ? 0 : ti.group - p.group_base;
+        const int nk = (ti.shared ? p.K_shared : p.K_routed) / kBK;
+        const int nb0 = ti.nb * BN + (M == Mode::kSwiGLU ? 0 : (int)rank * 128);  // this CTA's first B column
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % S;
+          if (!ptx::wait_bounded(&empty[s], ((kg / S) & 1) ^ 1, abort_flag)) {
+            raise_status(p.status, abort_flag, kStatusTimeout);
+            ok = false;
+            break;
+          }
+          const uint32_t bar = ptx::mapa(&full[s], 0);
+          if (lead) ptx::mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);  // both CTAs' bytes
+          uint8_t* st = stage0 + s * kPairStageBytes;
+          ptx::tma_load_2d_pair(st, mA, bar, kb * kBK, arow, pol_a);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            ptx::tma_load_3d_pair(st + kPairABytes + h * kBoxBytes, mB, bar, nb0 + 64 * h, kb * kBK, e3, pol_b);
+        }
+      }
+      // CTA 0 sees every copy of both CTAs land before the pair may exit (the
+      // final cluster barrier holds CTA 1 until then)
+      if (lead)
+        for (int j = (kg > S ? kg - S : 0); j < kg; ++j)
+          if (!ptx::wait_bounded(&full[j % S], (j / S) & 1, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && lead) {
+      constexpr uint32_t idesc = ptx::idesc_bf16(2 * kTileM, 256, false, true);
+      int kg = 0, tl = 0;
+      bool ok = true;
+      for (int tile = cluster; ok && tile < total; tile += clusters) {
+        TileInfo ti;
+        if (!tile_at(p, span, tile, BN, ti)) continue;
+        const int nk = (ti.shared ? p.K_shared : p.K_routed) / kBK;
+        const int sl = tl & 1;
+        if (!ptx::wait_bounded(&tempty[sl], ((tl >> 1) & 1) ^ 1, abort_flag)) {
+          raise_status(p.status, abort_flag, kStatusTimeout);
+          break;
+        }
+        ptx::tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % S;
+          if (!ptx::wait_bounded(&full[s], (kg / S) & 1, abort_flag)) {
+            raise_status(p.status, abort_flag, kStatusTimeout);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = ptx::smem_u32(stage0 + s * kPairStageBytes);
+          const uint32_t b0 = a0 + kPairABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            ptx::mma_bf16_pair(tmem + sl * kSlotCols, ptx::sdesc(a0 + kk * 32, 16, kASBO, kASwizzle),
+                               ptx::sdesc_sw128(b0 + kk * 2048, kBoxBytes, 1024), idesc, (kb | kk) != 0 ? 1u : 0u);
+          ptx::mma_commit_pair(&empty[s], 0x3);
+        }
+        if (!ok) break;
+        ptx::mma_commit_pair(&tfull[sl], 0x3);
+        ++tl;
+      }
+      ptx::mma_commit_pair(done, 0x1);
+      if (!ptx::wait_bounded(done, 0, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
+    }
+  } else {
+    // epilogue: this CTA's 128 rows; each lane drains its 128 columns, frees
+    // the slot on CTA 0's barrier, then computes and stores
+    constexpr int kChunks = BN / 32 / 2;  // 32-column chunks per part (two parts per lane quarter)
+    const int q = warp & 3;
+    const int part = (warp - 2) / 4;
+    const int row = (int)rank * kTileM + q * 32 + lane;  // row within the tile
+    const uint32_t tempty_lead0 = ptx::mapa(&tempty[0], 0), tempty_lead1 = ptx::mapa(&tempty[1], 0);
+    int tl = 0;
+    for (int tile = cluster; tile < total; tile += clusters) {
+      TileInfo ti;
+      if (!tile_at(p, span, tile, BN, ti)) continue;
+      const int sl = tl & 1;
+      if (!ptx::wait_bounded(&tfull[sl], (tl >> 1) & 1, abort_flag)) {
+        raise_status(p.status, abort_flag, kStatusTimeout);
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + sl * kSlotCols;
+      uint32_t buf[4][32];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int col = M == Mode::kSwiGLU ? (i >= 2 ? 128 : 0) + (part * kChunks + (i & 1)) * 32
+                                           : (part * kChunks + i) * 32;
+        ptx::tmem_ld32(tbase + col, buf[i]);
+      }
+      ptx::tmem_ld_wait(buf[0]);
+      ptx::tmem_ld_keep(buf[1]);
+      ptx::tmem_ld_keep(buf[2]);
+      ptx::tmem_ld_keep(buf[3]);
+      ptx::tc_fence_before();
+      ptx::mbar_arrive_cluster(sl ? tempty_lead1 : tempty_lead0);
+      ++tl;
+      if (row >= ti.rows) continue;
+      const int n0 = ti.nb * BN;
+      if (M == Mode::kSwiGLU) {
+        const int64_t hrow = (int64_t)ti.row0 + row + (ti.shared ? p.out_shared_row_offset : 0);
+        uint16_t* base = static_cast<uint16_t*>(ti.shared ? p.out_shared : p.out_routed);
+        uint4* out = reinterpret_cast<uint4*>(base + hrow * p.ld_out + n0);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const uint32_t* g = buf[cc];
+          const uint32_t* u = buf[2 + cc];
+          uint32_t hp[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+            hp[i] = ptx::pack_bf16x2(g0 / (1.0f + __expf(-g0)) * u0, g1 / (1.0f + __expf(-g1)) * u1);
+          }
+          const int c = part * kChunks + cc;
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            out[c * 4 + v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
+        }
+      } else {
+        const int64_t orow = (int64_t)ti.row0 + row + (ti.shared ? p.out_shared_row_offset : 0);
+        const int N = ti.shared ? p.N_shared : p.N_routed;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t* v32 = buf[i];
+          const int col = n0 + (part * kChunks + i) * 32;
+          if (col >= N) continue;
+          if (ti.shared) {
+            float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.out_shared) + orow * p.ld_out + col);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              out[v] = make_float4(__uint_as_float(v32[4 * v]), __uint_as_float(v32[4 * v + 1]),
+                                   __uint_as_float(v32[4 * v + 2]), __uint_as_float(v32[4 * v + 3]));
+          } else {
+            uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out_routed) + orow * p.ld_out + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              out[v] = make_uint4(ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 0]), __uint_as_float(v32[8 * v + 1])),
+                                  ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 2]), __uint_as_float(v32[8 * v + 3])),
+                                  ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 4]), __uint_as_float(v32[8 * v + 5])),
+                                  ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 6]), __uint_as_float(v32[8 * v + 7])));
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();  // no cross-CTA arrival or MMA operand read is still pending
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+template <Mode M>
+cudaError_t launch_pair(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtensorMap& b_r,
+                        const CUtensorMap& b_s, const CUtensorMap& c_r, const CUtensorMap& c_s, const GemmParams& p,
+                        int grid, cudaStream_t stream) {
+  const size_t smem = pair_smem_bytes();
+  cudaError_t err =
+      cudaFuncSetAttribute(grouped_gemm_pair_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  grid &= ~1;  // whole clusters
+  if (grid <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPairThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = MOE_PDL ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<M>, a_r, a_s, b_r, b_s, c_r, c_s, p);
+  return err != cudaSuccess ? err : cudaGetLastError();
+}
+
 template <Mode M, bool F8>
 cudaError_t launch(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtensorMap& b_r, const CUtensorMap& b_s,
                    const CUtensorMap& c_r, const CUtensorMap& c_s, const GemmParams& p, int grid,
@@ -712,6 +995,17 @@ cudaError_t launch_grouped_swiglu(const CUtensorMap& tmA_r, const CUtensorMap& t
 cudaError_t launch_grouped_down(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
                                 const GemmParams& p, int grid, cudaStream_t stream) {
   return launch<Mode::kDown, false>(tmA, tmA, tmW2_r, tmW2_s, tmW2_r, tmW2_s, p, grid, stream);
+}
+
+cudaError_t launch_grouped_swiglu_pair(const CUtensorMap& tmA_r, const CUtensorMap& tmA_s, const CUtensorMap& tmW1_r,
+                                       const CUtensorMap& tmW1_s, const CUtensorMap& tmW3_r, const CUtensorMap& tmW3_s,
+                                       const GemmParams& p, int grid, cudaStream_t stream) {
+  return launch_pair<Mode::kSwiGLU>(tmA_r, tmA_s, tmW1_r, tmW1_s, tmW3_r, tmW3_s, p, grid, stream);
+}
+
+cudaError_t launch_grouped_down_pair(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
+                                     const GemmParams& p, int grid, cudaStream_t stream) {
+  return launch_pair<Mode::kDown>(tmA, tmA, tmW2_r, tmW2_s, tmW2_r, tmW2_s, p, grid, stream);
 }
 
 cudaError_t launch_grouped_swiglu_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,

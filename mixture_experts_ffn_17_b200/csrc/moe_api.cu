@@ -44,7 +44,7 @@ moe_status validate_shape(const moe_shape* s) {
 }
 
 struct Layout {
-  size_t status, logits, rpart, idx, w, hist, base, counts, offsets, perm, row_of, tiles, ntiles, sched, x_perm, H, Y_perm,
+  size_t status, logits, rpart, idx, w, hist, base, counts, offsets, perm, row_of, tiles, tiles_pair, ntiles, sched, x_perm, H, Y_perm,
       Y_shared, total;
   int nb, max_mtiles, Hld;
   int64_t Hrows;
@@ -77,7 +77,8 @@ Layout make_layout(const moe_shape& s) {
   L.perm = take((size_t)Tk * 4);
   L.row_of = take((size_t)Tk * 4);
   L.tiles = take((size_t)L.max_mtiles * 16);
-  L.ntiles = take(8);
+  L.tiles_pair = take((size_t)L.max_mtiles * 16);
+  L.ntiles = take(16);
   L.sched = take(kNumSchedCounters * 4);
   L.x_perm = take((size_t)Tk * s.d * 2);
   L.H = take((size_t)L.Hrows * L.Hld * 2);
@@ -170,6 +171,18 @@ int num_sms() {
     if ((call) != cudaSuccess) return MOE_ERR_CUDA; \
   } while (0)
 
+// Full 256-row tiles run on CTA pairs (one tcgen05.mma.cta_group::2 M=256
+// per K step, B read once per 256 rows) when segments are long enough for
+// most rows to sit in full tiles: on average at least 384 rows per expert,
+// bf16 weights.  MOE_PAIR_TILES=1 / 0 in the environment forces it on / off.
+bool use_pair_tiles(const moe_shape& s) {
+  if (s.w_dtype == MOE_E4M3) return false;
+  const char* v = std::getenv("MOE_PAIR_TILES");
+  if (v && v[0] == '1') return true;
+  if (v && v[0] == '0') return false;
+  return s.T * (int64_t)s.k >= (int64_t)384 * s.E;
+}
+
 // ------------------------------------------------------------ stages
 moe_status run_router(const moe_shape& s, const void* x, const void* Wg, const float* bias, int32_t* idx, float* w,
                       float* logits, double* part, uint32_t* status, cudaStream_t st,
@@ -202,7 +215,9 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   int32_t* ntiles = at<int32_t>(ws, L.ntiles);
   uint16_t* H = at<uint16_t>(ws, L.H);
   int* sched = at<int>(ws, L.sched);
-  MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, shard, sh, tiles, ntiles, sched, st));
+  const bool pair = use_pair_tiles(s);
+  int4* tiles_pair = pair ? at<int4>(ws, L.tiles_pair) : nullptr;
+  MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, shard, sh, tiles, ntiles, sched, st, tiles_pair));
   const int E_w = shard.e_hi - shard.e_lo;  // expert slices held by the weight tensors
   if (ev) MOE_CUDA(cudaEventRecord(ev[0], st));
 
@@ -263,6 +278,12 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
       MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, q, grid1, st));
     }
   } else {
+    if (pair) {
+      GemmParams q = p1;  // full tiles on CTA pairs, then the partial tiles
+      q.tiles = tiles_pair;
+      q.ntiles = ntiles + 2;
+      MOE_CUDA(launch_grouped_swiglu_pair(a_r, a_s, w1_r, w1_s, w3_r, w3_s, q, sms, st));
+    }
     MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, p1, grid1, st));
   }
   if (ev) MOE_CUDA(cudaEventRecord(ev[1], st));
@@ -309,6 +330,12 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
       MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, q, grid2, st));
     }
   } else {
+    if (pair) {
+      GemmParams q = p2;
+      q.tiles = tiles_pair;
+      q.ntiles = ntiles + 2;
+      MOE_CUDA(launch_grouped_down_pair(h_map, w2_r, w2_s, q, sms, st));
+    }
     MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, p2, grid2, st));
   }
   if (ev) MOE_CUDA(cudaEventRecord(ev[2], st));
@@ -533,7 +560,8 @@ int moe_forward_launches(const moe_shape* shape) {
   const moe_shape& s = *shape;
   if (s.T == 0) return 0;
   const int splits = router_splits(s.T, s.d, s.E, std::min(num_sms(), kRouterMaxSms));
-  const int gemm_launches = (s.w_dtype == MOE_E4M3 && s.shared_inter > 0) ? 2 : 1;  // FP8: routed + shared launch
+  // FP8: routed + shared launch; pair tiles: pair launch + one-CTA launch
+  const int gemm_launches = ((s.w_dtype == MOE_E4M3 && s.shared_inter > 0) || use_pair_tiles(s)) ? 2 : 1;
   // router (+ split sum) + top-k, hist + scan + scatter, gather, tile list, two grouped GEMMs, combine
   return 1 + (splits > 1 ? 1 : 0) + 1 + 3 + 1 + 1 + 2 * gemm_launches + 1;
 }

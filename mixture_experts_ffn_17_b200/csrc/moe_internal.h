@@ -84,8 +84,11 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t
                                int e_hi = 0);
 // Also zeroes the grouped GEMMs' tile counters (kNumSchedCounters ints).
 constexpr int kNumSchedCounters = 4;
+// tiles_pair != nullptr: full 256-row tiles go to that list (ntiles[2], [3])
+// and only partial tiles to `tiles` (ntiles[0], [1]).
 cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, const Shard& shard, bool with_shared,
-                               int4* tiles, int32_t* ntiles, int* sched_counters, cudaStream_t stream);
+                               int4* tiles, int32_t* ntiles, int* sched_counters, cudaStream_t stream,
+                               int4* tiles_pair = nullptr);
 
 // grouped_gemm.cu
 // Which part of the tile list a grouped-GEMM launch walks.
@@ -122,6 +125,14 @@ int gemm_block_n_down();
 cudaError_t launch_grouped_swiglu(const CUtensorMap& tmA_r, const CUtensorMap& tmA_s, const CUtensorMap& tmW1_r,
                                   const CUtensorMap& tmW1_s, const CUtensorMap& tmW3_r, const CUtensorMap& tmW3_s,
                                   const GemmParams& p, int grid, cudaStream_t stream);
+// Full 256-row tiles of bf16 experts on 2-CTA clusters (tcgen05.mma
+// .cta_group::2, M=256): the tile list holds only full tiles; grid is
+// rounded down to whole clusters.
+cudaError_t launch_grouped_swiglu_pair(const CUtensorMap& tmA_r, const CUtensorMap& tmA_s, const CUtensorMap& tmW1_r,
+                                       const CUtensorMap& tmW1_s, const CUtensorMap& tmW3_r, const CUtensorMap& tmW3_s,
+                                       const GemmParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_grouped_down_pair(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
+                                     const GemmParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_grouped_down(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
                                 const GemmParams& p, int grid, cudaStream_t stream);
 // FP8 (e4m3 + 128x128 block scales) routed experts; the tensor maps of W are

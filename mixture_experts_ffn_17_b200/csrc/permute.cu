@@ -199,59 +199,76 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Tile list for the grouped GEMMs: one int4 {group, row_start, rows, 0} per
+// Tile lists for the grouped GEMMs: one int4 {group, row_start, rows, 0} per
 // 256-row tile of each expert segment of [e_lo, e_hi) (group e, rows in
 // permuted order), then the shared expert's tiles (group E, rows in token
-// order).  ntiles[0] = all tiles, ntiles[1] = routed tiles.
+// order).  Without a pair list every tile goes to `tiles` (ntiles[0] = all,
+// ntiles[1] = routed).  With one (tiles_pair != nullptr) the full 256-row
+// tiles go to `tiles_pair` (ntiles[2] = all, ntiles[3] = routed) and only the
+// partial tiles to `tiles`.
 __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, int e_lo, int e_hi, int T,
-                                   int with_shared, int4* __restrict__ tiles, int32_t* __restrict__ ntiles,
-                                   int* __restrict__ sched_counters) {
-  __shared__ int32_t warp_sums[32];
-  __shared__ int32_t total;
+                                   int with_shared, int4* __restrict__ tiles, int4* __restrict__ tiles_pair,
+                                   int32_t* __restrict__ ntiles, int* __restrict__ sched_counters) {
+  __shared__ long long warp_sums[32];
+  __shared__ long long total;
   const int e = threadIdx.x;
   const int lane = e & 31, warp = e >> 5;
-  int32_t start = 0, cnt = 0, mt = 0;
+  const bool split = tiles_pair != nullptr;
+  int32_t start = 0, cnt = 0, mt_full = 0, mt_part = 0;
   grid_dependency_wait();
   if (e >= e_lo && e < e_hi) {
     start = offsets[e];
     cnt = offsets[e + 1] - start;
-    mt = (cnt + kTileRows - 1) / kTileRows;
+    mt_full = split ? cnt / kTileRows : 0;
+    mt_part = split ? (cnt % kTileRows != 0) : (cnt + kTileRows - 1) / kTileRows;
   }
-  int32_t incl = mt;
+  // one scan of both counts: full tiles in the high word, partial in the low
+  const long long mine_t = ((long long)mt_full << 32) | (unsigned)mt_part;
+  long long incl = mine_t;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    const long long y = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += y;
   }
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
   if (warp == 0) {
     const int nw = blockDim.x >> 5;
-    const int32_t mine = (lane < nw) ? warp_sums[lane] : 0;
-    int32_t v = mine;
+    const long long mine = (lane < nw) ? warp_sums[lane] : 0;
+    long long v = mine;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int32_t y = __shfl_up_sync(0xffffffffu, v, o);
+      const long long y = __shfl_up_sync(0xffffffffu, v, o);
       if (lane >= o) v += y;
     }
     if (lane < nw) warp_sums[lane] = v - mine;
     if (lane == nw - 1) total = v;
   }
   __syncthreads();
-  const int32_t first = warp_sums[warp] + incl - mt;
-  for (int m = 0; m < mt; ++m) {
-    const int32_t r0 = m * kTileRows;
-    tiles[first + m] = make_int4(e, start + r0, min(kTileRows, cnt - r0), 0);
+  const long long first = warp_sums[warp] + incl - mine_t;
+  const int32_t first_full = (int32_t)(first >> 32), first_part = (int32_t)(first & 0xffffffffll);
+  for (int m = 0; m < mt_full; ++m)
+    tiles_pair[first_full + m] = make_int4(e, start + m * kTileRows, kTileRows, 0);
+  for (int m = 0; m < mt_part; ++m) {
+    const int32_t r0 = (mt_full + m) * kTileRows;
+    tiles[first_part + m] = make_int4(e, start + r0, min(kTileRows, cnt - r0), 0);
   }
-  const int32_t routed = total;
-  const int32_t shared_tiles = with_shared ? (T + kTileRows - 1) / kTileRows : 0;
-  for (int m = threadIdx.x; m < shared_tiles; m += blockDim.x) {
-    const int32_t r0 = m * kTileRows;
-    tiles[routed + m] = make_int4(E, r0, min(kTileRows, T - r0), 0);
+  const int32_t routed_full = (int32_t)(total >> 32), routed_part = (int32_t)(total & 0xffffffffll);
+  const int32_t shared_full = with_shared && split ? T / kTileRows : 0;
+  const int32_t shared_part = with_shared ? (split ? (T % kTileRows != 0) : (T + kTileRows - 1) / kTileRows) : 0;
+  for (int m = threadIdx.x; m < shared_full; m += blockDim.x)
+    tiles_pair[routed_full + m] = make_int4(E, m * kTileRows, kTileRows, 0);
+  for (int m = threadIdx.x; m < shared_part; m += blockDim.x) {
+    const int32_t r0 = (shared_full + m) * kTileRows;
+    tiles[routed_part + m] = make_int4(E, r0, min(kTileRows, T - r0), 0);
   }
   if (threadIdx.x == 0) {
-    ntiles[0] = routed + shared_tiles;
-    ntiles[1] = routed;
+    ntiles[0] = routed_part + shared_part;
+    ntiles[1] = routed_part;
+    if (split) {
+      ntiles[2] = routed_full + shared_full;
+      ntiles[3] = routed_full;
+    }
   }
   if (threadIdx.x < kNumSchedCounters) sched_counters[threadIdx.x] = 0;
 }
@@ -291,11 +308,12 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t
 }
 
 cudaError_t launch_build_tiles(const int32_t* offsets, int E, int64_t T, const Shard& shard, bool with_shared,
-                               int4* tiles, int32_t* ntiles, int* sched_counters, cudaStream_t stream) {
+                               int4* tiles, int32_t* ntiles, int* sched_counters, cudaStream_t stream,
+                               int4* tiles_pair) {
   const int threads = ((E + 31) / 32) * 32;
-  const cudaError_t err =
-      launch_chained(build_tiles_kernel, dim3(1), dim3(threads < 32 ? 32 : threads), 0, stream, offsets, E, shard.e_lo,
-                     shard.e_hi, (int)T, with_shared ? 1 : 0, tiles, ntiles, sched_counters);
+  const cudaError_t err = launch_chained(build_tiles_kernel, dim3(1), dim3(threads < 32 ? 32 : threads), 0, stream,
+                                         offsets, E, shard.e_lo, shard.e_hi, (int)T, with_shared ? 1 : 0, tiles,
+                                         tiles_pair, ntiles, sched_counters);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

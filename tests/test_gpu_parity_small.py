@@ -210,6 +210,25 @@ def test_grouped_swiglu_tile_half_boundaries(fp8):
     _experts_case(w, _boundary_idx(32))
 
 
+def test_grouped_swiglu_cta_pairs_on_full_tiles(monkeypatch):
+    # full 256-row tiles on 2-CTA clusters (tcgen05.mma.cta_group::2), the
+    # partial tiles on the one-CTA kernel, shared expert included
+    monkeypatch.setenv("MOE_PAIR_TILES", "1")
+    w = to_device(workloads.make_small("prefill", T=sum(HALF_BOUNDARY_COUNTS), d=256, E=32, k=1, inter=128,
+                                       shared_inter=128))
+    _experts_case(w, _boundary_idx(32))
+
+
+def test_forward_cta_pairs_match_one_cta_path(monkeypatch):
+    w = _medium(T=1536, E=32, k=8, shared_inter=512)  # ~384 rows per expert, 6 full shared tiles
+    monkeypatch.setenv("MOE_PAIR_TILES", "0")
+    y1, *_ = run_forward(w)
+    monkeypatch.setenv("MOE_PAIR_TILES", "1")
+    y2, err = _check_forward(w)
+    rms = float(y1.double().pow(2).mean().sqrt())
+    assert float((y1 - y2).abs().max()) <= 1e-5 * rms
+
+
 def test_grouped_swiglu_no_shared_expert():
     w = _medium(T=300, shared_inter=0)
     lg = oracle.logits(dec(w.x), dec(w.Wg))
