@@ -684,7 +684,8 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
 }
 
 // ------------------------------------------------------------ CTA pairs
-// Full 256-row tiles (bf16 weights) on a 2-CTA cluster: CTA r holds rows
+// Full 256-row tiles, and last tiles of more than kPairMinRows rows (bf16
+// weights), on a 2-CTA cluster: CTA r holds rows
 // 128r..128r+127 of the tile (A) and half of its B columns (SwiGLU: CTA 0 the
 // 128 W1 columns, CTA 1 the same 128 W3 columns; down: 128 of the 256 W2
 // columns each).  CTA 0's thread issues tcgen05.mma.cta_group::2 with M=256,

@@ -9,6 +9,9 @@ namespace moe {
 
 constexpr int kTileM = 128;     // rows per MMA (tcgen05 M) and per A box
 constexpr int kTileRows = 256;  // rows per grouped-GEMM tile list entry (two M halves)
+// A segment's last, partial tile runs on a CTA pair (as an M=256 MMA) when it
+// holds more than this many rows, else on one CTA.
+constexpr int kPairMinRows = 192;
 
 // K depth of one grouped-GEMM pipeline stage (32: A halves use a 64-byte
 // swizzle; 64: a 128-byte swizzle) and the number of stages.
@@ -126,7 +129,7 @@ cudaError_t launch_grouped_swiglu(const CUtensorMap& tmA_r, const CUtensorMap& t
                                   const CUtensorMap& tmW1_s, const CUtensorMap& tmW3_r, const CUtensorMap& tmW3_s,
                                   const GemmParams& p, int grid, cudaStream_t stream);
 // Full 256-row tiles of bf16 experts on 2-CTA clusters (tcgen05.mma
-// .cta_group::2, M=256): the tile list holds only full tiles; grid is
+// .cta_group::2, M=256): the pair tile list (full tiles and long last tiles); grid is
 // rounded down to whole clusters.
 cudaError_t launch_grouped_swiglu_pair(const CUtensorMap& tmA_r, const CUtensorMap& tmA_s, const CUtensorMap& tmW1_r,
                                        const CUtensorMap& tmW1_s, const CUtensorMap& tmW3_r, const CUtensorMap& tmW3_s,

@@ -204,8 +204,9 @@ __global__ void __launch_bounds__(256)
 // permuted order), then the shared expert's tiles (group E, rows in token
 // order).  Without a pair list every tile goes to `tiles` (ntiles[0] = all,
 // ntiles[1] = routed).  With one (tiles_pair != nullptr) the full 256-row
-// tiles go to `tiles_pair` (ntiles[2] = all, ntiles[3] = routed) and only the
-// partial tiles to `tiles`.
+// tiles, and a segment's last tile when it holds more than kPairMinRows rows,
+// go to `tiles_pair` (ntiles[2] = all, ntiles[3] = routed); the other partial
+// tiles to `tiles`.
 __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, int e_lo, int e_hi, int T,
                                    int with_shared, int4* __restrict__ tiles, int4* __restrict__ tiles_pair,
                                    int32_t* __restrict__ ntiles, int* __restrict__ sched_counters) {
@@ -219,8 +220,9 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
   if (e >= e_lo && e < e_hi) {
     start = offsets[e];
     cnt = offsets[e + 1] - start;
-    mt_full = split ? cnt / kTileRows : 0;
-    mt_part = split ? (cnt % kTileRows != 0) : (cnt + kTileRows - 1) / kTileRows;
+    const int rem = cnt % kTileRows;
+    mt_full = split ? cnt / kTileRows + (rem > kPairMinRows) : 0;
+    mt_part = split ? (rem != 0 && rem <= kPairMinRows) : (cnt + kTileRows - 1) / kTileRows;
   }
   // one scan of both counts: full tiles in the high word, partial in the low
   const long long mine_t = ((long long)mt_full << 32) | (unsigned)mt_part;
@@ -248,16 +250,18 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
   const long long first = warp_sums[warp] + incl - mine_t;
   const int32_t first_full = (int32_t)(first >> 32), first_part = (int32_t)(first & 0xffffffffll);
   for (int m = 0; m < mt_full; ++m)
-    tiles_pair[first_full + m] = make_int4(e, start + m * kTileRows, kTileRows, 0);
+    tiles_pair[first_full + m] = make_int4(e, start + m * kTileRows, min(kTileRows, cnt - m * kTileRows), 0);
   for (int m = 0; m < mt_part; ++m) {
     const int32_t r0 = (mt_full + m) * kTileRows;
     tiles[first_part + m] = make_int4(e, start + r0, min(kTileRows, cnt - r0), 0);
   }
   const int32_t routed_full = (int32_t)(total >> 32), routed_part = (int32_t)(total & 0xffffffffll);
-  const int32_t shared_full = with_shared && split ? T / kTileRows : 0;
-  const int32_t shared_part = with_shared ? (split ? (T % kTileRows != 0) : (T + kTileRows - 1) / kTileRows) : 0;
+  const int t_rem = T % kTileRows;
+  const int32_t shared_full = with_shared && split ? T / kTileRows + (t_rem > kPairMinRows) : 0;
+  const int32_t shared_part =
+      with_shared ? (split ? (t_rem != 0 && t_rem <= kPairMinRows) : (T + kTileRows - 1) / kTileRows) : 0;
   for (int m = threadIdx.x; m < shared_full; m += blockDim.x)
-    tiles_pair[routed_full + m] = make_int4(E, m * kTileRows, kTileRows, 0);
+    tiles_pair[routed_full + m] = make_int4(E, m * kTileRows, min(kTileRows, T - m * kTileRows), 0);
   for (int m = threadIdx.x; m < shared_part; m += blockDim.x) {
     const int32_t r0 = (shared_full + m) * kTileRows;
     tiles[routed_part + m] = make_int4(E, r0, min(kTileRows, T - r0), 0);
