@@ -101,6 +101,7 @@ constexpr size_t smem_bytes() {
 
 struct TileInfo {
   int group, row0, rows, nb, halves, k_routed;
+  int seg_tiles;  // row tiles of the group's segment (its weights are read once per row tile)
   bool shared;
 };
 
@@ -143,6 +144,7 @@ __device__ __forceinline__ bool tile_at(const GemmParams& p, const TileSpan& sp,
   ti.group = e.x;
   ti.row0 = e.y;
   ti.rows = e.z;
+  ti.seg_tiles = e.w;
   ti.halves = e.z > kTileM ? 2 : 1;
   ti.shared = (e.x == p.E);
   const int N = ti.shared ? p.N_shared : p.N_routed;
@@ -322,7 +324,9 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         if (tile < 0) break;
         TileInfo ti;
         if (!tile_at(p, span, tile, BN, ti)) continue;
-        const uint64_t pol_b = ti.shared ? pol_ws : pol_w;
+        // weights of an expert with several row tiles are read again by each
+        // of them: keep them in L2 (evict-normal) instead of streaming them
+        const uint64_t pol_b = ti.shared ? pol_ws : (ti.seg_tiles > 1 ? pol_a : pol_w);
         const CUtensorMap* mA = ti.shared ? &tmA_s : &tmA_r;
         const CUtensorMap* mB = ti.shared ? &tmB_s : &tmB_r;
         const CUtensorMap* mC = ti.shared ? &tmC_s : &tmC_r;
@@ -777,7 +781,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int tile = cluster; ok && tile < total; tile += clusters) {
         TileInfo ti;
         if (!tile_at(p, span, tile, BN, ti)) continue;
-        const uint64_t pol_b = ti.shared ? pol_ws : pol_w;
+        // weights of an expert with several row tiles are read again by each
+        // of them: keep them in L2 (evict-normal) instead of streaming them
+        const uint64_t pol_b = ti.shared ? pol_ws : (ti.seg_tiles > 1 ? pol_a : pol_w);
         const CUtensorMap* mA = ti.shared ? &tmA_s : &tmA_r;
         // SwiGLU: CTA 0 loads W1's columns, CTA 1 the same columns of W3
         const CUtensorMap* mB = (M == Mode::kSwiGLU && rank == 1) ? (ti.shared ? &tmC_s : &tmC_r)

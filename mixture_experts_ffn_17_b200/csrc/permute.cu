@@ -199,7 +199,8 @@ __global__ void __launch_bounds__(256)
   }
 }
 
-// Tile lists for the grouped GEMMs: one int4 {group, row_start, rows, 0} per
+// Tile lists for the grouped GEMMs: one int4 {group, row_start, rows,
+// row tiles of the group's segment} per
 // 256-row tile of each expert segment of [e_lo, e_hi) (group e, rows in
 // permuted order), then the shared expert's tiles (group E, rows in token
 // order).  Without a pair list every tile goes to `tiles` (ntiles[0] = all,
@@ -250,10 +251,11 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
   const long long first = warp_sums[warp] + incl - mine_t;
   const int32_t first_full = (int32_t)(first >> 32), first_part = (int32_t)(first & 0xffffffffll);
   for (int m = 0; m < mt_full; ++m)
-    tiles_pair[first_full + m] = make_int4(e, start + m * kTileRows, min(kTileRows, cnt - m * kTileRows), 0);
+    tiles_pair[first_full + m] =
+        make_int4(e, start + m * kTileRows, min(kTileRows, cnt - m * kTileRows), mt_full + mt_part);
   for (int m = 0; m < mt_part; ++m) {
     const int32_t r0 = (mt_full + m) * kTileRows;
-    tiles[first_part + m] = make_int4(e, start + r0, min(kTileRows, cnt - r0), 0);
+    tiles[first_part + m] = make_int4(e, start + r0, min(kTileRows, cnt - r0), mt_full + mt_part);
   }
   const int32_t routed_full = (int32_t)(total >> 32), routed_part = (int32_t)(total & 0xffffffffll);
   const int t_rem = T % kTileRows;
@@ -261,7 +263,7 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
   const int32_t shared_part =
       with_shared ? (split ? (t_rem != 0 && t_rem <= kPairMinRows) : (T + kTileRows - 1) / kTileRows) : 0;
   for (int m = threadIdx.x; m < shared_full; m += blockDim.x)
-    tiles_pair[routed_full + m] = make_int4(E, m * kTileRows, min(kTileRows, T - m * kTileRows), 0);
+    tiles_pair[routed_full + m] = make_int4(E, m * kTileRows, min(kTileRows, T - m * kTileRows), 0);  // shared
   for (int m = threadIdx.x; m < shared_part; m += blockDim.x) {
     const int32_t r0 = (shared_full + m) * kTileRows;
     tiles[routed_part + m] = make_int4(E, r0, min(kTileRows, T - r0), 0);
