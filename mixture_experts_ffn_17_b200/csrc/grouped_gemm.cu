@@ -945,6 +945,323 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   }
 }
 
+// FP8 weights on CTA pairs: per K step each CTA brings its 128 rows of A
+// (counted on CTA 0's barrier) and the raw e4m3 codes of its half of B
+// ([64 K x 128 N], counted on its own barrier); its converter warps widen them
+// (code x block scale -> bf16) into its own converted ring and arrive on CTA
+// 0's barrier; CTA 0 issues the M=256 pair MMA once both CTAs' A and both
+// conversions are in.  Routed tiles only (the shared expert is bf16).
+#ifndef MOE_PAIR_F8_STAGES
+#define MOE_PAIR_F8_STAGES 5
+#endif
+#ifndef MOE_PAIR_F8_CONV_STAGES
+#define MOE_PAIR_F8_CONV_STAGES 5
+#endif
+// The converted ring is as deep as the operand ring: its hand-off (MMA done on
+// CTA 0 -> commit to CTA 1 -> CTA 1 converts -> arrival on CTA 0) crosses the
+// pair twice per K step.
+constexpr int kPairF8Stages = MOE_PAIR_F8_STAGES;
+constexpr uint32_t kPairF8RawBytes = 64 * 128;                         // one raw box
+constexpr uint32_t kPairF8StageBytes = kPairABytes + kPairF8RawBytes;  // 24 KB
+constexpr int kPairF8ConvStages = MOE_PAIR_F8_CONV_STAGES;
+constexpr uint32_t kPairF8ConvBytes = 2 * kF8BoxBytes;  // 16 KB: two bf16 [64 K x 64 N] boxes
+constexpr int kPairF8EpiWarps = 4;
+constexpr int kPairF8Threads = 64 + 32 * kPairF8EpiWarps + 32 * kConvWarps;
+constexpr size_t pair_f8_smem_bytes() {
+  return 1024 + kPairF8Stages * kPairF8StageBytes + kPairF8ConvStages * kPairF8ConvBytes + 512;
+}
+static_assert(pair_f8_smem_bytes() <= 232448, "shared memory budget (FP8 pair)");
+
+template <Mode M>
+__global__ void __launch_bounds__(kPairF8Threads, 1)
+    grouped_gemm_pair_f8_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmB_r,
+                                const __grid_constant__ CUtensorMap tmC_r, const GemmParams p) {
+  constexpr int S = kPairF8Stages;
+  constexpr int CS = kPairF8ConvStages;
+  constexpr int BN = Cfg<M>::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* stage0 = align_1024(smem_raw);
+  uint8_t* conv0 = stage0 + S * kPairF8StageBytes;
+  uint64_t* afull = reinterpret_cast<uint64_t*>(conv0 + CS * kPairF8ConvBytes);  // CTA 0: both CTAs' A
+  uint64_t* rfull = afull + S;   // each CTA: its raw codes
+  uint64_t* empty = rfull + S;   // each CTA: stage free (MMA commit)
+  uint64_t* cfull = empty + S;   // CTA 0: both CTAs' conversions
+  uint64_t* cempty = cfull + CS; // each CTA: converted buffer free (MMA commit)
+  uint64_t* tfull = cempty + CS;
+  uint64_t* tempty = tfull + 2;  // CTA 0: both CTAs' epilogues
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  __shared__ uint32_t never;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool lead = rank == 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(&afull[s], 1);
+      ptx::mbar_init(&rfull[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int c = 0; c < CS; ++c) {
+      ptx::mbar_init(&cfull[c], 2 * kConvWarps);  // one arrival per converter warp of either CTA
+      ptx::mbar_init(&cempty[c], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&tfull[b], 1);
+      ptx::mbar_init(&tempty[b], 2 * 32 * kPairF8EpiWarps);
+    }
+    ptx::mbar_init(done, 1);
+    *abort_flag = 0u;
+    never = 0u;
+    ptx::fence_barrier_init();
+    ptx::fence_proxy_async();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(tmem_slot, kTmemCols);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();
+
+  const TileSpan span = tile_span(p);
+  const int total = span.count * p.n_nb;
+  const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tmA_r);
+      ptx::prefetch_tmap(&tmB_r);
+      if (M == Mode::kSwiGLU) ptx::prefetch_tmap(&tmC_r);
+      const uint64_t pol_a = ptx::policy_evict_normal();
+      const uint64_t pol_w = ptx::policy_evict_first();
+      int kg = 0;
+      bool ok = !p.debug_withhold_loads;
+      for (int tile = cluster; ok && tile < total; tile += clusters) {
+        TileInfo ti;
+        if (!tile_at(p, span, tile, BN, ti)) continue;
+        const uint64_t pol_b = ti.seg_tiles > 1 ? pol_a : pol_w;
+        // raw codes: SwiGLU CTA 0 W1 / CTA 1 W3 at columns n0; down W2 at n0 + 128r
+        const CUtensorMap* mR = (M == Mode::kSwiGLU && rank == 1) ? &tmC_r : &tmB_r;
+        const int rcol = ti.nb * BN + (M == Mode::kSwiGLU ? 0 : (int)rank * 128);
+        const int arow = ti.row0 + (int)rank * kTileM;
+        const int e3 = ti.group - p.group_base;
+        const int nk = p.K_routed / kF8BK;
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % S;
+          if (!ptx::wait_bounded(&empty[s], ((kg / S) & 1) ^ 1, abort_flag)) {
+            raise_status(p.status, abort_flag, kStatusTimeout);
+            ok = false;
+            break;
+          }
+          if (lead) ptx::mbar_arrive_expect_tx(&afull[s], 2 * kPairABytes);
+          ptx::mbar_arrive_expect_tx(&rfull[s], kPairF8RawBytes);
+          uint8_t* st = stage0 + s * kPairF8StageBytes;
+          ptx::tma_load_2d_pair(st, &tmA_r, ptx::mapa(&afull[s], 0), kb * kF8BK, arow, pol_a);
+          ptx::tma_load_3d(st + kPairABytes, mR, &rfull[s], rcol, kb * kF8BK, e3, pol_b);
+        }
+      }
+      // every copy of both CTAs lands before the pair may exit
+      for (int j = (kg > S ? kg - S : 0); j < kg; ++j) {
+        if (!ptx::wait_bounded(&rfull[j % S], (j / S) & 1, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
+        if (lead && !ptx::wait_bounded(&afull[j % S], (j / S) & 1, &never))
+          raise_status(p.status, abort_flag, kStatusTimeout);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && lead) {
+      constexpr uint32_t idesc = ptx::idesc_bf16(2 * kTileM, 256, false, true);
+      int kg = 0, tl = 0;
+      bool ok = true;
+      for (int tile = cluster; ok && tile < total; tile += clusters) {
+        TileInfo ti;
+        if (!tile_at(p, span, tile, BN, ti)) continue;
+        const int nk = p.K_routed / kF8BK;
+        const int sl = tl & 1;
+        if (!ptx::wait_bounded(&tempty[sl], ((tl >> 1) & 1) ^ 1, abort_flag)) {
+          raise_status(p.status, abort_flag, kStatusTimeout);
+          break;
+        }
+        ptx::tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb, ++kg) {
+          const int s = kg % S;
+          const int c = kg % CS;
+          if (!ptx::wait_bounded(&afull[s], (kg / S) & 1, abort_flag) ||
+              !ptx::wait_bounded(&cfull[c], (kg / CS) & 1, abort_flag)) {
+            raise_status(p.status, abort_flag, kStatusTimeout);
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a0 = ptx::smem_u32(stage0 + s * kPairF8StageBytes);
+          const uint32_t b0 = ptx::smem_u32(conv0 + c * kPairF8ConvBytes);
+#pragma unroll
+          for (int kk = 0; kk < kF8BK / 16; ++kk)
+            ptx::mma_bf16_pair(tmem + sl * kSlotCols, ptx::sdesc_sw128(a0 + kk * 32, 16, 1024),
+                               ptx::sdesc_sw128(b0 + kk * 2048, kF8BoxBytes, 1024), idesc, (kb | kk) != 0 ? 1u : 0u);
+          ptx::mma_commit_pair(&empty[s], 0x3);
+          ptx::mma_commit_pair(&cempty[c], 0x3);
+        }
+        if (!ok) break;
+        ptx::mma_commit_pair(&tfull[sl], 0x3);
+        ++tl;
+      }
+      ptx::mma_commit_pair(done, 0x1);
+      if (!ptx::wait_bounded(done, 0, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
+    }
+  } else if (warp < 2 + kPairF8EpiWarps) {
+    // epilogue: one warp per TMEM lane quarter, streaming 32-column chunks
+    const int q = warp & 3;
+    const int row = (int)rank * kTileM + q * 32 + lane;
+    const uint32_t tempty_lead0 = ptx::mapa(&tempty[0], 0), tempty_lead1 = ptx::mapa(&tempty[1], 0);
+    int tl = 0;
+    for (int tile = cluster; tile < total; tile += clusters) {
+      TileInfo ti;
+      if (!tile_at(p, span, tile, BN, ti)) continue;
+      const int sl = tl & 1;
+      if (!ptx::wait_bounded(&tfull[sl], (tl >> 1) & 1, abort_flag)) {
+        raise_status(p.status, abort_flag, kStatusTimeout);
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + sl * kSlotCols;
+      const bool valid = row < ti.rows;
+      const int n0 = ti.nb * BN;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t va[32], vb[32];
+        // SwiGLU: g and u of outputs n0 + 32c; down: W2 columns n0 + 64c, +32
+        ptx::tmem_ld32(tbase + (M == Mode::kSwiGLU ? c * 32 : c * 64), va);
+        ptx::tmem_ld32(tbase + (M == Mode::kSwiGLU ? 128 + c * 32 : c * 64 + 32), vb);
+        ptx::tmem_ld_wait2(va, vb);
+        if (c == 3) {
+          ptx::tc_fence_before();
+          ptx::mbar_arrive_cluster(sl ? tempty_lead1 : tempty_lead0);
+        }
+        if (!valid) continue;
+        if (M == Mode::kSwiGLU) {
+          uint16_t* base = static_cast<uint16_t*>(p.out_routed);
+          uint4* out = reinterpret_cast<uint4*>(base + ((int64_t)ti.row0 + row) * p.ld_out + n0 + c * 32);
+          uint32_t hp[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float g0 = __uint_as_float(va[2 * i]), g1 = __uint_as_float(va[2 * i + 1]);
+            const float u0 = __uint_as_float(vb[2 * i]), u1 = __uint_as_float(vb[2 * i + 1]);
+            hp[i] = ptx::pack_bf16x2(g0 / (1.0f + __expf(-g0)) * u0, g1 / (1.0f + __expf(-g1)) * u1);
+          }
+#pragma unroll
+          for (int v = 0; v < 4; ++v) out[v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
+        } else {
+#pragma unroll
+          for (int z = 0; z < 2; ++z) {
+            const uint32_t* v32 = z ? vb : va;
+            const int col = n0 + c * 64 + z * 32;
+            if (col >= p.N_routed) continue;
+            uint4* out =
+                reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out_routed) + ((int64_t)ti.row0 + row) * p.ld_out + col);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              out[v] = make_uint4(ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 0]), __uint_as_float(v32[8 * v + 1])),
+                                  ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 2]), __uint_as_float(v32[8 * v + 3])),
+                                  ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 4]), __uint_as_float(v32[8 * v + 5])),
+                                  ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 6]), __uint_as_float(v32[8 * v + 7])));
+          }
+        }
+      }
+      ++tl;
+    }
+  } else {
+    // converters: this CTA's raw box [64 K x 128 N] -> two bf16 [64 K x 64 N]
+    // boxes (128-byte swizzle, N-major); a warp step is 4 rows, a lane 16 codes
+    const int cw = warp - 2 - kPairF8EpiWarps;
+    const int sub_row = lane >> 3;
+    const int col16 = lane & 7;
+    int kg = 0;
+    bool ok = true;
+    for (int tile = cluster; ok && tile < total; tile += clusters) {
+      TileInfo ti;
+      if (!tile_at(p, span, tile, BN, ti)) continue;
+      const int nk = p.K_routed / kF8BK;
+      const int ncol = ti.nb * BN + (M == Mode::kSwiGLU ? 0 : (int)rank * 128);  // first raw column
+      const int ksb = p.K_routed / 128, nsb = p.N_routed / 128;
+      const float* scales = (M == Mode::kSwiGLU && rank == 1) ? p.scale_c : p.scale_b;
+      for (int kb = 0; kb < nk; ++kb, ++kg) {
+        const int s = kg % S;
+        const int c = kg % CS;
+        if (!ptx::wait_bounded(&rfull[s], (kg / S) & 1, abort_flag) ||
+            !ptx::wait_bounded(&cempty[c], ((kg / CS) & 1) ^ 1, abort_flag)) {
+          raise_status(p.status, abort_flag, kStatusTimeout);
+          ok = false;
+          break;
+        }
+        const uint8_t* raw = stage0 + s * kPairF8StageBytes + kPairABytes;
+        uint8_t* conv = conv0 + c * kPairF8ConvBytes;
+        const float scale =
+            scales[((int64_t)(ti.group - p.group_base) * ksb + (kb * kF8BK) / 128) * nsb + ncol / 128];
+#pragma unroll
+        for (int i = 0; i < 64 / (4 * kConvWarps); ++i) {
+          const int k = cw * (64 / kConvWarps) + i * 4 + sub_row;  // 0..63
+          const uint4 qv = *reinterpret_cast<const uint4*>(raw + k * 128 + col16 * 16);
+          const uint2 v0 = e4m3x4_to_bf16x4(qv.x, scale), v1 = e4m3x4_to_bf16x4(qv.y, scale);
+          const uint2 v2 = e4m3x4_to_bf16x4(qv.z, scale), v3 = e4m3x4_to_bf16x4(qv.w, scale);
+          uint8_t* dst = conv + (col16 >> 2) * kF8BoxBytes + k * 128;
+          const int ch = 2 * (col16 & 3);
+          *reinterpret_cast<uint4*>(dst + ((ch ^ (k & 7)) << 4)) = make_uint4(v0.x, v0.y, v1.x, v1.y);
+          *reinterpret_cast<uint4*>(dst + (((ch + 1) ^ (k & 7)) << 4)) = make_uint4(v2.x, v2.y, v3.x, v3.y);
+        }
+        // every lane's stores are made visible to the tensor cores' proxy, then
+        // one arrival per warp (a remote arrival per lane would cost a cluster
+        // transaction each)
+        ptx::fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa(&cfull[c], 0));
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem, kTmemCols);
+  }
+}
+
+template <Mode M>
+cudaError_t launch_pair_f8(const CUtensorMap& a_r, const CUtensorMap& b_r, const CUtensorMap& c_r,
+                           const GemmParams& p, int grid, cudaStream_t stream) {
+  const size_t smem = pair_f8_smem_bytes();
+  cudaError_t err =
+      cudaFuncSetAttribute(grouped_gemm_pair_f8_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  grid &= ~1;
+  if (grid <= 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kPairF8Threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = MOE_PDL ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_f8_kernel<M>, a_r, b_r, c_r, p);
+  return err != cudaSuccess ? err : cudaGetLastError();
+}
+
 template <Mode M>
 cudaError_t launch_pair(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtensorMap& b_r,
                         const CUtensorMap& b_s, const CUtensorMap& c_r, const CUtensorMap& c_s, const GemmParams& p,
@@ -1013,6 +1330,17 @@ cudaError_t launch_grouped_swiglu_pair(const CUtensorMap& tmA_r, const CUtensorM
 cudaError_t launch_grouped_down_pair(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
                                      const GemmParams& p, int grid, cudaStream_t stream) {
   return launch_pair<Mode::kDown>(tmA, tmA, tmW2_r, tmW2_s, tmW2_r, tmW2_s, p, grid, stream);
+}
+
+cudaError_t launch_grouped_swiglu_pair_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,
+                                           const CUtensorMap& tmW3_r, const GemmParams& p, int grid,
+                                           cudaStream_t stream) {
+  return launch_pair_f8<Mode::kSwiGLU>(tmA_r, tmW1_r, tmW3_r, p, grid, stream);
+}
+
+cudaError_t launch_grouped_down_pair_fp8(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const GemmParams& p,
+                                         int grid, cudaStream_t stream) {
+  return launch_pair_f8<Mode::kDown>(tmA, tmW2_r, tmW2_r, p, grid, stream);
 }
 
 cudaError_t launch_grouped_swiglu_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,

@@ -171,15 +171,19 @@ int num_sms() {
     if ((call) != cudaSuccess) return MOE_ERR_CUDA; \
   } while (0)
 
-// Full 256-row tiles run on CTA pairs (one tcgen05.mma.cta_group::2 M=256
-// per K step, B read once per 256 rows) when segments are long enough for
-// most rows to sit in full tiles: on average at least 384 rows per expert,
-// bf16 weights.  MOE_PAIR_TILES=1 / 0 in the environment forces it on / off.
+// Full 256-row tiles (and last tiles of more than 192 rows) run on CTA pairs
+// (one tcgen05.mma.cta_group::2 M=256 per K step, B read from shared memory
+// once per 256 rows; FP8 weights also converted once per 256 rows) when
+// segments are long enough for most rows to sit in such tiles: on average at
+// least 384 rows per expert, bf16 weights.  With FP8 weights the pair kernels
+// measured no faster than the one-CTA path (T=8192 layer: 9.53 vs 9.61 ms), so
+// they run only when forced.  MOE_PAIR_TILES=1 / 0 in the environment forces
+// pairs on / off.
 bool use_pair_tiles(const moe_shape& s) {
-  if (s.w_dtype == MOE_E4M3) return false;
   const char* v = std::getenv("MOE_PAIR_TILES");
   if (v && v[0] == '1') return true;
   if (v && v[0] == '0') return false;
+  if (s.w_dtype == MOE_E4M3) return false;
   return s.T * (int64_t)s.k >= (int64_t)384 * s.E;
 }
 
@@ -270,10 +274,22 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
     q.tile_set = kTilesRouted;
     q.scale_b = s1;
     q.scale_c = s3;
+    if (pair) {
+      GemmParams qp = q;
+      qp.tiles = tiles_pair;
+      qp.ntiles = ntiles + 2;
+      MOE_CUDA(launch_grouped_swiglu_pair_fp8(a8_r, w18_r, w38_r, qp, sms, st));
+    }
     MOE_CUDA(launch_grouped_swiglu_fp8(a8_r, w18_r, w38_r, q, grid1, st));
     if (sh) {
       q = p1;
       q.tile_set = kTilesShared;
+      if (pair) {
+        GemmParams qp = q;
+        qp.tiles = tiles_pair;
+        qp.ntiles = ntiles + 2;
+        MOE_CUDA(launch_grouped_swiglu_pair(a_r, a_s, w1_r, w1_s, w3_r, w3_s, qp, sms, st));
+      }
       q.sched_counter = sched + 1;
       MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, q, grid1, st));
     }
@@ -322,10 +338,22 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
     q.tile_set = kTilesRouted;
     q.scale_b = s2;
     q.scale_c = s2;
+    if (pair) {
+      GemmParams qp = q;
+      qp.tiles = tiles_pair;
+      qp.ntiles = ntiles + 2;
+      MOE_CUDA(launch_grouped_down_pair_fp8(h8_map, w28_r, qp, sms, st));
+    }
     MOE_CUDA(launch_grouped_down_fp8(h8_map, w28_r, q, grid2, st));
     if (sh) {
       q = p2;
       q.tile_set = kTilesShared;
+      if (pair) {
+        GemmParams qp = q;
+        qp.tiles = tiles_pair;
+        qp.ntiles = ntiles + 2;
+        MOE_CUDA(launch_grouped_down_pair(h_map, w2_r, w2_s, qp, sms, st));
+      }
       q.sched_counter = sched + 3;
       MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, q, grid2, st));
     }
@@ -560,8 +588,11 @@ int moe_forward_launches(const moe_shape* shape) {
   const moe_shape& s = *shape;
   if (s.T == 0) return 0;
   const int splits = router_splits(s.T, s.d, s.E, std::min(num_sms(), kRouterMaxSms));
-  // FP8: routed + shared launch; pair tiles: pair launch + one-CTA launch
-  const int gemm_launches = ((s.w_dtype == MOE_E4M3 && s.shared_inter > 0) || use_pair_tiles(s)) ? 2 : 1;
+  // per grouped GEMM: the routed tiles (CTA-pair launch + one-CTA launch with
+  // pairs), and with FP8 experts the bf16 shared expert's launches as well
+  const bool pair = use_pair_tiles(s);
+  int gemm_launches = pair ? 2 : 1;
+  if (s.w_dtype == MOE_E4M3 && s.shared_inter > 0) gemm_launches += pair ? 2 : 1;
   // router (+ split sum) + top-k, hist + scan + scatter, gather, tile list, two grouped GEMMs, combine
   return 1 + (splits > 1 ? 1 : 0) + 1 + 3 + 1 + 1 + 2 * gemm_launches + 1;
 }

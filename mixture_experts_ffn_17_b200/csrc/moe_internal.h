@@ -136,6 +136,13 @@ cudaError_t launch_grouped_swiglu_pair(const CUtensorMap& tmA_r, const CUtensorM
                                        const GemmParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_grouped_down_pair(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
                                      const GemmParams& p, int grid, cudaStream_t stream);
+// FP8 routed tiles of the pair list on 2-CTA clusters (tile_set must be
+// kTilesRouted: the shared expert is bf16).
+cudaError_t launch_grouped_swiglu_pair_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,
+                                           const CUtensorMap& tmW3_r, const GemmParams& p, int grid,
+                                           cudaStream_t stream);
+cudaError_t launch_grouped_down_pair_fp8(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const GemmParams& p,
+                                         int grid, cudaStream_t stream);
 cudaError_t launch_grouped_down(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
                                 const GemmParams& p, int grid, cudaStream_t stream);
 // FP8 (e4m3 + 128x128 block scales) routed experts; the tensor maps of W are

@@ -197,8 +197,13 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// Arrival on a barrier of either CTA of the cluster (default .release.cta
+// semantics: a cluster-scope release would fence all of this thread's memory
+// traffic cluster-wide on every arrival; the data handed over through these
+// barriers is tensor-core operand data in shared memory, published by
+// fence.proxy.async / tcgen05 fences before the arrival).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr) : "memory");
 }
 
 // TMA into this CTA's shared memory, completion counted on a barrier of the

@@ -185,3 +185,14 @@ def test_forward_launch_count():
     assert B.forward_launches(B.make_shape(T=0, d=512, E=32, k=4, inter=256, shared_inter=256)) == 0
     with pytest.raises(B.MoeError):
         B.forward_launches(B.make_shape(T=16, d=500, E=32, k=4, inter=256, shared_inter=256))
+
+
+def test_forward_launch_count_with_cta_pairs_forced(monkeypatch):
+    # pairs add a launch per grouped GEMM (pair + one-CTA), and with FP8
+    # experts the bf16 shared expert gets its own pair launch too
+    from mixture_experts_ffn_17_b200 import workloads
+    monkeypatch.setenv("MOE_PAIR_TILES", "1")
+    assert B.forward_launches(B.shape_of(workloads.CONFIGS["prefill"])) == 12
+    assert B.forward_launches(B.shape_of(workloads.CONFIGS["fp8"])) == 16
+    monkeypatch.setenv("MOE_PAIR_TILES", "0")
+    assert B.forward_launches(B.shape_of(workloads.CONFIGS["skewed"])) == 10

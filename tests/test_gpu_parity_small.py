@@ -229,6 +229,20 @@ def test_forward_cta_pairs_match_one_cta_path(monkeypatch):
     assert float((y1 - y2).abs().max()) <= 1e-5 * rms
 
 
+def test_grouped_swiglu_fp8_cta_pairs(monkeypatch):
+    # FP8 experts on CTA pairs: each CTA converts its half of the weight
+    # columns; the shared expert (bf16) runs on the bf16 pair kernel
+    monkeypatch.setenv("MOE_PAIR_TILES", "1")
+    w = to_device(workloads.make_small("fp8", T=sum(HALF_BOUNDARY_COUNTS), d=256, E=32, k=1, inter=128,
+                                       shared_inter=128, n_group=4, topk_group=2))
+    _experts_case(w, _boundary_idx(32))
+
+
+def test_forward_fp8_cta_pairs(monkeypatch):
+    monkeypatch.setenv("MOE_PAIR_TILES", "1")
+    _check_forward(_fp8(T=2048, k=8, E=64), tol=TOL_FP8)
+
+
 def test_grouped_swiglu_no_shared_expert():
     w = _medium(T=300, shared_inter=0)
     lg = oracle.logits(dec(w.x), dec(w.Wg))
