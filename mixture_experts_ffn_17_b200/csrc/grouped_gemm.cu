@@ -18,14 +18,15 @@
 //             swizzle: the weights' natural [K, N] row-major layout) into a
 //             3-stage ring (the K depth and stage count are build-time knobs,
 //             MOE_GEMM_BK / MOE_GEMM_STAGES; 64 x 3 measured fastest);
-//   warp 1    single-thread tcgen05.mma issuer, M=128, K=16 per instruction,
-//             fp32 accumulators in TMEM: two 256-column slots handed out
-//             round-robin (a one-half tile takes one, a two-half tile both),
-//             so one-half tiles overlap their epilogue with the next main loop;
+//   warp 1    single-thread tcgen05.mma issuer, M=128 (M=64 for a half of
+//             at most 64 rows), K=16 per instruction, fp32 accumulators in
+//             TMEM: two 256-column slots handed out round-robin (a one-half
+//             tile takes one, a two-half tile both), so one-half tiles overlap
+//             their epilogue with the next main loop;
 //   warps 2-9 epilogue (2-5 with FP8 weights): tcgen05.ld the accumulator
 //             rows (one row per thread, two warps per TMEM lane quarter each
-//             taking half of the columns), apply silu(g)*u (SwiGLU kernel)
-//             and store;
+//             taking half of the columns; bf16: the whole share is read before
+//             the slot is released), apply silu(g)*u (SwiGLU kernel) and store;
 //   warps 6-13 (FP8 weights only) converters: the producer brings raw e4m3
 //             weight tiles [64 K x 128 N] into the stage; these warps turn
 //             them into bf16 (code * the tile's 128 x 128 block scale) in the
@@ -40,6 +41,11 @@
 //                     bf16(silu(g) * u).
 // Kernel B (down):    N = 256 columns of W2 per tile; routed rows are stored
 //                     bf16 into Y_perm, shared-expert rows fp32 into Y_shared.
+//
+// Long segments (the Zipf-skewed workload) also use the CTA-pair kernels at
+// the end of this file: full 256-row tiles and last tiles of more than 192
+// rows run on 2-CTA clusters with tcgen05.mma.cta_group::2 (M=256), so each
+// weight byte is read from shared memory once per 256 rows.
 #include <algorithm>
 #include <cstdint>
 
