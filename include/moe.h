@@ -23,6 +23,9 @@
  *    returns.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default
  *    stream) and never synchronise the host, except moe_check_device_status.
+ *    A moe_forward call on a capturing stream is recorded into the CUDA graph
+ *    (kernels and memsets only); replays read whatever the captured buffers
+ *    hold at replay time.
  *  - Arguments are validated on the host before any launch; an invalid call
  *    returns an error and launches nothing.  T == 0 is valid and does nothing.
  *  - Dtypes: x, Wg, the shared expert and bf16 routed weights are bfloat16.
