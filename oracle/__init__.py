@@ -19,6 +19,9 @@ helpers written in the order of the pages' definitions:
 * sigmoid group-limited routing with selection bias (the FP8 group-routing
   workload's statement; the Baidu page's "Hierarchical Dynamic Routing" and the
   freedom251 page's "How V3 balances expert traffic" only hint at it).
+
+``backward.py`` (numpy, fp64) holds the layer's gradient: the derivative of
+the forward definition above, with the expert selection held fixed.
 """
 from __future__ import annotations
 
