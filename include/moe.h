@@ -189,6 +189,34 @@ moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const void*
 moe_status moe_combine(const moe_shape* shape, const void* Y_perm, const float* Y_shared, const int32_t* row_of,
                        const float* topk_w, void* y, void* stream);
 
+/* Backward of the combine (first step of the layer's backward pass).  The
+ * pages print no backward arithmetic; this is the derivative of the combine
+ * above with the expert selection held fixed.  For every (t, j) with
+ * r = row_of[t*k+j] >= 0:
+ *   dO_perm[r] = bf16(topk_w[t,j] * dy[t])     (the gradient of the routed
+ *                expert output, in the permuted row order of moe_permute)
+ *   dw[t,j]    = dy[t] . Y_perm[r]             (fp32 sum, fixed order)
+ * and dw[t,j] = 0 where r < 0.
+ *   dy [T, d] fp32; Y_perm [T*k, d] bf16 (the forward's routed expert
+ *   outputs, as moe_grouped_swiglu writes them); row_of [T*k], topk_w [T, k]
+ *   as moe_permute / moe_router_topk return them; dO_perm [T*k, d] bf16 out
+ *   (rows not addressed by row_of are not written); dw [T, k] fp32 out. */
+moe_status moe_combine_backward(const moe_shape* shape, const float* dy, const void* Y_perm, const int32_t* row_of,
+                                const float* topk_w, void* dO_perm, float* dw, void* stream);
+
+/* Backward of the routing weights with the selection held fixed: dlogits
+ * [T, E] fp32 out, zero outside each token's k selected experts.
+ *   top-k/softmax mode:  dl_j = w_j (dw_j - sum_i w_i dw_i)
+ *   group mode:          s = sigmoid(logit), Z = sum of the selected s,
+ *                        dl_j = route_scale (dw_j / Z - sum_i dw_i s_i / Z^2) s_j (1 - s_j)
+ * (derivatives of the weight rules of moe_route; the selection bias moves
+ * only the selection and gets no gradient).  logits [T, E] fp32 and
+ * topk_idx, topk_w [T, k] as moe_router_topk returns them; dw [T, k] fp32 as
+ * moe_combine_backward returns it.  An index outside [0, E) gets no
+ * gradient. */
+moe_status moe_router_backward(const moe_shape* shape, const float* logits, const int32_t* topk_idx,
+                               const float* topk_w, const float* dw, float* dlogits, void* stream);
+
 /* The whole layer: router, dispatch, grouped experts, shared expert and
  * combine, with no host synchronisation.
  *   y [T, d] out (fp32 or bf16 per shape->y_dtype)

@@ -24,7 +24,7 @@ MOE_ROUTE_TOPK_SOFTMAX, MOE_ROUTE_SIGMOID_GROUP = 0, 1
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
             "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version",
             "moe_permute_noalloc", "moe_router_topk_limited", "moe_expert_utilisation", "moe_forward_ep",
-            "moe_forward_launches")
+            "moe_forward_launches", "moe_combine_backward", "moe_router_backward")
 NUM_STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "experts_up", "experts_down", "combine")
 
@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.moe_permute_noalloc.restype = ctypes.c_int
         L.moe_grouped_swiglu.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_combine.argtypes = [S, P, P, P, P, P, P]
+        L.moe_combine_backward.argtypes = [S, P, P, P, P, P, P, P]
+        L.moe_router_backward.argtypes = [S, P, P, P, P, P, P]
         L.moe_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_forward_profiled.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P, P]
         I = ctypes.c_int
@@ -84,7 +86,8 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_launches.argtypes = [S]
         L.moe_forward_launches.restype = ctypes.c_int
         L.moe_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
-        for fn in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_forward",
+        for fn in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_combine_backward",
+                   "moe_router_backward", "moe_forward",
                    "moe_forward_profiled", "moe_forward_ep", "moe_check_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         L.moe_status_string.argtypes = [ctypes.c_int]
@@ -163,6 +166,18 @@ def grouped_swiglu(shape, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, 
 def combine(shape, Y_perm, Y_shared, row_of, topk_w, y, stream=None):
     _check(lib().moe_combine(ctypes.byref(shape), _ptr(Y_perm), _ptr(Y_shared), _ptr(row_of), _ptr(topk_w), _ptr(y),
                              _stream(stream)), "moe_combine")
+
+
+def combine_backward(shape, dy, Y_perm, row_of, topk_w, dO_perm, dw, stream=None):
+    """Backward of the combine (moe_combine_backward): dO_perm rows and dw."""
+    _check(lib().moe_combine_backward(ctypes.byref(shape), _ptr(dy), _ptr(Y_perm), _ptr(row_of), _ptr(topk_w),
+                                      _ptr(dO_perm), _ptr(dw), _stream(stream)), "moe_combine_backward")
+
+
+def router_backward(shape, logits, topk_idx, topk_w, dw, dlogits, stream=None):
+    """Backward of the routing weights (moe_router_backward): dlogits [T, E]."""
+    _check(lib().moe_router_backward(ctypes.byref(shape), _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(dw),
+                                     _ptr(dlogits), _stream(stream)), "moe_router_backward")
 
 
 def forward(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, ws, topk_idx=None, topk_w=None,

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "moe.h"
+#include "backward.h"
 #include "moe_internal.h"
 
 namespace moe {
@@ -560,6 +561,36 @@ moe_status moe_combine(const moe_shape* shape, const void* Y_perm, const float* 
   if (s.T == 0) return MOE_OK;
   MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, topk_w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16,
                           static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_combine_backward(const moe_shape* shape, const float* dy, const void* Y_perm, const int32_t* row_of,
+                                const float* topk_w, void* dO_perm, float* dw, void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  if (!dy || !Y_perm || !row_of || !topk_w || !dO_perm || !dw) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(dy) || !aligned16(Y_perm) || !aligned16(row_of) || !aligned16(topk_w) || !aligned16(dO_perm) ||
+      !aligned16(dw))
+    return MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  MOE_CUDA(launch_combine_backward(dy, Y_perm, row_of, topk_w, s.T, s.k, s.d, dO_perm, dw,
+                                   static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_router_backward(const moe_shape* shape, const float* logits, const int32_t* topk_idx,
+                               const float* topk_w, const float* dw, float* dlogits, void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  if (!logits || !topk_idx || !topk_w || !dw || !dlogits) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(logits) || !aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(dw) || !aligned16(dlogits))
+    return MOE_ERR_INVALID_ARG;
+  if (s.T == 0) return MOE_OK;
+  MOE_CUDA(launch_router_backward(logits, topk_idx, topk_w, dw, s.T, s.E, s.k,
+                                  s.route == MOE_ROUTE_SIGMOID_GROUP ? 1 : 0, s.route_scale, dlogits,
+                                  static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 

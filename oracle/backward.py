@@ -1,8 +1,8 @@
 """fp64 gradient of the MoE feed-forward layer.
 
 TEST INFRASTRUCTURE ONLY, like the rest of this package: only the tests may
-import it.  Nothing in ``mixture_experts_ffn_17_b200`` computes a backward pass
-yet; this is the reference a future backward kernel is checked against.
+import it.  The library's backward kernels (the combine and routing steps so
+far) are checked against it.
 
 The pages define the forward pass only (n4n.ai page "DeepSeek-V3's
 mixture-of-experts architecture explained", "The architecture in one diagram";
@@ -28,9 +28,11 @@ from __future__ import annotations
 
 import numpy as np
 
+from . import dispatch as _dispatch
 from . import logits as _logits
 from . import route_sigmoid_group as _route_group
 from . import route_topk_softmax as _route_topk
+from . import swiglu_rows as _swiglu_rows
 
 
 def _sigmoid(z: np.ndarray) -> np.ndarray:
@@ -58,6 +60,24 @@ def swiglu_backward(X: np.ndarray, W1: np.ndarray, W3: np.ndarray, W2: np.ndarra
     return dX, dW1, dW3, dW2, O
 
 
+def combine_backward(dy: np.ndarray, Yp: np.ndarray, row_of: np.ndarray, w: np.ndarray):
+    """Adjoint of y[t] = sum_j w[t,j] Yp[row_of[t,j]] (+ shared): for every
+    (t, j) with r = row_of[t*k + j] >= 0, dO[r] = w[t,j] dy[t] and
+    dw[t,j] = dy[t] . Yp[r]; dw is 0 where r < 0.  -> (dO [T*k, d], dw [T, k])."""
+    dy = np.asarray(dy, dtype=np.float64)
+    Yp = np.asarray(Yp, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    T, k = w.shape
+    r = np.asarray(row_of).reshape(T, k)
+    dO = np.zeros_like(Yp)
+    dw = np.zeros((T, k))
+    ok = r >= 0
+    tt, jj = np.nonzero(ok)
+    dO[r[tt, jj]] = w[tt, jj][:, None] * dy[tt]
+    dw[tt, jj] = np.einsum("nd,nd->n", dy[tt], Yp[r[tt, jj]])
+    return dO, dw
+
+
 def routing_backward(lg_sel: np.ndarray, w: np.ndarray, dw: np.ndarray, route: int, route_scale: float) -> np.ndarray:
     """Gradient of the k selected logits of one token from the gradient dw of
     its routing weights.
@@ -80,8 +100,10 @@ def moe_backward(x, Wg, W1, W3, W2, W1s=None, W3s=None, W2s=None, *, dy, k: int,
     Shapes as the forward oracle: x [T, d], Wg [E, d], W1/W3 [E, d, I],
     W2 [E, I, d], shared W1s/W3s [d, Is], W2s [Is, d] (or None).
     Returns a dict with dx, dWg, dW1, dW3, dW2 (and dW1s, dW3s, dW2s when the
-    shared expert is present), plus the selection idx, weights w, logits lg
-    and the forward output y it was computed at."""
+    shared expert is present); the intermediate gradients dO_perm (of the
+    routed expert outputs, permuted order), dw (of the routing weights) and dl
+    (of the logits); and the selection idx, weights w, logits lg, permuted
+    expert outputs Y_perm, row_of and the forward output y it was computed at."""
     x, Wg, W1, W3, W2, dy = (np.asarray(a, dtype=np.float64) for a in (x, Wg, W1, W3, W2, dy))
     T, d = x.shape
     E = W1.shape[0]
@@ -91,34 +113,40 @@ def moe_backward(x, Wg, W1, W3, W2, W1s=None, W3s=None, W2s=None, *, dy, k: int,
     else:
         idx, w, _, _ = _route_group(lg, bias, k, n_group, topk_group, group_topn, route_scale)
 
-    y = np.zeros((T, d))
+    # forward: every routed expert output in the permuted row order (experts
+    # ascending, then tokens), then y
+    _, offsets, perm, row_of = _dispatch(idx, E)
+    Yp = np.zeros((T * k, d))
+    for e in range(E):
+        rows = slice(offsets[e], offsets[e + 1])
+        if offsets[e + 1] > offsets[e]:
+            Yp[rows] = _swiglu_rows(x[perm[rows]], W1[e], W3[e], W2[e])
+    r = row_of.reshape(T, k)
+    y = np.einsum("tj,tjd->td", w, Yp[r])
+    # backward through the combine, then through each expert's SwiGLU
+    dO, dw = combine_backward(dy, Yp, row_of, w)
     dx = np.zeros((T, d))
     dW1 = np.zeros_like(W1)
     dW3 = np.zeros_like(W3)
     dW2 = np.zeros_like(W2)
-    dw = np.zeros((T, k))
-    # routed experts: each expert's rows together (the order of the rows does
-    # not change the sums beyond rounding)
     for e in range(E):
-        toks, slots = np.nonzero(idx == e)
-        if toks.size == 0:
+        if offsets[e + 1] == offsets[e]:
             continue
-        wt = w[toks, slots][:, None]
-        dO = wt * dy[toks]  # y_t = ... + w_tj o_tj
-        dX, g1, g3, g2, O = swiglu_backward(x[toks], W1[e], W3[e], W2[e], dO)
-        np.add.at(y, toks, wt * O)
+        rows = slice(offsets[e], offsets[e + 1])
+        toks = perm[rows]
+        dX, g1, g3, g2, _ = swiglu_backward(x[toks], W1[e], W3[e], W2[e], dO[rows])
         np.add.at(dx, toks, dX)
         dW1[e] += g1
         dW3[e] += g3
         dW2[e] += g2
-        dw[toks, slots] = np.einsum("nd,nd->n", dy[toks], O)  # d(sum dy*y)/dw_tj = dy_t . o_tj
     # routing weights -> logits -> x and Wg
     dl = np.zeros((T, E))
     for t in range(T):
         dl[t, idx[t]] = routing_backward(lg[t, idx[t]], w[t], dw[t], route, route_scale)
     dx += dl @ Wg
     dWg = dl.T @ x
-    out = dict(dx=dx, dWg=dWg, dW1=dW1, dW3=dW3, dW2=dW2, idx=idx, w=w, lg=lg)
+    out = dict(dx=dx, dWg=dWg, dW1=dW1, dW3=dW3, dW2=dW2, idx=idx, w=w, lg=lg, dw=dw, dl=dl, dO_perm=dO,
+               Y_perm=Yp, row_of=row_of)
     if W1s is not None:
         W1s, W3s, W2s = (np.asarray(a, dtype=np.float64) for a in (W1s, W3s, W2s))
         dXs, out["dW1s"], out["dW3s"], out["dW2s"], Os = swiglu_backward(x, W1s, W3s, W2s, dy)

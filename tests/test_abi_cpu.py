@@ -139,6 +139,12 @@ def test_stage_entry_points_validation_without_gpu():
                                 nul) == B.MOE_ERR_INVALID_ARG
     assert L.moe_combine(ctypes.byref(s), p, nul, nul, p, p, nul) == B.MOE_ERR_INVALID_ARG
     assert L.moe_check_device_status(nul, nul, None) == B.MOE_ERR_INVALID_ARG
+    # backward steps: a null or misaligned pointer is refused before any launch
+    odd = ctypes.c_void_p(p.value + 4)
+    assert L.moe_combine_backward(ctypes.byref(s), p, p, nul, p, p, p, nul) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_combine_backward(ctypes.byref(s), odd, p, p, p, p, p, nul) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_router_backward(ctypes.byref(s), p, p, p, nul, p, nul) == B.MOE_ERR_INVALID_ARG
+    assert L.moe_router_backward(ctypes.byref(s), p, p, p, p, odd, nul) == B.MOE_ERR_INVALID_ARG
 
 
 def test_empty_batch_is_a_no_op_without_gpu():
@@ -150,6 +156,8 @@ def test_empty_batch_is_a_no_op_without_gpu():
     assert L.moe_forward(ctypes.byref(s), p, p, None, p, p, p, None, None, None, p, p, p, p, None, None, None, p, n,
                          None) == B.MOE_OK
     assert L.moe_combine(ctypes.byref(s), p, p, p, p, p, None) == B.MOE_OK
+    assert L.moe_combine_backward(ctypes.byref(s), p, p, p, p, p, p, None) == B.MOE_OK
+    assert L.moe_router_backward(ctypes.byref(s), p, p, p, p, p, None) == B.MOE_OK
 
 
 def test_binding_refuses_without_library(monkeypatch, tmp_path):
