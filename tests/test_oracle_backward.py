@@ -135,6 +135,43 @@ def test_single_expert_k1_has_no_routing_gradient():
     assert np.all(g["w"] == 1.0)
 
 
+def test_combine_backward_is_the_adjoint_of_the_combine():
+    # <dy, combine(Yp, w)> = <dO, Yp> = <dw, w>, with the forward oracle's combine
+    rng = np.random.default_rng(7)
+    T, d, E, k = 40, 24, 9, 3
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    _, _, _, row_of = oracle.dispatch(idx, E)
+    Yp = rng.normal(size=(T * k, d))
+    w = rng.uniform(0.1, 1.0, size=(T, k))
+    dy = rng.normal(size=(T, d))
+    y = oracle.combine(Yp, None, row_of, w)
+    dO, dw = bw.combine_backward(dy, Yp, row_of, w)
+    lhs = np.sum(dy * y)
+    assert abs(lhs - np.sum(dO * Yp)) <= 1e-12 * (1 + abs(lhs))
+    assert abs(lhs - np.sum(dw * w)) <= 1e-12 * (1 + abs(lhs))
+
+
+@pytest.mark.parametrize("route", [0, 1])
+def test_routing_backward_matches_directional_differences_of_the_weight_rule(route):
+    # d/dh sum(dw * w(l + h v)) at h = 0 equals sum(dl * v), with w from the
+    # forward oracle's weight rule for a fixed selection
+    rng = np.random.default_rng(17 + route)
+    T, E, k = 30, 12, 4
+    lg = rng.normal(0, 1.5, size=(T, E))
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    dw = rng.normal(size=(T, k))
+    v = rng.normal(size=(T, E))
+    w0 = oracle.weights_for(lg, idx, route, 2.5)
+    dl = np.zeros((T, E))
+    for t in range(T):
+        dl[t, idx[t]] = bw.routing_backward(lg[t, idx[t]], w0[t], dw[t], route, 2.5)
+    h = 1e-6
+    fd = (np.sum(dw * oracle.weights_for(lg + h * v, idx, route, 2.5))
+          - np.sum(dw * oracle.weights_for(lg - h * v, idx, route, 2.5))) / (2 * h)
+    an = np.sum(dl * v)
+    assert abs(fd - an) <= 1e-7 * (1 + abs(an))
+
+
 # ------------------------------------------------------------ planted mistakes
 _ROUTING = bw.routing_backward
 
