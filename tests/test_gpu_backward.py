@@ -67,8 +67,8 @@ def test_combine_and_router_backward_match_oracle(case):
     dO_o, dw_o = obw.combine_backward(to_np(dy).astype(np.float64), dec(Y_perm), to_np(row_of),
                                       to_np(tw).astype(np.float64))
     dO_d = dec(dO)
-    # bf16(fp32(w * dy)): within one bf16 rounding of the exact product
-    assert np.all(np.abs(dO_d - dO_o) <= 2.0 ** -8 * np.abs(dO_o) + 1e-30)
+    # bf16(fp32(w * dy)): within one bf16 unit in the last place of the exact product
+    assert np.all(np.abs(dO_d - dO_o) <= 2.0 ** -7 * np.abs(dO_o) + 1e-30)
     scale = np.abs(to_np(dy)).astype(np.float64) @ np.ones(cfg.d) * np.abs(dec(Y_perm)).max()
     err = np.abs(to_np(dw).astype(np.float64) - dw_o)
     assert np.all(err <= 1e-5 * scale[:, None]), err.max()
