@@ -87,10 +87,12 @@ def oracle_sampled(w: workloads.Workload, lg: np.ndarray, idx: np.ndarray, token
     return y
 
 
-def choose_sample(idx: np.ndarray, counts: np.ndarray, near_tie_tokens, size: int, seed: int) -> np.ndarray:
+def choose_sample(idx: np.ndarray, counts: np.ndarray, near_tie_tokens, size: int, seed: int,
+                  per_expert: int = 4) -> np.ndarray:
     """Sample of tokens for output checks at full size: every near-tie token,
-    tokens on the 3 most- and 3 least-loaded non-empty experts, the first and
-    last token, the rest seeded random."""
+    tokens on the 3 most- and 3 least-loaded non-empty experts (up to
+    `per_expert` each), the first and last token, the rest seeded random, up
+    to `size` tokens in all."""
     T = idx.shape[0]
     pick = set(int(t) for t in near_tie_tokens)
     pick.update((0, T - 1))
@@ -98,7 +100,7 @@ def choose_sample(idx: np.ndarray, counts: np.ndarray, near_tie_tokens, size: in
     order = nz[np.argsort(counts[nz], kind="stable")]
     for e in list(order[:3]) + list(order[-3:]):
         toks = np.nonzero((idx == e).any(axis=1))[0]
-        pick.update(int(t) for t in toks[:2])
+        pick.update(int(t) for t in toks[:per_expert])
     rng = np.random.default_rng(seed)
     rest = [t for t in rng.permutation(T) if t not in pick]
     pick.update(int(t) for t in rest[:max(0, size - len(pick))])
@@ -110,13 +112,18 @@ def oracle_logits(w: workloads.Workload) -> np.ndarray:
 
 
 def route_with_exemptions(w, lg, idx_dev):
-    """Oracle routing, the exemption check, and the merged index set."""
-    from parity import compare_indices
+    """Oracle routing, the per-slot exemption check, and the merged index set
+    (the oracle's, with exempted tokens replaced by the device's choice).
+
+    Returns (idx_o, w_o, merged, report, n_near) where n_near counts the tokens
+    whose oracle routing has a near-tie at all."""
+    from parity import compare_indices, near_tie_tokens
     cfg = w.cfg
     bias = None if w.bias is None else dec(w.bias)
     idx_o, w_o, scores, gaps, ggap = oracle_route(cfg, lg, bias)
-    n_ex, report = compare_indices(idx_dev, idx_o, scores, gaps, ggap, cfg.E)
+    group = (cfg.n_group, cfg.topk_group, cfg.group_topn) if cfg.route == 1 else None
+    n_ex, report = compare_indices(idx_dev, idx_o, scores, gaps, ggap, cfg.E, group=group)
     merged = idx_o.copy()
-    for t, _ in report:
+    for t, _, _ in report:
         merged[t] = idx_dev[t]
-    return idx_o, w_o, merged, report
+    return idx_o, w_o, merged, report, len(near_tie_tokens(gaps, ggap))

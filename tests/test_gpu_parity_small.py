@@ -55,8 +55,8 @@ def test_router_matches_oracle(make):
     lg = oracle.logits(dec(w.x), dec(w.Wg))
     err = np.abs(to_np(lg_dev).astype(np.float64) - lg)
     assert err.max() <= 1e-6 * (1 + np.abs(lg).max()), err.max()
-    idx_o, w_o, merged, report = route_with_exemptions(w, lg, to_np(idx))
-    assert len(report) <= max(1, cfg.T // 100)
+    idx_o, w_o, merged, report, n_near = route_with_exemptions(w, lg, to_np(idx))
+    assert len(report) <= n_near, report      # exemptions only where the oracle itself has a near-tie
     ok = np.all(to_np(idx) == merged, axis=1)
     assert np.allclose(to_np(tw)[ok], w_o[ok], rtol=0, atol=2e-6)
 
@@ -72,7 +72,8 @@ def test_router_group_mode_matches_oracle():
     B.router_topk(shape, w.x, w.Wg, w.bias, idx, tw, None, ws)
     torch.cuda.synchronize()
     lg = oracle.logits(dec(w.x), dec(w.Wg))
-    idx_o, w_o, merged, report = route_with_exemptions(w, lg, to_np(idx))
+    idx_o, w_o, merged, report, n_near = route_with_exemptions(w, lg, to_np(idx))
+    assert len(report) <= n_near, report
     ok = np.all(to_np(idx) == merged, axis=1)
     assert np.allclose(to_np(tw)[ok], w_o[ok], rtol=0, atol=1e-5)
     assert np.allclose(to_np(tw).sum(1), 2.5, atol=1e-5)
@@ -274,7 +275,8 @@ def test_combine_matches_oracle(shared):
 def _check_forward(w, tol=TOL_BF16):
     y, idx, tw, counts, ws = run_forward(w)
     y_o, idx_o, w_o, lg = oracle_full(w)
-    _, _, merged, report = route_with_exemptions(w, lg, to_np(idx))
+    _, _, merged, report, n_near = route_with_exemptions(w, lg, to_np(idx))
+    assert len(report) <= n_near, report
     if report:
         y_o, *_ = oracle_full(w, force_idx=merged)
     c, _, _, _ = oracle.dispatch(merged, w.cfg.E)
@@ -376,6 +378,7 @@ def test_router_limited_matches_oracle():
     masked = np.where(allowed[None, :] > 0, lg, -np.inf)
     from parity import compare_indices
     n_ex, report = compare_indices(to_np(idx), idx_o, masked, gaps, None, cfg.E)
+    assert n_ex <= int(np.sum(np.any(gaps < 1e-6, axis=1))), report
     assert all(allowed[e] for e in to_np(idx).ravel())
     ok = np.all(to_np(idx) == idx_o, axis=1)
     assert np.allclose(to_np(tw)[ok], w_o[ok], rtol=0, atol=2e-6)
@@ -462,7 +465,8 @@ def test_forward_expert_parallel_shares_sum_to_the_layer(fp8, world):
     rms = float(y_full.double().pow(2).mean().sqrt())
     assert float((acc - y_full).abs().max()) <= 1e-4 * rms
     y_o, _, _, lg = oracle_full(w)
-    _, _, merged, report = route_with_exemptions(w, lg, to_np(idx))
+    _, _, merged, report, n_near = route_with_exemptions(w, lg, to_np(idx))
+    assert len(report) <= n_near, report
     if report:
         y_o, *_ = oracle_full(w, force_idx=merged)
     assert max_rel_err(to_np(acc).astype(np.float64), y_o) <= (TOL_FP8 if fp8 else TOL_BF16)

@@ -2,9 +2,13 @@
 256 routed experts, top-8, inter 2048, shared expert 2048), in the launch
 configuration the benchmark times (moe_forward, fp32 output).
 
-Routing, per-expert counts and the permutation are checked on all tokens
-(bit-exact up to reported near-ties); outputs on every token for the decode
-batch and on a seeded sample of tokens for the larger batches."""
+Routing, per-expert counts and the permutation are checked on all tokens,
+slot by slot (bit-exact except at a slot touched by an oracle near-tie, each
+such token reported with its gaps, and never more exemptions than tokens the
+oracle finds near-tied); outputs on every token for the decode batch and on a
+sample of S = 256 tokens for the larger batches (every near-tie token, tokens
+of the 3 most- and 3 least-loaded experts, the first and last token, the rest
+seeded random), the rms taken over that sample."""
 import numpy as np
 import pytest
 import torch
@@ -19,6 +23,8 @@ from parity import TOL_BF16, TOL_FP8, max_rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
+SAMPLE = 256   # output-check sample at the larger V3 batches
+
 
 @pytest.fixture(scope="module", autouse=True)
 def built():
@@ -32,7 +38,10 @@ def _check_v3(name, sample_size, tol=TOL_BF16):
     y, idx, tw, counts, ws = run_forward(w)
     idx_d = to_np(idx)
     lg = oracle_logits(w)
-    idx_o, w_o, merged, report = route_with_exemptions(w, lg, idx_d)
+    idx_o, w_o, merged, report, n_near = route_with_exemptions(w, lg, idx_d)
+    for t, slots, gg in report:
+        print(f"{name}: exempted token {t}: slots/gaps {slots}, group gap {gg}")
+    assert len(report) <= n_near, (len(report), n_near)
     # counts and permutation order: the oracle's dispatch of the accepted routing
     c, o, p, r = oracle.dispatch(merged, cfg.E)
     assert np.array_equal(to_np(counts), c)
@@ -49,11 +58,12 @@ def _check_v3(name, sample_size, tol=TOL_BF16):
     if sample_size is None:
         toks = np.arange(cfg.T)
     else:
-        toks = choose_sample(merged, c, [t for t, _ in report], sample_size, cfg.seed)
+        toks = choose_sample(merged, c, [t for t, _, _ in report], sample_size, cfg.seed)
+        assert len(toks) >= sample_size
     y_o = oracle_sampled(w, lg, merged, toks)
     err = max_rel_err(to_np(y[torch.as_tensor(toks, device="cuda")]).astype(np.float64), y_o)
-    print(f"{name}: near-ties {len(report)} {report[:5]}, touched {int((c > 0).sum())}, max count {c.max()}, "
-          f"empty {int((c == 0).sum())}, max|err|/rms over {len(toks)} tokens = {err:.3e}")
+    print(f"{name}: oracle near-tie tokens {n_near}, exempted {len(report)}, touched {int((c > 0).sum())}, "
+          f"max count {c.max()}, empty {int((c == 0).sum())}, max|err|/rms over {len(toks)} tokens = {err:.3e}")
     assert err <= tol, err
     return c, report
 
@@ -63,12 +73,12 @@ def test_v3_decode_all_tokens():
 
 
 def test_v3_prefill_sampled():
-    c, _ = _check_v3("prefill", 64)
+    c, _ = _check_v3("prefill", SAMPLE)
     assert (c > 0).all()                      # near-uniform routing touches every expert
 
 
 def test_v3_skewed_sampled():
-    c, _ = _check_v3("skewed", 64)
+    c, _ = _check_v3("skewed", SAMPLE)
     srt = np.sort(c)[::-1]
     share = srt[:26].sum() / srt.sum()
     assert 0.44 <= share <= 0.56, share       # about half the assignments on 10% of experts
@@ -76,5 +86,5 @@ def test_v3_skewed_sampled():
 
 
 def test_v3_fp8_group_routing_sampled():
-    c, _ = _check_v3("fp8", 64, tol=TOL_FP8)
+    c, _ = _check_v3("fp8", SAMPLE, tol=TOL_FP8)
     assert (c > 0).sum() > 200

@@ -36,6 +36,16 @@ MUTANTS = {
     "expert-parallel rank skips its first expert": ("if (e < e_lo || e >= e_lo + El) continue;",
                                                     "if (e <= e_lo || e >= e_lo + El) continue;"),
     "expert-parallel rank drops its shared slice": ("    if (Isl > 0)\n", "    if (0)\n"),
+    "top-k gap taken against slot j+2": ("gaps[t * k + j] = (j + 1 < m) ? l[top[j]] - l[top[j + 1]] : INFINITY;",
+                                         "gaps[t * k + j] = (j + 2 < m) ? l[top[j]] - l[top[j + 2]] : INFINITY;"),
+    "group slot gap on unbiased scores": ("gaps[t * k + j] = (j + 1 < m) ? sel[top[j]] - sel[top[j + 1]] : INFINITY;",
+                                          "gaps[t * k + j] = (j + 1 < m) ? s[top[j]] - s[top[j + 1]] : INFINITY;"),
+    "group-boundary gap against the wrong group": (
+        "gscore_gap[t] = (topk_group < n_group) ? gscore[gtop[topk_group - 1]] - gscore[gtop[topk_group]]",
+        "gscore_gap[t] = (topk_group < n_group) ? gscore[gtop[topk_group - 2]] - gscore[gtop[topk_group]]"),
+    "group weight rule without the scale": (
+        "for (int j = 0; j < k; ++j) w[t * k + j] = route_scale * (1.0 / (1.0 + exp(-l[idx[t * k + j]]))) / den;",
+        "for (int j = 0; j < k; ++j) w[t * k + j] = (1.0 / (1.0 + exp(-l[idx[t * k + j]]))) / den;"),
     "combine drops shared": ("        if (Ys)\n            for (int64_t c = 0; c < d; ++c) yt[c] += Ys[t * d + c];",
                              "        if (0)\n            for (int64_t c = 0; c < d; ++c) yt[c] += Ys[t * d + c];"),
 }

@@ -129,8 +129,12 @@ def test_topk_brute_force_random(E, k):
     idx, w, gaps = oracle.route_topk_softmax(lg, k)
     for t in range(40):
         assert idx[t].tolist() == _brute_topk(lg[t].tolist(), k)
-        # margins that decide each slot are positive for distinct values
-        assert np.all(gaps[t][: k if k < E else k - 1] > 0)
+        # the margin that decides slot j is the j-th minus the (j+1)-th score
+        # of all E experts in (score desc, index asc) order; +inf for the last
+        # slot when k == E (no expert was dropped)
+        ranked = sorted(range(E), key=lambda i: (-lg[t, i], i))
+        ref = [lg[t, ranked[j]] - lg[t, ranked[j + 1]] if j + 1 < E else math.inf for j in range(k)]
+        assert gaps[t].tolist() == ref
 
 
 @pytest.mark.parametrize("E,k", [(8, 3), (12, 4), (10, 2)])
@@ -195,7 +199,13 @@ def _brute_group(l, b, k, n_group, topk_group, topn, scale):
             best, best_key = comb, key
     chosen = sorted(best, key=lambda i: (-sel[i], i))
     den = sum(s[i] for i in chosen)
-    return chosen, [scale * s[i] / den for i in chosen], set(keep)
+    # the margins: each slot against the next candidate in (sel desc, index
+    # asc) order, and the last kept group's score against the best dropped one
+    ranked = sorted(cand, key=lambda i: (-sel[i], i))
+    gaps = [sel[ranked[j]] - sel[ranked[j + 1]] if j + 1 < len(ranked) else math.inf for j in range(k)]
+    granked = sorted(range(n_group), key=lambda g: (-gscore[g], g))
+    ggap = gscore[granked[topk_group - 1]] - gscore[granked[topk_group]] if topk_group < n_group else math.inf
+    return chosen, [scale * s[i] / den for i in chosen], set(keep), gaps, ggap
 
 
 @pytest.mark.parametrize("E,n_group,topk_group,k", [(16, 4, 2, 3), (12, 3, 2, 4), (16, 8, 4, 3)])
@@ -206,12 +216,20 @@ def test_group_routing_brute_force(E, n_group, topk_group, k):
     idx, w, gaps, ggap = oracle.route_sigmoid_group(lg, b, k, n_group, topk_group, 2, 2.5)
     gs = E // n_group
     for t in range(40):
-        chosen, wref, keep = _brute_group(lg[t].tolist(), b.tolist(), k, n_group, topk_group, 2, 2.5)
+        chosen, wref, keep, gref, ggref = _brute_group(lg[t].tolist(), b.tolist(), k, n_group, topk_group, 2, 2.5)
         assert idx[t].tolist() == chosen
         assert np.allclose(w[t], wref, rtol=1e-13, atol=0)
         assert all(i // gs in keep for i in idx[t])
         assert math.isclose(w[t].sum(), 2.5, rel_tol=1e-13)
-        assert ggap[t] >= 0
+        assert np.allclose(gaps[t], gref, rtol=0, atol=1e-15)
+        assert math.isclose(ggap[t], ggref, rel_tol=0, abs_tol=1e-15)
+    # the weight rule alone, on the brute-force selection: unbiased sigmoid
+    # scores normalised to sum 1, times the scale
+    brute_idx = np.array([_brute_group(lg[t].tolist(), b.tolist(), k, n_group, topk_group, 2, 2.5)[0]
+                          for t in range(40)], dtype=np.int32)
+    brute_w = np.array([_brute_group(lg[t].tolist(), b.tolist(), k, n_group, topk_group, 2, 2.5)[1]
+                        for t in range(40)])
+    assert np.allclose(oracle.weights_for(lg, brute_idx, route=1, route_scale=2.5), brute_w, rtol=1e-13, atol=0)
 
 
 def test_group_routing_one_group_no_bias_reduces_to_topk_of_logits():
