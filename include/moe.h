@@ -135,9 +135,12 @@ moe_status moe_expert_utilisation(const moe_shape* shape, const int32_t* counts,
  *   perm_token [T*k] int32 out: token at permuted position r
  *   row_of     [T*k] int32 out: permuted position of entry (t, j) at t*k + j
  *   x, x_perm  optional pair: when both are non-NULL, x_perm [T*k, d] bf16
- *              receives x[perm_token[r]] at row r.
+ *              receives x[perm_token[r]] at row r, for r < offsets[E].
  * An index outside [0, E) is skipped (its row_of is -1) and raises
- * MOE_ERR_DEVICE_BOUNDS in the workspace status word. */
+ * MOE_ERR_DEVICE_BOUNDS in the workspace status word; the skipped entries
+ * take no permuted position, so perm_token and x_perm hold offsets[E] < T*k
+ * rows and their tails are left untouched.  With T == 0 only counts and
+ * offsets are written (all zero) and the other pointers may be NULL. */
 moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t* counts, int32_t* offsets,
                        int32_t* perm_token, int32_t* row_of, const void* x, void* x_perm, void* ws,
                        size_t ws_bytes, void* stream);
@@ -151,9 +154,11 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t*
  * such callers.
  *  - Limit: ceil(T / 256) * E <= 65472 (e.g. T <= 65280 with E = 256);
  *    larger shapes return MOE_ERR_UNSUPPORTED and launch nothing.
- *  - The first call on a device looks up the array's device address (once per
- *    device, with that device current); make that first call before any
- *    stream capture.
+ *  - Every call looks up the array's device address in the calling thread's
+ *    current context (the array has one copy per context that loads the
+ *    library: the device's primary context, or a context the host runtime
+ *    made itself); the first call in a context may load the library's device
+ *    code there, so make that first call before any stream capture.
  *  - Allocates nothing (no cudaMalloc/cudaFree, no allocating library call).
  *  - All calls share the one array and it keeps the last call's contents:
  *    calls that overlap on the GPU (other streams, other threads) race;

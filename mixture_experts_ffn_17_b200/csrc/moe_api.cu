@@ -425,8 +425,7 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   if (ev) MOE_CUDA(cudaEventRecord(ev[1], st));
   MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
                           perm, row_of, status, st));
-  MOE_CUDA(launch_gather_rows(x, perm, s.T * s.k, s.d, x_perm, num_sms(), st, whole ? nullptr : offsets, shard.e_lo,
-                              shard.e_hi));
+  MOE_CUDA(launch_gather_rows(x, perm, s.T * s.k, s.d, x_perm, num_sms(), st, offsets, shard.e_lo, shard.e_hi));
   r = run_experts(sl, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared, status, st,
                   shard, ev ? ev + 2 : nullptr);
   if (r != MOE_OK) return r;
@@ -504,8 +503,10 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t*
   moe_status v = validate_shape(shape);
   if (v != MOE_OK) return v;
   const moe_shape& s = *shape;
-  if (!topk_idx || !counts || !offsets || !perm_token || !row_of) return MOE_ERR_INVALID_ARG;
-  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+  // an empty batch writes counts and offsets only: its [T*k] arrays may be NULL
+  if (s.T > 0 && (!topk_idx || !perm_token || !row_of)) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && (x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(topk_idx) || !aligned16(counts) || !aligned16(offsets) || !aligned16(perm_token) ||
       !aligned16(row_of) || (x && !aligned16(x)) || (x_perm && !aligned16(x_perm)))
     return MOE_ERR_INVALID_ARG;
@@ -521,7 +522,9 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t*
   }
   MOE_CUDA(launch_permute(topk_idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
                           perm_token, row_of, status, st));
-  if (x) MOE_CUDA(launch_gather_rows(x, perm_token, s.T * s.k, s.d, x_perm, num_sms(), st));
+  // only the rows the scatter wrote: entries with an out-of-range index are
+  // skipped, so perm_token holds offsets[E] <= T*k tokens
+  if (x) MOE_CUDA(launch_gather_rows(x, perm_token, s.T * s.k, s.d, x_perm, num_sms(), st, offsets, 0, s.E));
   return MOE_OK;
 }
 
@@ -677,34 +680,28 @@ const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
 // loads the library holds the array (512 KiB) until the process exits.
 //
 // In host code `g_noalloc_scratch` names a host-side stand-in, not a device
-// address, so its device address is fetched once per device with
-// cudaGetSymbolAddress (with that device current) and passed to the kernels.
+// address, so its device address is fetched with cudaGetSymbolAddress in the
+// caller's current context (the current device's) and passed to the kernels.
 // ---------------------------------------------------------------------------
 namespace moe {
 namespace {
 
 constexpr int64_t kNoallocScratchInts = 1 << 17;  // 512 KiB of int32
 constexpr int64_t kNoallocStatusInts = 64;        // status word, padded to 256 bytes
-constexpr int kNoallocMaxDevices = 64;
 
 static __device__ __align__(256) int32_t g_noalloc_scratch[kNoallocScratchInts];
 
-std::mutex g_noalloc_mu;
-int32_t* g_noalloc_ptr[kNoallocMaxDevices] = {};
-
-// Device address of the static scratch on the current device (set up on the
-// first call per device).
+// Device address of the static scratch in the calling thread's current
+// context.  A __device__ array has one copy per context that loads this
+// library's device code (the primary context of each device, and any context
+// a host runtime creates itself), and a context destroyed by cudaDeviceReset
+// takes its copy with it, so the address is looked up on every call rather
+// than cached.  The lookup allocates nothing; in a context where the library's
+// device code is not loaded yet (lazy module loading) it loads it first.
 moe_status noalloc_scratch(int32_t** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (dev < 0 || dev >= kNoallocMaxDevices) return MOE_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
-    g_noalloc_ptr[dev] = static_cast<int32_t*>(p);
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+  *out = static_cast<int32_t*>(p);
   return MOE_OK;
 }
 
@@ -719,8 +716,10 @@ extern "C" moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t*
   moe_status v = validate_shape(shape);
   if (v != MOE_OK) return v;
   const moe_shape& s = *shape;
-  if (!topk_idx || !counts || !offsets || !perm_token || !row_of) return MOE_ERR_INVALID_ARG;
-  if ((x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+  // an empty batch writes counts and offsets only: its [T*k] arrays may be NULL
+  if (s.T > 0 && (!topk_idx || !perm_token || !row_of)) return MOE_ERR_INVALID_ARG;
+  if (s.T > 0 && (x == nullptr) != (x_perm == nullptr)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(topk_idx) || !aligned16(counts) || !aligned16(offsets) || !aligned16(perm_token) ||
       !aligned16(row_of) || (x && !aligned16(x)) || (x_perm && !aligned16(x_perm)))
     return MOE_ERR_INVALID_ARG;
@@ -742,6 +741,8 @@ extern "C" moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t*
   int32_t* hist = scratch + kNoallocStatusInts;
   int32_t* base = hist + per;
   MOE_CUDA(launch_permute(topk_idx, s.T, s.k, s.E, hist, base, counts, offsets, perm_token, row_of, status, st));
-  if (x) MOE_CUDA(launch_gather_rows(x, perm_token, s.T * s.k, s.d, x_perm, num_sms(), st));
+  // only the rows the scatter wrote: entries with an out-of-range index are
+  // skipped, so perm_token holds offsets[E] <= T*k tokens
+  if (x) MOE_CUDA(launch_gather_rows(x, perm_token, s.T * s.k, s.d, x_perm, num_sms(), st, offsets, 0, s.E));
   return MOE_OK;
 }

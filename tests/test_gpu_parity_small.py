@@ -145,6 +145,39 @@ def test_permute_reports_out_of_range_index():
     assert to_np(out[0]).sum() == T * k - 2
 
 
+def test_permute_out_of_range_index_gathers_only_the_written_rows():
+    # the skipped entries take no permuted position: the row gather copies the
+    # offsets[E] = T*k - 2 rows the scatter wrote and leaves the tail alone
+    T, E, k, d = 300, 64, 4, 256
+    shape = B.make_shape(T=T, d=d, E=E, k=k, inter=128, shared_inter=0)
+    ws = B.alloc_workspace(shape)
+    rng = np.random.default_rng(31)
+    idx_np = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    idx_np[17, 2] = E
+    idx_np[250, 0] = -5
+    idx = torch.as_tensor(idx_np, device="cuda")
+    counts, offsets = (torch.empty(n, dtype=torch.int32, device="cuda") for n in (E, E + 1))
+    perm = torch.zeros(T * k, dtype=torch.int32, device="cuda")
+    row_of = torch.empty(T * k, dtype=torch.int32, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(6)
+    x = torch.randn(T, d, generator=g, device="cuda").to(torch.bfloat16)
+    x_perm = torch.full((T * k, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    B.permute(shape, idx, counts, offsets, perm, row_of, x, x_perm, ws)
+    rc, raw = B.check_device_status(ws)
+    assert rc == B.MOE_ERR_DEVICE_BOUNDS
+    valid = np.where((idx_np >= 0) & (idx_np < E), idx_np, -1)
+    n = T * k - 2
+    assert int(to_np(offsets)[E]) == n and int(to_np(counts).sum()) == n
+    assert np.array_equal(to_np(counts), np.bincount(valid[valid >= 0], minlength=E))
+    # expert-major, then (token, slot) order over the valid entries
+    tok, slot = np.nonzero(valid >= 0)
+    order = np.lexsort((slot, tok, valid[tok, slot]))
+    pv = to_np(perm)[:n]
+    assert np.array_equal(pv, tok[order])
+    assert torch.equal(x_perm[:n], x[torch.as_tensor(pv, device="cuda").long()])
+    assert bool((x_perm[n:] == 7.0).all())
+
+
 # --------------------------------------------------------------- experts
 def _experts_case(w, idx_np):
     cfg = w.cfg
