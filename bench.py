@@ -21,6 +21,7 @@ from __future__ import annotations
 import argparse
 import datetime
 import json
+import math
 import os
 import statistics
 import sys
@@ -35,6 +36,10 @@ import torch  # noqa: E402
 
 METRIC = "MoE-layer tokens/s and TFLOPS at V3 shapes (T=4096 bf16); % of roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures (dense): the second denominator every fraction is
+# also reported against
+DATASHEET_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0, "fp8_tflops": 4500.0}
+FP8_OVER_BF16 = 2.0  # nominal dense FP8 : bf16 tensor throughput
 
 
 def parse_args():
@@ -50,6 +55,10 @@ def parse_args():
     p.add_argument("--cpu-sample", type=int, default=16, help="tokens the CPU baseline runs through the oracle")
     p.add_argument("--ref-sample", type=int, default=2, help="tokens per step of the reference arm")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--sustain-s", type=float, default=2.5,
+                   help="seconds of back-to-back layers in the sustained leg (0: skip it)")
+    p.add_argument("--no-decode", action="store_true",
+                   help="skip the decode-batch record that the prefill run adds to its line")
     p.add_argument("--ep-size", type=int, default=1,
                    help="expert-parallel layer over this many ranks (moe_forward_ep + an all-reduce of y)")
     p.add_argument("--ep-rank", type=int, default=0,
@@ -97,13 +106,18 @@ class Dist:
 
 
 def load_peaks():
+    """Measured peaks of this machine's B200s (MEASURED_PEAKS.json) or the
+    fallback figures; FP8 tensor peaks are the bf16 ones x the nominal ratio."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             p = json.load(f)
-        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+        peaks, src = {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
     except (OSError, KeyError, ValueError):
-        return dict(FALLBACK_PEAKS), "fallback"
+        peaks, src = dict(FALLBACK_PEAKS), "fallback"
+    peaks["fp8_tflops"] = peaks["bf16_tflops"] * FP8_OVER_BF16
+    peaks["fp8_tflops_sustained"] = peaks["bf16_tflops_sustained"] * FP8_OVER_BF16
+    return peaks, src
 
 
 class ClockSampler:
@@ -216,6 +230,53 @@ def layer_work(cfg, counts, y_bytes_per_el):
     return flops, routed_w + shared_w + cfg.E * cfg.d * 2 + act, n_touched
 
 
+def layer_roofline(cfg, counts, ms, peaks, peak_src, y_bytes_per_el=4):
+    """max(FLOPs / tensor peak, bytes / HBM bandwidth) of one layer and the
+    fraction of it a measured step time reaches.  The routed experts' FLOPs of
+    an FP8 workload are priced at the FP8 peak and the router's and shared
+    expert's at the bf16 one; `frac_bf16_rate` prices every FLOP at the bf16
+    peak (the MMA runs kind::f16: the activations stay bf16).  Both against the
+    measured peaks (sustained tensor peak) and against the datasheet."""
+    flops, nbytes, n_touched = layer_work(cfg, counts, y_bytes_per_el)
+    f_routed = cfg.T * cfg.k * 6 * cfg.d * cfg.inter
+    f_fp8 = f_routed if cfg.fp8 else 0
+    f_bf16 = flops - f_fp8
+
+    def terms(bf16, fp8, hbm):
+        t_tc = f_bf16 / (bf16 * 1e12) + f_fp8 / (fp8 * 1e12)
+        t_tc16 = flops / (bf16 * 1e12)
+        t_hbm = nbytes / (hbm * 1e9)
+        return t_tc, t_tc16, t_hbm
+
+    t_tc, t_tc16, t_hbm = terms(peaks["bf16_tflops_sustained"], peaks["fp8_tflops_sustained"], peaks["hbm_gbs"])
+    d_tc, d_tc16, d_hbm = terms(DATASHEET_PEAKS["bf16_tflops"], DATASHEET_PEAKS["fp8_tflops"],
+                                DATASHEET_PEAKS["hbm_gbs"])
+    roof = max(t_tc, t_hbm)
+    out = {"roofline_ms": 1e3 * roof, "tensor_ms": 1e3 * t_tc, "hbm_ms": 1e3 * t_hbm,
+           "bound": "hbm" if t_hbm >= t_tc else "tensor", "frac": 1e3 * roof / ms,
+           "frac_datasheet": 1e3 * max(d_tc, d_hbm) / ms,
+           "flops": flops, "bytes": nbytes, "touched_experts": n_touched,
+           "peaks": f"{peak_src}: hbm {peaks['hbm_gbs']} GB/s, bf16 {peaks['bf16_tflops_sustained']} TF/s sustained"
+                    + (f", fp8 {peaks['fp8_tflops_sustained']} TF/s (bf16 x {FP8_OVER_BF16:g})" if cfg.fp8 else "")
+                    + f"; datasheet: hbm {DATASHEET_PEAKS['hbm_gbs']:g} GB/s, bf16 {DATASHEET_PEAKS['bf16_tflops']:g}"
+                    + (f", fp8 {DATASHEET_PEAKS['fp8_tflops']:g}" if cfg.fp8 else "") + " TF/s"}
+    if cfg.fp8:
+        out["frac_bf16_rate"] = 1e3 * max(t_tc16, t_hbm) / ms
+        out["frac_bf16_rate_datasheet"] = 1e3 * max(d_tc16, d_hbm) / ms
+    return out
+
+
+def touched_weight_bytes(cfg, counts):
+    """Weight bytes a layer must stream: the touched routed experts (with FP8
+    block scales) and the shared expert."""
+    wb = 1 if cfg.fp8 else 2
+    n = touched_experts(counts)
+    b = n * 3 * cfg.d * cfg.inter * wb + 3 * cfg.d * cfg.shared_inter * 2
+    if cfg.fp8:
+        b += n * 3 * (cfg.d // 128) * (cfg.inter // 128) * 4
+    return b
+
+
 def kernel_work(cfg, counts, stage):
     """Algorithmic FLOPs / bytes of one launch of an expert kernel: the
     touched experts' weight slices plus the shared expert's, the activation
@@ -321,6 +382,81 @@ def config_of(cfg, args):
             "parallelism": f"replicas x{args.gpus}"}
 
 
+def time_loop(step, K, stream, dev, dist):
+    """K calls of step(i) between events on the launching stream, with a
+    barrier and a synchronize on both sides and NVML clock samples during the
+    loop.  Returns (ms per step, max over ranks; clock summary)."""
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    with sampler:
+        start.record(stream)
+        for i in range(K):
+            step(i)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier()
+    return dist.max(start.elapsed_time(end) / K), sampler.summary()
+
+
+def sustained_leg(B, fwd_args, counts, cfg, K_min, ms_burst, seconds, stream, dev, dist, peaks, peak_src):
+    """Back-to-back layers for about `seconds` (the power cap sets the clock
+    after a few hundred ms): its own step time, clocks and roofline fraction."""
+    K = max(K_min, int(math.ceil(seconds * 1e3 / ms_burst)))
+    ms, clocks = time_loop(lambda i: B.forward(*fwd_args, counts=counts), K, stream, dev, dist)
+    c = counts.cpu().numpy()
+    roof = layer_roofline(cfg, c, ms, peaks, peak_src)
+    out = {"steps": K, "seconds": K * ms / 1e3, "ms_per_step": ms, "tokens_per_s": dist.world * cfg.T / (ms / 1e3),
+           "tflops": dist.world * roof["flops"] / (ms / 1e3) / 1e12, "frac": roof["frac"],
+           "frac_datasheet": roof["frac_datasheet"], "clocks": clocks}
+    if "frac_bf16_rate" in roof:
+        out["frac_bf16_rate"] = roof["frac_bf16_rate"]
+    if clocks.get("sm_mhz"):
+        out["mcycles_per_step"] = ms * clocks["sm_mhz"] / 1e3   # step time x median SM clock
+    return out
+
+
+def decode_record(args, dist, dev, stream, peaks, peak_src):
+    """The decode layer (T=64) timed in the same run: touched-expert weight
+    streaming against HBM bandwidth, burst and sustained."""
+    from mixture_experts_ffn_17_b200 import binding as B
+    from mixture_experts_ffn_17_b200 import workloads
+    cfg = workloads.CONFIGS["decode"]
+    w = workloads.make(cfg, device=dev)
+    shape = B.shape_of(cfg, B.MOE_F32)
+    ws = B.alloc_workspace(shape, dev)
+    y = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device=dev)
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    fwd_args = (shape, w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s, y, ws)
+    for _ in range(max(args.warmup, 3)):
+        B.forward(*fwd_args, counts=counts)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"decode: device status after warm-up (raw {raw})")
+    K = max(args.steps, 50)
+    ms, clocks = time_loop(lambda i: B.forward(*fwd_args, counts=counts), K, stream, dev, dist)
+    c = counts.cpu().numpy()
+    roof = layer_roofline(cfg, c, ms, peaks, peak_src)
+    wbytes = touched_weight_bytes(cfg, c)
+    rec = {"workload": config_of(cfg, args)["workload"], "steps": K, "ms_per_step": ms,
+           "tokens_per_s": dist.world * cfg.T / (ms / 1e3), "touched_experts": roof["touched_experts"],
+           "touched_weight_bytes": wbytes,
+           "touched_weight_gbs": wbytes / (ms / 1e3) / 1e9,
+           "hbm_frac": wbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+           "hbm_frac_datasheet": wbytes / (ms / 1e3) / 1e9 / DATASHEET_PEAKS["hbm_gbs"],
+           "roofline_layer": roof, "clocks": clocks}
+    if args.sustain_s > 0:
+        sus = sustained_leg(B, fwd_args, counts, cfg, K, ms, args.sustain_s, stream, dev, dist, peaks, peak_src)
+        sus["hbm_frac"] = wbytes / (sus["ms_per_step"] / 1e3) / 1e9 / peaks["hbm_gbs"]
+        rec["sustained"] = sus
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"decode: device status after the timed steps (raw {raw})")
+    rec["gpu_launches_per_step"] = B.forward_launches(shape)
+    return rec
+
+
 def run_ours(args, dist):
     from mixture_experts_ffn_17_b200 import binding as B
     from mixture_experts_ffn_17_b200 import workloads
@@ -346,24 +482,13 @@ def run_ours(args, dist):
     if rc != B.MOE_OK:
         raise B.MoeError(rc, f"device status after warm-up (raw {raw})")
 
+    # the timed steps: K layers, each with events at its stage boundaries
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(B.NUM_STAGE_EVENTS)] for _ in range(K)]
     for row in evs:
         for e in row:
             e.record(stream)
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(dev.index)
-    dist.barrier()
-    torch.cuda.synchronize(dev)
-    with sampler:
-        start.record(stream)
-        for i in range(K):
-            B.forward_profiled(*fwd_args, evs[i], counts=counts)
-        end.record(stream)
-        torch.cuda.synchronize(dev)
-    dist.barrier()
-    ms = start.elapsed_time(end) / K
-    ms_max = dist.max(ms)
+    ms_max, clocks = time_loop(lambda i: B.forward_profiled(*fwd_args, evs[i], counts=counts), K, stream, dev, dist)
     rc, raw = B.check_device_status(ws)
     if rc != B.MOE_OK:
         raise B.MoeError(rc, f"device status after the timed steps (raw {raw})")
@@ -372,29 +497,41 @@ def run_ours(args, dist):
                 for j, name in enumerate(B.STAGES)}
     counts_np = counts.cpu().numpy()
     peaks, peak_src = load_peaks()
-    flops, nbytes, n_touched = layer_work(cfg, counts_np, 4)
+    roof_layer = layer_roofline(cfg, counts_np, ms_max, peaks, peak_src)
+    flops = roof_layer["flops"]
     tokens_per_s = dist.world * cfg.T / (ms_max / 1e3)
-    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
-    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    roof_ms = 1e3 * max(t_tc, t_hbm)
 
+    # the dominant kernel against its own roofline (the tensor peak of its
+    # weights' dtype: FP8 routed experts at the FP8 peak)
     dom = max(("experts_up", "experts_down"), key=lambda s: stage_ms[s])
     kf, kb = kernel_work(cfg, counts_np, dom)
     k_ms = stage_ms[dom]
-    k_tc = kf / (peaks["bf16_tflops_sustained"] * 1e12)
+    tc_key = "fp8_tflops_sustained" if cfg.fp8 else "bf16_tflops_sustained"
+    k_tc = kf / (peaks[tc_key] * 1e12)
     k_hbm = kb / (peaks["hbm_gbs"] * 1e9)
     if k_hbm >= k_tc:
         roof = {"bound": "hbm", "achieved": kb / (k_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        roof["frac_datasheet"] = roof["achieved"] / DATASHEET_PEAKS["hbm_gbs"]
     else:
-        roof = {"bound": "tensor", "achieved": kf / (k_ms / 1e3) / 1e12, "peak": peaks["bf16_tflops_sustained"],
+        roof = {"bound": "tensor", "achieved": kf / (k_ms / 1e3) / 1e12, "peak": peaks[tc_key],
                 "unit": "TFLOP/s"}
+        roof["frac_datasheet"] = roof["achieved"] / DATASHEET_PEAKS["fp8_tflops" if cfg.fp8 else "bf16_tflops"]
+        if cfg.fp8:
+            roof["frac_bf16_rate"] = roof["achieved"] / peaks["bf16_tflops_sustained"]
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = captured_traffic(dom, args)
     roof["kernel"] = f"grouped_gemm_kernel<{'SwiGLU' if dom == 'experts_up' else 'Down'}> ({dom})"
-    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if roof['bound'] == 'hbm' else 'bf16_tflops_sustained'})"
+    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if roof['bound'] == 'hbm' else tc_key})"
     roof["algorithmic_bytes_per_launch"] = kb
     roof["algorithmic_flops_per_launch"] = kf
     roof["ms_per_launch"] = k_ms
+
+    sustained = None
+    if args.sustain_s > 0:
+        sustained = sustained_leg(B, fwd_args, counts, cfg, K, ms_max, args.sustain_s, stream, dev, dist, peaks,
+                                  peak_src)
+        if clocks.get("sm_mhz"):
+            sustained["burst_mcycles_per_step"] = ms_max * clocks["sm_mhz"] / 1e3
 
     e2e = None
     if not args.no_e2e:
@@ -405,17 +542,21 @@ def run_ours(args, dist):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": config_of(cfg, args),
             "tflops": dist.world * flops / (ms_max / 1e3) / 1e12,
-            "roofline_layer": {"roofline_ms": roof_ms, "tensor_ms": 1e3 * t_tc, "hbm_ms": 1e3 * t_hbm,
-                               "bound": "hbm" if t_hbm >= t_tc else "tensor", "frac": roof_ms / ms,
-                               "flops": flops, "bytes": nbytes, "touched_experts": n_touched,
-                               "peaks": f"{peak_src}: hbm {peaks['hbm_gbs']} GB/s, bf16 "
-                                        f"{peaks['bf16_tflops_sustained']} TF/s sustained"},
-            "roofline": roof, "stage_ms": stage_ms, "clocks": sampler.summary(),
+            "roofline_layer": roof_layer, "roofline": roof, "stage_ms": stage_ms, "clocks": clocks,
             "gpu_launches": B.forward_launches(shape) * K}
+    if sustained:
+        line["sustained"] = sustained
     if e2e:
         line["e2e"] = e2e
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = run_cpu_baseline(args, w, cfg)
+    if args.workload == "prefill" and not (args.tokens or args.experts or args.no_decode):
+        # the decode batch of the same layer shapes, in the same run (its own
+        # weights; the prefill ones are released first)
+        del w, ws, fwd_args, y
+        torch.cuda.empty_cache()
+        line["decode"] = decode_record(args, dist, dev, stream, peaks, peak_src)
+        line["config"]["workload"] += "; decode record: " + line["decode"]["workload"]
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
 
