@@ -57,6 +57,8 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--sustain-s", type=float, default=2.5,
                    help="seconds of back-to-back layers in the sustained leg (0: skip it)")
+    p.add_argument("--no-backward", action="store_true",
+                   help="skip the backward-pass record that the prefill run adds to its line")
     p.add_argument("--no-decode", action="store_true",
                    help="skip the decode-batch record that the prefill run adds to its line")
     p.add_argument("--ep-size", type=int, default=1,
@@ -457,6 +459,61 @@ def decode_record(args, dist, dev, stream, peaks, peak_src):
     return rec
 
 
+def backward_work(cfg, counts, grad_bytes):
+    """Algorithmic FLOPs and bytes of one moe_backward call (the forward it
+    recomputes, then the gradients): FLOPs = the forward's + per routed and
+    shared row 12 d I (dH, dX, and the three weight gradients) + 4 T E d
+    (dl Wg and dWg); bytes = the touched experts' and the shared expert's
+    weights read twice (forward, then dH / dX), every weight gradient written
+    once, Wg read twice, dWg written, x and dy read, dx written."""
+    T, d, E, k, I, Is = cfg.T, cfg.d, cfg.E, cfg.k, cfg.inter, cfg.shared_inter
+    flops = T * cfg.flops_per_token() + T * k * 12 * d * I + T * 12 * d * Is + 4 * T * E * d
+    wbytes = touched_weight_bytes(cfg, counts)
+    grads = (E * 3 * d * I + 3 * d * Is + E * d) * grad_bytes
+    nbytes = 2 * wbytes + grads + 2 * E * d * 2 + T * d * 2 + T * d * 4 + T * d * grad_bytes
+    return flops, nbytes
+
+
+def backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src):
+    """moe_backward (the training pass: forward recompute and every gradient,
+    bf16 gradient outputs) on the same weights, timed like the forward."""
+    from mixture_experts_ffn_17_b200 import binding as B
+    shape = B.shape_of(cfg, B.MOE_BF16)
+    ws = B.alloc_backward_workspace(shape, dev)
+    e = lambda *sz: torch.empty(sz, dtype=torch.bfloat16, device=dev)
+    grads = [e(cfg.T, cfg.d), e(cfg.E, cfg.d), e(cfg.E, cfg.d, cfg.inter), e(cfg.E, cfg.d, cfg.inter),
+             e(cfg.E, cfg.inter, cfg.d), e(cfg.d, cfg.shared_inter), e(cfg.d, cfg.shared_inter),
+             e(cfg.shared_inter, cfg.d)]
+    dy = torch.randn(cfg.T, cfg.d, generator=torch.Generator(device=dev).manual_seed(cfg.seed + 100), device=dev)
+    bargs = (shape, w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.W1s, w.W3s, w.W2s, dy, *grads, ws)
+    for _ in range(max(3, args.warmup)):
+        B.backward(*bargs)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"backward: device status after warm-up (raw {raw})")
+    K = max(5, args.steps // 2)
+    ms, clocks = time_loop(lambda i: B.backward(*bargs), K, stream, dev, dist)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"backward: device status after the timed steps (raw {raw})")
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    y = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device=dev)
+    fws = B.alloc_workspace(B.shape_of(cfg, B.MOE_F32), dev)
+    B.forward(B.shape_of(cfg, B.MOE_F32), w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s,
+              y, fws, counts=counts)
+    flops, nbytes = backward_work(cfg, counts.cpu().numpy(), 2)
+    t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    d_roof = max(flops / (DATASHEET_PEAKS["bf16_tflops"] * 1e12), nbytes / (DATASHEET_PEAKS["hbm_gbs"] * 1e9))
+    return {"what": "moe_backward: forward recompute + dx, dWg, dW1, dW3, dW2 and the shared expert's gradients "
+                    "(bf16 gradient outputs, fp32 dy)",
+            "steps": K, "ms_per_step": ms, "tokens_per_s": dist.world * cfg.T / (ms / 1e3),
+            "tflops": dist.world * flops / (ms / 1e3) / 1e12, "flops": flops, "bytes": nbytes,
+            "roofline_ms": 1e3 * max(t_tc, t_hbm), "bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "frac": 1e3 * max(t_tc, t_hbm) / ms, "frac_datasheet": 1e3 * d_roof / ms,
+            "peaks": peak_src, "clocks": clocks}
+
+
 def run_ours(args, dist):
     from mixture_experts_ffn_17_b200 import binding as B
     from mixture_experts_ffn_17_b200 import workloads
@@ -550,10 +607,14 @@ def run_ours(args, dist):
         line["e2e"] = e2e
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = run_cpu_baseline(args, w, cfg)
+    if args.workload == "prefill" and not (args.tokens or args.experts or args.no_backward):
+        fwd_args = None
+        line["backward"] = backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src)
+        torch.cuda.empty_cache()
     if args.workload == "prefill" and not (args.tokens or args.experts or args.no_decode):
         # the decode batch of the same layer shapes, in the same run (its own
         # weights; the prefill ones are released first)
-        del w, ws, fwd_args, y
+        fwd_args = w = ws = y = None
         torch.cuda.empty_cache()
         line["decode"] = decode_record(args, dist, dev, stream, peaks, peak_src)
         line["config"]["workload"] += "; decode record: " + line["decode"]["workload"]

@@ -222,6 +222,42 @@ moe_status moe_combine_backward(const moe_shape* shape, const float* dy, const v
 moe_status moe_router_backward(const moe_shape* shape, const float* logits, const int32_t* topk_idx,
                                const float* topk_w, const float* dw, float* dlogits, void* stream);
 
+/* Gradient of the whole layer (training): for the loss sum(dy * y) with
+ * y = moe_forward(...), the gradients with respect to x, Wg, W1, W3, W2 and
+ * the shared expert's weights, the expert selection held fixed (it is
+ * piecewise constant in the inputs; the selection bias only moves it and gets
+ * no gradient).  The pages print no backward arithmetic (the n4n page's
+ * "Training infrastructure that made this possible" only names training);
+ * this is the chain rule through the forward steps of the atlas page ("All 5
+ * steps", and the MoE forward block of its "Code" section):
+ *   dO = w dy (per routed slot),  dw = dy . o,  dl from dw through the weight
+ *   rule (as moe_router_backward),
+ *   dH = dO W2^T,  dG = dH u silu'(g),  dU = dH silu(g),
+ *   dW2 = H^T dO,  dW1 = X^T dG,  dW3 = X^T dU   (each expert over its rows),
+ *   dx = sum over slots of (dG W1^T + dU W3^T) + the shared expert's input
+ *        gradient + dl Wg,   dWg = dl^T x,
+ * with silu'(g) = sigmoid(g) (1 + g (1 - sigmoid(g))).  The call recomputes
+ * the forward (routing, g, u, H and the expert outputs; they stay in the
+ * workspace) and then runs the backward steps, all on the device, with no
+ * host synchronisation and no atomics (deterministic results).
+ *   x, Wg, bias, W1, W3, W2, W1s, W3s, W2s: as moe_forward (bf16 experts only:
+ *     w_dtype must be MOE_BF16, else MOE_ERR_UNSUPPORTED)
+ *   dy [T, d] fp32: gradient of the layer output
+ *   outputs, all in shape->y_dtype (fp32 or bf16), row-major, every element
+ *   written (experts no token chose get zero):
+ *     dx [T, d]; dWg [E, d]; dW1, dW3 [E, d, inter]; dW2 [E, inter, d];
+ *     dW1s, dW3s [d, shared_inter], dW2s [shared_inter, d] (NULL when there is
+ *     no shared expert)
+ *   ws: caller-owned device workspace of moe_backward_workspace_size(shape)
+ *     bytes, 256-byte aligned (its head holds the status word that
+ *     moe_check_device_status reads).
+ * Errors as moe_forward. */
+size_t moe_backward_workspace_size(const moe_shape* shape);
+moe_status moe_backward(const moe_shape* shape, const void* x, const void* Wg, const float* bias, const void* W1,
+                        const void* W3, const void* W2, const void* W1s, const void* W3s, const void* W2s,
+                        const float* dy, void* dx, void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s,
+                        void* dW2s, void* ws, size_t ws_bytes, void* stream);
+
 /* The whole layer: router, dispatch, grouped experts, shared expert and
  * combine, with no host synchronisation.
  *   y [T, d] out (fp32 or bf16 per shape->y_dtype)

@@ -24,7 +24,8 @@ MOE_ROUTE_TOPK_SOFTMAX, MOE_ROUTE_SIGMOID_GROUP = 0, 1
 EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine",
             "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version",
             "moe_permute_noalloc", "moe_router_topk_limited", "moe_expert_utilisation", "moe_forward_ep",
-            "moe_forward_launches", "moe_combine_backward", "moe_router_backward")
+            "moe_forward_launches", "moe_combine_backward", "moe_router_backward", "moe_backward_workspace_size",
+            "moe_backward")
 NUM_STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "experts_up", "experts_down", "combine")
 
@@ -85,10 +86,13 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_ep.argtypes = [S, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_forward_launches.argtypes = [S]
         L.moe_forward_launches.restype = ctypes.c_int
+        L.moe_backward_workspace_size.argtypes = [S]
+        L.moe_backward_workspace_size.restype = sz
+        L.moe_backward.argtypes = [S] + [P] * 18 + [P, sz, P]
         L.moe_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         for fn in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_combine_backward",
                    "moe_router_backward", "moe_forward",
-                   "moe_forward_profiled", "moe_forward_ep", "moe_check_device_status"):
+                   "moe_forward_profiled", "moe_forward_ep", "moe_backward", "moe_check_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -223,6 +227,27 @@ def forward_profiled(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, 
                                       _ptr(y), _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(ws),
                                       ws.numel() if ws is not None else 0, _stream(stream), handles),
            "moe_forward_profiled")
+
+
+def backward_workspace_size(shape: MoeShape) -> int:
+    return int(lib().moe_backward_workspace_size(ctypes.byref(shape)))
+
+
+def alloc_backward_workspace(shape: MoeShape, device="cuda") -> torch.Tensor:
+    n = backward_workspace_size(shape)
+    if n == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_backward_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def backward(shape, x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, dy, dx, dWg, dW1, dW3, dW2, dW1s, dW3s, dW2s, ws,
+             stream=None):
+    """Gradient of sum(dy * y) of the layer (moe_backward): dx, dWg, dW1, dW3,
+    dW2 and the shared expert's dW1s, dW3s, dW2s, in shape.y_dtype."""
+    _check(lib().moe_backward(ctypes.byref(shape), _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2),
+                              _ptr(W1s), _ptr(W3s), _ptr(W2s), _ptr(dy), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3),
+                              _ptr(dW2), _ptr(dW1s), _ptr(dW3s), _ptr(dW2s), _ptr(ws),
+                              ws.numel() if ws is not None else 0, _stream(stream)), "moe_backward")
 
 
 def check_device_status(ws, stream=None) -> tuple[int, int]:

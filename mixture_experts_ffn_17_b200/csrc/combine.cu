@@ -34,7 +34,7 @@ __global__ void __launch_bounds__(128)
     // a shard adds only the rows of its own experts
     if (offsets && (r < offsets[e_lo] || r >= offsets[e_hi])) r = -1;
     rows[threadIdx.x] = r;
-    ws[threadIdx.x] = topk_w[t * k + threadIdx.x];
+    ws[threadIdx.x] = topk_w ? topk_w[t * k + threadIdx.x] : 1.0f;  // no weights: a plain sum
   }
   __syncthreads();
   const int nv = d / 8;

@@ -523,6 +523,23 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
 #pragma unroll
                 for (int v = 0; v < 4; ++v)
                   out[c * 4 + v] = make_uint4(hp[4 * v], hp[4 * v + 1], hp[4 * v + 2], hp[4 * v + 3]);
+                if (p.out_gu) {
+                  // the backward pass's copy of g and u (bf16, same row as H)
+                  uint16_t* gu_row = static_cast<uint16_t*>(p.out_gu) + hrow * 2 * p.ld_out + n0 + c * 32;
+                  uint4* og = reinterpret_cast<uint4*>(gu_row);
+                  uint4* ou = reinterpret_cast<uint4*>(gu_row + p.ld_out);
+#pragma unroll
+                  for (int v = 0; v < 4; ++v) {
+                    og[v] = make_uint4(ptx::pack_bf16x2(__uint_as_float(g[8 * v]), __uint_as_float(g[8 * v + 1])),
+                                       ptx::pack_bf16x2(__uint_as_float(g[8 * v + 2]), __uint_as_float(g[8 * v + 3])),
+                                       ptx::pack_bf16x2(__uint_as_float(g[8 * v + 4]), __uint_as_float(g[8 * v + 5])),
+                                       ptx::pack_bf16x2(__uint_as_float(g[8 * v + 6]), __uint_as_float(g[8 * v + 7])));
+                    ou[v] = make_uint4(ptx::pack_bf16x2(__uint_as_float(u[8 * v]), __uint_as_float(u[8 * v + 1])),
+                                       ptx::pack_bf16x2(__uint_as_float(u[8 * v + 2]), __uint_as_float(u[8 * v + 3])),
+                                       ptx::pack_bf16x2(__uint_as_float(u[8 * v + 4]), __uint_as_float(u[8 * v + 5])),
+                                       ptx::pack_bf16x2(__uint_as_float(u[8 * v + 6]), __uint_as_float(u[8 * v + 7])));
+                  }
+                }
               }
             } else {
               const int64_t orow = (int64_t)ti.row0 + r + (ti.shared ? p.out_shared_row_offset : 0);

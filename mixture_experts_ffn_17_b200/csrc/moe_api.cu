@@ -435,6 +435,314 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   return MOE_OK;
 }
 
+// ------------------------------------------------------------ backward pass
+// Workspace of moe_backward: the forward's layout (routing, dispatch, x_perm,
+// H, Y_perm) and the backward's own buffers after it.
+struct BwdLayout {
+  Layout f;
+  size_t tiles, gu, dgu, dO, dy_b, dw, dl, dl_b, wgT, dX, dXs, total;
+  int max_mtiles, Ep;
+  int64_t rows;  // T*k routed rows + T shared rows of gu / dgu
+};
+
+BwdLayout make_bwd_layout(const moe_shape& s) {
+  BwdLayout B{};
+  B.f = make_layout(s);
+  const int64_t T = s.T, Tk = s.T * s.k;
+  size_t off = B.f.total;
+  auto take = [&](size_t bytes) {
+    size_t at = off;
+    off += align_up(std::max<size_t>(bytes, 1));
+    return at;
+  };
+  // the shared expert's tiles are always listed: with no shared expert they
+  // still carry the router's part of the input gradient (dl Wg)
+  B.max_mtiles = (int)((Tk + kTileRows - 1) / kTileRows + s.E + (T + kTileRows - 1) / kTileRows);
+  B.Ep = (s.E + 63) / 64 * 64;
+  B.rows = Tk + T;
+  const int64_t Hld = B.f.Hld;
+  B.tiles = take((size_t)B.max_mtiles * 16);
+  B.gu = take((size_t)B.rows * 2 * Hld * 2);
+  B.dgu = take((size_t)B.rows * 2 * Hld * 2);
+  B.dO = take((size_t)Tk * s.d * 2);
+  B.dy_b = take((size_t)T * s.d * 2);
+  B.dw = take((size_t)Tk * 4);
+  B.dl = take((size_t)T * s.E * 4);
+  B.dl_b = take((size_t)T * B.Ep * 2);
+  B.wgT = take((size_t)s.d * B.Ep * 2);
+  B.dX = take((size_t)Tk * s.d * 2);
+  B.dXs = take((size_t)T * s.d * 4);
+  B.total = off;
+  return B;
+}
+
+moe_status validate_backward(const moe_shape* s) {
+  moe_status v = validate_shape(s);
+  if (v != MOE_OK) return v;
+  if (s->w_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;  // bf16 experts only
+  return MOE_OK;
+}
+
+// bf16 row-major [outer, inner] map with [box_outer rows x 64] boxes
+bool map_rows(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+  return map_2d(m, ptr, inner, outer, 64, box_outer);
+}
+
+moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, const float* bias, const void* W1,
+                         const void* W3, const void* W2, const void* W1s, const void* W3s, const void* W2s,
+                         const float* dy, void* dx, void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s,
+                         void* dW2s, void* ws, cudaStream_t st) {
+  const BwdLayout B = make_bwd_layout(s);
+  const Layout& L = B.f;
+  const bool sh = s.shared_inter > 0;
+  const int64_t T = s.T, Tk = s.T * s.k;
+  const int Hld = L.Hld;
+  const int sms = num_sms();
+  const bool gbf16 = s.y_dtype == MOE_BF16;
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  int32_t* idx = at<int32_t>(ws, L.idx);
+  float* w = at<float>(ws, L.w);
+  float* logits = at<float>(ws, L.logits);
+  int32_t* counts = at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* perm = at<int32_t>(ws, L.perm);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  void* x_perm = at<void>(ws, L.x_perm);
+  uint16_t* H = at<uint16_t>(ws, L.H);
+  void* Y_perm = at<void>(ws, L.Y_perm);
+  int4* tiles = at<int4>(ws, B.tiles);
+  int32_t* ntiles = at<int32_t>(ws, L.ntiles);
+  int* sched = at<int>(ws, L.sched);
+  void* GU = at<void>(ws, B.gu);
+  void* dGU = at<void>(ws, B.dgu);
+  void* dO = at<void>(ws, B.dO);
+  void* dy_b = at<void>(ws, B.dy_b);
+  float* dw = at<float>(ws, B.dw);
+  float* dl = at<float>(ws, B.dl);
+  void* dl_b = at<void>(ws, B.dl_b);
+  void* wgT = at<void>(ws, B.wgT);
+  void* dX = at<void>(ws, B.dX);
+  float* dXs = at<float>(ws, B.dXs);
+
+  // ---- forward, keeping what the gradient needs: logits, routing, x_perm,
+  // g and u (bf16), H, and the routed expert outputs Y_perm
+  moe_status r = run_router(s, x, Wg, bias, idx, w, logits, at<double>(ws, L.rpart), status, st);
+  if (r != MOE_OK) return r;
+  MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
+                          perm, row_of, status, st));
+  MOE_CUDA(launch_gather_rows(x, perm, Tk, s.d, x_perm, sms, st, offsets, 0, s.E));
+  MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, whole_layer(s), true, tiles, ntiles, sched, st, nullptr));
+
+  CUtensorMap a_r, a_s, w1_r, w1_s, w3_r, w3_s;
+  if (!map_2d(&a_r, x_perm, s.d, Tk, kGemmBK, kTileM) || !map_2d(&a_s, x, s.d, s.T, kGemmBK, kTileM) ||
+      !map_3d(&w1_r, W1, s.inter, s.d, s.E, kGemmBK) || !map_3d(&w3_r, W3, s.inter, s.d, s.E, kGemmBK))
+    return MOE_ERR_CUDA;
+  if (sh) {
+    if (!map_3d(&w1_s, W1s, s.shared_inter, s.d, 1, kGemmBK) || !map_3d(&w3_s, W3s, s.shared_inter, s.d, 1, kGemmBK))
+      return MOE_ERR_CUDA;
+  } else {
+    w1_s = w1_r;  // placeholders: shared tiles have no columns without a shared expert
+    w3_s = w3_r;
+  }
+  GemmParams p1{};
+  p1.tiles = tiles;
+  p1.ntiles = ntiles;
+  p1.max_mtiles = B.max_mtiles;
+  p1.tile_set = kTilesAll;
+  p1.E = s.E;
+  p1.group_base = 0;
+  p1.n_nb = (Hld + gemm_block_n_swiglu() - 1) / gemm_block_n_swiglu();
+  p1.K_routed = s.d;
+  p1.K_shared = s.d;
+  p1.N_routed = s.inter;
+  p1.N_shared = s.shared_inter;
+  p1.out_routed = H;
+  p1.out_shared = H;
+  p1.out_shared_row_offset = Tk;
+  p1.ld_out = Hld;
+  p1.status = status;
+  p1.sched_counter = sched + 0;
+  p1.out_gu = GU;
+  const int grid1 = (int)std::min<int64_t>(sms, (int64_t)B.max_mtiles * p1.n_nb);
+  MOE_CUDA(launch_grouped_swiglu(a_r, a_s, w1_r, w1_s, w3_r, w3_s, p1, grid1, st));
+
+  CUtensorMap h_map, w2_r, w2_s;
+  if (!map_2d(&h_map, H, Hld, L.Hrows, kGemmBK, kTileM) || !map_3d(&w2_r, W2, s.d, s.inter, s.E, kGemmBK))
+    return MOE_ERR_CUDA;
+  w2_s = w2_r;
+  GemmParams p2 = p1;
+  p2.out_gu = nullptr;
+  p2.tile_set = kTilesRouted;  // Y_perm only: the shared expert's output has no gradient use
+  p2.sched_counter = sched + 2;
+  p2.n_nb = (s.d + gemm_block_n_down() - 1) / gemm_block_n_down();
+  p2.K_routed = s.inter;
+  p2.K_shared = s.shared_inter;
+  p2.N_routed = s.d;
+  p2.N_shared = s.d;
+  p2.a_shared_row_offset = (int)Tk;
+  p2.out_routed = Y_perm;
+  p2.out_shared = nullptr;
+  p2.ld_out = s.d;
+  const int grid2 = (int)std::min<int64_t>(sms, (int64_t)B.max_mtiles * p2.n_nb);
+  MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, p2, grid2, st));
+
+  // ---- combine and routing steps
+  MOE_CUDA(launch_combine_backward(dy, Y_perm, row_of, w, s.T, s.k, s.d, dO, dw, st));
+  MOE_CUDA(launch_router_backward(logits, idx, w, dw, s.T, s.E, s.k, s.route == MOE_ROUTE_SIGMOID_GROUP ? 1 : 0,
+                                  s.route_scale, dl, st));
+  MOE_CUDA(launch_cast_pad_bf16(dl, T, s.E, B.Ep, dl_b, sms, st));
+  MOE_CUDA(launch_cast_pad_bf16(dy, T, s.d, s.d, dy_b, sms, st));
+  MOE_CUDA(launch_transpose_pad_bf16(Wg, s.E, s.d, B.Ep, wgT, st));
+
+  // ---- dH = dO W2^T (routed), dy W2s^T (shared) -> dG | dU
+  {
+    DgradMaps m{};
+    if (!map_rows(&m.a[0], dO, s.d, Tk, kTileM) || !map_rows(&m.a[1], dy_b, s.d, T, kTileM) ||
+        !map_3d(&m.b[0], W2, s.d, s.inter, s.E, 256))
+      return MOE_ERR_CUDA;
+    if (sh) {
+      if (!map_3d(&m.b[1], W2s, s.d, s.shared_inter, 1, 256)) return MOE_ERR_CUDA;
+    } else {
+      m.b[1] = m.b[0];
+    }
+    m.a[2] = m.a[0];
+    m.b[2] = m.b[3] = m.b[4] = m.b[0];
+    DgradParams q{};
+    q.tiles = tiles;
+    q.ntiles = ntiles;
+    q.max_mtiles = B.max_mtiles;
+    q.E = s.E;
+    q.n_nb = (Hld + 255) / 256;
+    q.N_routed = s.inter;
+    q.N_shared = s.shared_inter;  // 0: the shared tiles are skipped
+    q.parts_routed[0] = KPart{s.d / 64, kMapA0, 0, 0, kMapB0};
+    q.n_parts_routed = 1;
+    q.parts_shared[0] = KPart{s.d / 64, kMapA1, 0, 0, kMapB1};
+    q.n_parts_shared = 1;
+    q.gu = GU;
+    q.ld_gu = 2 * (int64_t)Hld;
+    q.u_off = Hld;
+    q.shared_row_off = Tk;
+    q.out_routed = dGU;
+    q.status = status;
+    MOE_CUDA(launch_dgrad(kDgradH, m, q, (int)std::min<int64_t>(sms, (int64_t)B.max_mtiles * q.n_nb), st));
+  }
+  // ---- dX = [dG | dU] [W1 ; W3]^T (routed rows), and for the shared expert's
+  // tiles [dGs | dUs] [W1s ; W3s]^T + dl Wg
+  {
+    DgradMaps m{};
+    if (!map_rows(&m.a[0], dGU, 2 * (uint64_t)Hld, B.rows, kTileM) || !map_rows(&m.a[1], dl_b, B.Ep, T, kTileM) ||
+        !map_3d(&m.b[0], W1, s.inter, s.d, s.E, 256) || !map_3d(&m.b[1], W3, s.inter, s.d, s.E, 256) ||
+        !map_3d(&m.b[4], wgT, B.Ep, s.d, 1, 256))
+      return MOE_ERR_CUDA;
+    if (sh) {
+      if (!map_3d(&m.b[2], W1s, s.shared_inter, s.d, 1, 256) || !map_3d(&m.b[3], W3s, s.shared_inter, s.d, 1, 256))
+        return MOE_ERR_CUDA;
+    } else {
+      m.b[2] = m.b[3] = m.b[0];
+    }
+    m.a[2] = m.a[0];
+    DgradParams q{};
+    q.tiles = tiles;
+    q.ntiles = ntiles;
+    q.max_mtiles = B.max_mtiles;
+    q.E = s.E;
+    q.n_nb = (s.d + 255) / 256;
+    q.N_routed = s.d;
+    q.N_shared = s.d;
+    q.parts_routed[0] = KPart{s.inter / 64, kMapA0, 0, 0, kMapB0};
+    q.parts_routed[1] = KPart{s.inter / 64, kMapA0, Hld, 0, kMapB1};
+    q.n_parts_routed = 2;
+    int np = 0;
+    if (sh) {
+      q.parts_shared[np++] = KPart{s.shared_inter / 64, kMapA0, 0, (int)Tk, kMapB2};
+      q.parts_shared[np++] = KPart{s.shared_inter / 64, kMapA0, Hld, (int)Tk, kMapB3};
+    }
+    q.parts_shared[np++] = KPart{B.Ep / 64, kMapA1, 0, 0, kMapB4};
+    q.n_parts_shared = np;
+    q.out_routed = dX;
+    q.out_shared = dXs;
+    q.ld_out = s.d;
+    q.status = status;
+    MOE_CUDA(launch_dgrad(kDgradX, m, q, (int)std::min<int64_t>(sms, (int64_t)B.max_mtiles * q.n_nb), st));
+  }
+  // ---- dx[t] = sum_j dX[row_of[t, j]] + dX_shared[t] (which holds dl Wg)
+  MOE_CUDA(launch_combine(dX, dXs, row_of, nullptr, s.T, s.k, s.d, dx, gbf16, st));
+
+  // ---- weight gradients
+  {
+    CUtensorMap ax_r, ax_s, bg;
+    if (!map_rows(&ax_r, x_perm, s.d, Tk, 64) || !map_rows(&ax_s, x, s.d, T, 64) ||
+        !map_rows(&bg, dGU, 2 * (uint64_t)Hld, B.rows, 64))
+      return MOE_ERR_CUDA;
+    WgradParams q{};
+    q.offsets = offsets;
+    q.n_routed = s.E;
+    q.has_shared = sh ? 1 : 0;
+    q.mb_routed = s.d / 128;
+    q.nb_routed = s.inter / 128;
+    q.mb_shared = s.d / 128;
+    q.nb_shared = s.shared_inter / 128;
+    q.M_routed = q.M_shared = s.d;
+    q.ncols_routed = s.inter;
+    q.ncols_shared = s.shared_inter;
+    q.a_shared_row0 = 0;
+    q.b_shared_row0 = (int)Tk;
+    q.shared_rows = s.T;
+    q.u_off = Hld;
+    q.out1 = dW1;
+    q.out2 = dW3;
+    q.out1_shared = dW1s;
+    q.out2_shared = dW3s;
+    q.out_bf16 = gbf16 ? 1 : 0;
+    q.status = status;
+    MOE_CUDA(launch_wgrad(kWgradW13, ax_r, ax_s, bg, bg, q, sms, st));
+  }
+  {
+    CUtensorMap ah, bo_r, bo_s;
+    if (!map_rows(&ah, H, Hld, L.Hrows, 64) || !map_rows(&bo_r, dO, s.d, Tk, 64) ||
+        !map_rows(&bo_s, dy_b, s.d, T, 64))
+      return MOE_ERR_CUDA;
+    WgradParams q{};
+    q.offsets = offsets;
+    q.n_routed = s.E;
+    q.has_shared = sh ? 1 : 0;
+    q.mb_routed = s.inter / 128;
+    q.nb_routed = (s.d + 255) / 256;
+    q.mb_shared = s.shared_inter / 128;
+    q.nb_shared = (s.d + 255) / 256;
+    q.M_routed = s.inter;
+    q.M_shared = s.shared_inter;
+    q.ncols_routed = q.ncols_shared = s.d;
+    q.a_shared_row0 = (int)Tk;
+    q.b_shared_row0 = 0;
+    q.shared_rows = s.T;
+    q.out1 = dW2;
+    q.out1_shared = dW2s;
+    q.out_bf16 = gbf16 ? 1 : 0;
+    q.status = status;
+    MOE_CUDA(launch_wgrad(kWgradPlain, ah, ah, bo_r, bo_s, q, sms, st));
+  }
+  {
+    CUtensorMap al, bx;
+    if (!map_rows(&al, dl_b, B.Ep, T, 64) || !map_rows(&bx, x, s.d, T, 64)) return MOE_ERR_CUDA;
+    WgradParams q{};
+    q.offsets = offsets;
+    q.n_routed = 0;
+    q.has_shared = 1;
+    q.mb_shared = (s.E + 127) / 128;
+    q.nb_shared = (s.d + 255) / 256;
+    q.M_shared = s.E;
+    q.ncols_shared = s.d;
+    q.shared_rows = s.T;
+    q.out1_shared = dWg;
+    q.out_bf16 = gbf16 ? 1 : 0;
+    q.status = status;
+    MOE_CUDA(launch_wgrad(kWgradPlain, al, al, bx, bx, q, sms, st));
+  }
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -638,6 +946,47 @@ moe_status moe_forward_ep(const moe_shape* shape, int ep_rank, int ep_size, cons
                           void* stream) {
   return forward_impl(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out,
                       counts_out, ws, ws_bytes, stream, nullptr, ep_rank, ep_size);
+}
+
+size_t moe_backward_workspace_size(const moe_shape* shape) {
+  if (validate_backward(shape) != MOE_OK) return 0;
+  return make_bwd_layout(*shape).total;
+}
+
+moe_status moe_backward(const moe_shape* shape, const void* x, const void* Wg, const float* bias, const void* W1,
+                        const void* W3, const void* W2, const void* W1s, const void* W3s, const void* W2s,
+                        const float* dy, void* dx, void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s,
+                        void* dW2s, void* ws, size_t ws_bytes, void* stream) {
+  moe_status v = validate_backward(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  const bool sh = s.shared_inter > 0;
+  if (!x || !Wg || !W1 || !W3 || !W2 || !dy || !dx || !dWg || !dW1 || !dW3 || !dW2) return MOE_ERR_INVALID_ARG;
+  if (sh && (!W1s || !W3s || !W2s || !dW1s || !dW3s || !dW2s)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, dy, dx, dWg, dW1, dW3, dW2, dW1s, dW3s, dW2s};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const BwdLayout B = make_bwd_layout(s);
+  if (!ws_ok(ws, ws_bytes, B.total)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_CUDA(cudaMemsetAsync(at<uint32_t>(ws, B.f.status), 0, 4, st));
+  if (s.T == 0) {
+    // no tokens: every weight gradient is zero
+    const size_t gb = s.y_dtype == MOE_BF16 ? 2 : 4;
+    const size_t eI = (size_t)s.E * s.d * s.inter * gb, sI = (size_t)s.d * s.shared_inter * gb;
+    MOE_CUDA(cudaMemsetAsync(dWg, 0, (size_t)s.E * s.d * gb, st));
+    MOE_CUDA(cudaMemsetAsync(dW1, 0, eI, st));
+    MOE_CUDA(cudaMemsetAsync(dW3, 0, eI, st));
+    MOE_CUDA(cudaMemsetAsync(dW2, 0, eI, st));
+    if (sh) {
+      MOE_CUDA(cudaMemsetAsync(dW1s, 0, sI, st));
+      MOE_CUDA(cudaMemsetAsync(dW3s, 0, sI, st));
+      MOE_CUDA(cudaMemsetAsync(dW2s, 0, sI, st));
+    }
+    return MOE_OK;
+  }
+  return backward_impl(s, x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, dy, dx, dWg, dW1, dW3, dW2, dW1s, dW3s, dW2s, ws,
+                       st);
 }
 
 moe_status moe_check_device_status(const void* ws, void* stream, uint32_t* raw) {

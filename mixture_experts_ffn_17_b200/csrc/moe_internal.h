@@ -121,6 +121,11 @@ struct GemmParams {
   // Failure-path testing: when nonzero the producer issues no loads, so the
   // MMA issuer's bounded wait runs out and the launch reports a timeout.
   int debug_withhold_loads;
+  // SwiGLU, bf16 weights, one-CTA kernel (the backward pass keeps the
+  // forward's g and u): when non-null, g and u are also stored bf16 in rows of
+  // 2 * ld_out elements, g at column n and u at column ld_out + n, on the same
+  // rows as H.
+  void* out_gu;
 };
 
 int gemm_block_n_swiglu();
@@ -155,7 +160,7 @@ cudaError_t launch_grouped_down_fp8(const CUtensorMap& tmA, const CUtensorMap& t
 
 // combine.cu
 // offsets != nullptr: only permuted rows of experts [shard.e_lo, shard.e_hi)
-// are added.
+// are added.  topk_w == nullptr: every row has weight 1.
 cudaError_t launch_combine(const void* Y_perm, const float* Y_shared, const int32_t* row_of, const float* topk_w,
                            int64_t T, int k, int d, void* y, bool y_bf16, cudaStream_t stream,
                            const int32_t* offsets = nullptr, const Shard* shard = nullptr);

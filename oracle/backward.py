@@ -1,8 +1,8 @@
 """fp64 gradient of the MoE feed-forward layer.
 
 TEST INFRASTRUCTURE ONLY, like the rest of this package: only the tests may
-import it.  The library's backward kernels (the combine and routing steps so
-far) are checked against it.
+import it.  The library's backward pass (moe_backward and its combine and
+routing steps) is checked against it.
 
 The pages define the forward pass only (n4n.ai page "DeepSeek-V3's
 mixture-of-experts architecture explained", "The architecture in one diagram";
@@ -33,6 +33,7 @@ from . import logits as _logits
 from . import route_sigmoid_group as _route_group
 from . import route_topk_softmax as _route_topk
 from . import swiglu_rows as _swiglu_rows
+from . import weights_for as _weights_for
 
 
 def _sigmoid(z: np.ndarray) -> np.ndarray:
@@ -94,7 +95,8 @@ def routing_backward(lg_sel: np.ndarray, w: np.ndarray, dw: np.ndarray, route: i
 
 
 def moe_backward(x, Wg, W1, W3, W2, W1s=None, W3s=None, W2s=None, *, dy, k: int, route: int = 0, bias=None,
-                 n_group: int = 1, topk_group: int = 1, group_topn: int = 2, route_scale: float = 2.5):
+                 n_group: int = 1, topk_group: int = 1, group_topn: int = 2, route_scale: float = 2.5,
+                 force_idx=None):
     """Gradient of sum(dy * y) for the layer y = moe_forward(...) (fp64).
 
     Shapes as the forward oracle: x [T, d], Wg [E, d], W1/W3 [E, d, I],
@@ -103,12 +105,17 @@ def moe_backward(x, Wg, W1, W3, W2, W1s=None, W3s=None, W2s=None, *, dy, k: int,
     shared expert is present); the intermediate gradients dO_perm (of the
     routed expert outputs, permuted order), dw (of the routing weights) and dl
     (of the logits); and the selection idx, weights w, logits lg, permuted
-    expert outputs Y_perm, row_of and the forward output y it was computed at."""
+    expert outputs Y_perm, row_of and the forward output y it was computed at.
+    force_idx [T, k]: use this selection (weights from the same rule) instead
+    of selecting, as the forward oracle's force_idx does."""
     x, Wg, W1, W3, W2, dy = (np.asarray(a, dtype=np.float64) for a in (x, Wg, W1, W3, W2, dy))
     T, d = x.shape
     E = W1.shape[0]
     lg = _logits(x, Wg)
-    if route == 0:
+    if force_idx is not None:
+        idx = np.ascontiguousarray(force_idx, dtype=np.int32)
+        w = _weights_for(lg, idx, route, route_scale)
+    elif route == 0:
         idx, w, _ = _route_topk(lg, k)
     else:
         idx, w, _, _ = _route_group(lg, bias, k, n_group, topk_group, group_topn, route_scale)

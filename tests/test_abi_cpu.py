@@ -204,3 +204,28 @@ def test_forward_launch_count_with_cta_pairs_forced(monkeypatch):
     assert B.forward_launches(B.shape_of(workloads.CONFIGS["fp8"])) == 16
     monkeypatch.setenv("MOE_PAIR_TILES", "0")
     assert B.forward_launches(B.shape_of(workloads.CONFIGS["skewed"])) == 10
+
+
+def test_backward_validation_without_gpu():
+    L = B.lib()
+    s = B.make_shape(T=128, d=512, E=32, k=4, inter=256, shared_inter=256)
+    n = B.backward_workspace_size(s)
+    assert n > B.workspace_size(s)           # the forward's buffers and the backward's after them
+    keep, p = _fake()
+    nul = None
+    # x Wg bias W1 W3 W2 W1s W3s W2s dy | dx dWg dW1 dW3 dW2 dW1s dW3s dW2s | ws n stream
+    args = [p, p, nul, p, p, p, p, p, p, p, p, p, p, p, p, p, p, p, p, n, nul]
+    for i in (0, 1, 3, 9, 10, 11, 12, 13, 14, 15):
+        a = list(args); a[i] = nul
+        assert L.moe_backward(ctypes.byref(s), *a) == B.MOE_ERR_INVALID_ARG, i
+    a = list(args); a[19] = n - 1
+    assert L.moe_backward(ctypes.byref(s), *a) == B.MOE_ERR_WORKSPACE
+    a = list(args); a[10] = ctypes.c_void_p(p.value + 4)
+    assert L.moe_backward(ctypes.byref(s), *a) == B.MOE_ERR_INVALID_ARG
+    # the backward pass takes bf16 experts only
+    s8 = B.make_shape(T=128, d=512, E=32, k=4, inter=256, shared_inter=256, w_dtype=B.MOE_E4M3)
+    assert B.backward_workspace_size(s8) == 0
+    assert L.moe_backward(ctypes.byref(s8), *args) == B.MOE_ERR_UNSUPPORTED
+    # without a shared expert its weights and gradients may be NULL
+    s0 = B.make_shape(T=128, d=512, E=32, k=4, inter=256, shared_inter=0)
+    assert B.backward_workspace_size(s0) > 0

@@ -133,3 +133,153 @@ def test_backward_steps_after_the_forward_match_the_layer_gradient():
         # same selection everywhere: the permuted rows line up with the oracle's
         dO_d = dec(dO)
         assert np.max(np.abs(dO_d - g["dO_perm"])) <= 2.0 ** -8 * np.abs(g["dO_perm"]).max()
+
+
+# ------------------------------------------------------ the whole backward pass
+def _backward(w, dy, grad_bf16=False):
+    """moe_backward on the device -> dict of gradients (torch tensors)."""
+    cfg = w.cfg
+    shape = B.shape_of(cfg, B.MOE_BF16 if grad_bf16 else B.MOE_F32)
+    ws = B.alloc_backward_workspace(shape)
+    dt = torch.bfloat16 if grad_bf16 else torch.float32
+    z = lambda *s: torch.full(s, float("nan"), dtype=dt, device="cuda")   # every element must be written
+    g = dict(dx=z(cfg.T, cfg.d), dWg=z(cfg.E, cfg.d), dW1=z(cfg.E, cfg.d, cfg.inter), dW3=z(cfg.E, cfg.d, cfg.inter),
+             dW2=z(cfg.E, cfg.inter, cfg.d))
+    sh = cfg.shared_inter > 0
+    if sh:
+        g.update(dW1s=z(cfg.d, cfg.shared_inter), dW3s=z(cfg.d, cfg.shared_inter), dW2s=z(cfg.shared_inter, cfg.d))
+    B.backward(shape, w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.W1s, w.W3s, w.W2s, dy, g["dx"], g["dWg"], g["dW1"],
+               g["dW3"], g["dW2"], g.get("dW1s"), g.get("dW3s"), g.get("dW2s"), ws)
+    rc, raw = B.check_device_status(ws)
+    assert rc == B.MOE_OK, (rc, raw)
+    return g, ws
+
+
+def _oracle_backward(w, dy, force_idx=None):
+    cfg = w.cfg
+    sh = {} if cfg.shared_inter == 0 else dict(W1s=dec(w.W1s), W3s=dec(w.W3s), W2s=dec(w.W2s))
+    return obw.moe_backward(dec(w.x), dec(w.Wg), dec(w.W1), dec(w.W3), dec(w.W2), dy=to_np(dy).astype(np.float64),
+                            k=cfg.k, route=cfg.route, bias=None if w.bias is None else dec(w.bias),
+                            n_group=cfg.n_group, topk_group=cfg.topk_group, group_topn=cfg.group_topn,
+                            route_scale=cfg.route_scale, force_idx=force_idx, **sh)
+
+
+GRADS = ("dx", "dWg", "dW1", "dW3", "dW2", "dW1s", "dW3s", "dW2s")
+PER_EXPERT = ("dW1", "dW3", "dW2")
+TOL_FRO = 1e-2   # relative Frobenius error of each gradient tensor
+TOL_MAX = 2e-2   # max error over each tensor (each expert's block) / its largest entry
+
+
+def _check_backward(w, seed=7, grad_bf16=False):
+    """Every gradient against the fp64 oracle, element by element.
+
+    The device keeps the forward's g and u, the output gradient w dy, dG and
+    dU, and H in bf16 (each a rounding of at most 2^-9 relative), and sums in
+    fp32: every gradient is then a sum of products carrying a relative error of
+    a few 2^-9, about 0.3% in norm.  The bound is norm-wise, not the forward
+    output's max-over-rms rule: an expert's weight gradient is a sum of outer
+    products over its few rows, whose largest entries are 15-20x its rms, so
+    a max-over-rms measure scales with that spread rather than with the
+    arithmetic.  Per tensor: ||err||_F <= 1e-2 ||ref||_F; per tensor (per
+    expert for the routed weight gradients): max|err| <= 2e-2 max|ref|; an
+    expert no token chose has an exactly zero gradient."""
+    from gpu_util import route_with_exemptions
+    cfg = w.cfg
+    dy = torch.randn(cfg.T, cfg.d, generator=torch.Generator(device="cuda").manual_seed(seed), device="cuda")
+    g, ws = _backward(w, dy, grad_bf16)
+    # the device's routing (for near-tie tokens the oracle follows it)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    y = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+    fws = B.alloc_workspace(B.shape_of(cfg))
+    B.forward(B.shape_of(cfg), w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, None, None, None, w.W1s, w.W3s, w.W2s, y, fws,
+              topk_idx=idx)
+    lg = obw._logits(dec(w.x), dec(w.Wg))
+    _, _, merged, report, n_near = route_with_exemptions(w, lg, to_np(idx))
+    assert len(report) <= n_near, report
+    ref = _oracle_backward(w, dy, force_idx=merged if report else None)
+    stats = {}
+    for name in GRADS:
+        if name not in g:
+            continue
+        d = to_np(g[name].float()).astype(np.float64)
+        o = ref[name]
+        assert np.isfinite(d).all(), f"{name}: not every element written"
+        fro = float(np.linalg.norm(d - o) / np.linalg.norm(o))
+        blocks = [(d[e], o[e]) for e in range(d.shape[0])] if name in PER_EXPERT else [(d, o)]
+        worst = 0.0
+        for db, ob in blocks:
+            m = float(np.abs(ob).max())
+            if m == 0.0:
+                assert not db.any(), f"{name}: an expert without rows has a nonzero gradient"
+                continue
+            worst = max(worst, float(np.abs(db - ob).max()) / m)
+        stats[name] = (fro, worst)
+    print({k: f"fro {a:.1e} max {b:.1e}" for k, (a, b) in stats.items()})
+    for name, (fro, worst) in stats.items():
+        assert fro <= TOL_FRO and worst <= TOL_MAX, (name, fro, worst)
+    return g, ref
+
+
+def _medium(**kw):
+    shape = dict(T=1000, d=1024, E=64, k=6, inter=512, shared_inter=384)
+    shape.update(kw)
+    return to_device(workloads.make_small("prefill", **shape))
+
+
+def test_backward_tiny():
+    _check_backward(to_device(workloads.make("tiny")))
+
+
+def test_backward_medium_ragged():
+    # I != Is, a partial 256-column block of the shared expert, ragged segments
+    _check_backward(_medium())
+
+
+def test_backward_no_shared_expert():
+    # the shared expert's tiles then carry only the router's dl Wg part of dx
+    _check_backward(_medium(T=300, shared_inter=0))
+
+
+def test_backward_group_routing():
+    w = to_device(workloads.make_small("fp8", T=600, d=1024, E=64, k=8, inter=256, shared_inter=256, n_group=8,
+                                       topk_group=4, fp8=False))
+    _check_backward(w)
+
+
+def test_backward_empty_and_oversize_segments():
+    # a shared direction in x and gate rows aligned with it: expert 0 takes
+    # nearly every token (a segment of several 256-row tiles), experts 1-3 most
+    # second slots, and most other experts receive no row (zero weight gradient)
+    w = workloads.make_small("prefill", T=700, d=512, E=64, k=2, inter=256, shared_inter=256)
+    gen = torch.Generator().manual_seed(3)
+    u = torch.randn(w.cfg.d, generator=gen)
+    u = u / u.norm()
+    x = w.x.float() + 3.0 * u
+    x = x / x.pow(2).mean(dim=1, keepdim=True).sqrt()
+    Wg = w.Wg.float()
+    Wg[0] += 6.0 * u
+    Wg[1:4] += 2.5 * u
+    Wg[4:] -= 2.0 * u
+    w.x, w.Wg = x.to(torch.bfloat16), Wg.to(torch.bfloat16)
+    w = to_device(w)
+    g, ref = _check_backward(w)
+    c = np.bincount(ref["idx"].ravel(), minlength=w.cfg.E)
+    assert c[0] > 512 and (c == 0).sum() >= 40, c      # several 256-row tiles; most experts empty
+    empty = np.nonzero(c == 0)[0]
+    assert not to_np(g["dW1"][torch.as_tensor(empty, device="cuda")]).any()
+    assert not to_np(g["dW2"][torch.as_tensor(empty, device="cuda")]).any()
+
+
+def test_backward_bf16_gradients_and_determinism():
+    w = to_device(workloads.make("tiny"))
+    g32, _ = _check_backward(w)
+    dy = torch.randn(w.cfg.T, w.cfg.d, generator=torch.Generator(device="cuda").manual_seed(7), device="cuda")
+    a, _ = _backward(w, dy)
+    b, _ = _backward(w, dy)
+    for name in a:
+        assert torch.equal(a[name], b[name]), name        # bit-identical repeat
+        assert torch.equal(a[name], g32[name]), name
+    h, _ = _backward(w, dy, grad_bf16=True)
+    for name in h:
+        # the bf16 gradients are the fp32 ones rounded once
+        assert torch.equal(h[name], g32[name].to(torch.bfloat16)), name
