@@ -607,7 +607,7 @@ def run_ours(args, dist):
         line["e2e"] = e2e
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = run_cpu_baseline(args, w, cfg)
-    if args.workload == "prefill" and not (args.tokens or args.experts or args.no_backward):
+    if args.workload == "prefill" and not args.no_backward:
         fwd_args = None
         line["backward"] = backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src)
         torch.cuda.empty_cache()

@@ -222,6 +222,39 @@ moe_status moe_combine_backward(const moe_shape* shape, const float* dy, const v
 moe_status moe_router_backward(const moe_shape* shape, const float* logits, const int32_t* topk_idx,
                                const float* topk_w, const float* dw, float* dlogits, void* stream);
 
+/* The shared expert alone (atlas page, "Code" section, MoE forward block:
+ * y += shared_experts(x)): Y_shared[t] = (bf16(silu(x[t] W1s) * (x[t] W3s)))
+ * W2s in fp32 for the T tokens of x, with the grouped-GEMM kernels of
+ * moe_grouped_swiglu.  Used by the all-to-all flavour of expert parallelism,
+ * where each rank's routed rows run on other ranks and its shared expert on
+ * its own tokens.  shape->shared_inter must be > 0; x [T, d] bf16; W1s, W3s
+ * [d, shared_inter], W2s [shared_inter, d] bf16; Y_shared [T, d] fp32 out;
+ * ws as for moe_forward (moe_workspace_size bytes). */
+moe_status moe_shared_expert(const moe_shape* shape, const void* x, const void* W1s, const void* W3s,
+                             const void* W2s, float* Y_shared, void* ws, size_t ws_bytes, void* stream);
+
+/* All-to-all expert parallelism, the receiving side's regrouping (n4n page,
+ * "Why 256 experts with top-8 routing?": hidden states travel to the devices
+ * that hold their experts).  A rank holding E_local experts receives from each
+ * of n_src source ranks, in source order, that source's rows for its experts
+ * in expert order; recv_counts [n_src, E_local] int32 (device) gives how many
+ * rows each source sends for each local expert.  Writes, for the R =
+ * sum(recv_counts) received rows:
+ *   offsets_local [E_local + 1]: expert-major segment starts (R at the end),
+ *   to_expert_major [R]: the received (source-major) row at expert-major
+ *                        position p,
+ *   to_source_major [R]: the expert-major position of received row r
+ * (expert-major order: experts ascending, then sources, then each source's
+ * order), so that moe_gather_rows through them moves rows either way.
+ * n_src * E_local <= 1024. */
+moe_status moe_ep_regroup_layout(int n_src, int E_local, const int32_t* recv_counts, int32_t* offsets_local,
+                                 int32_t* to_expert_major, int32_t* to_source_major, void* stream);
+
+/* Row gather: dst[r] = src[index[r]] for r < rows, rows of d bf16 (d a
+ * multiple of 8), 16-byte aligned device buffers.  Indices must address rows
+ * of src (not checked). */
+moe_status moe_gather_rows(const void* src, const int32_t* index, int64_t rows, int d, void* dst, void* stream);
+
 /* Gradient of the whole layer (training): for the loss sum(dy * y) with
  * y = moe_forward(...), the gradients with respect to x, Wg, W1, W3, W2 and
  * the shared expert's weights, the expert selection held fixed (it is

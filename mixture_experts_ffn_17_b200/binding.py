@@ -25,7 +25,7 @@ EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped
             "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version",
             "moe_permute_noalloc", "moe_router_topk_limited", "moe_expert_utilisation", "moe_forward_ep",
             "moe_forward_launches", "moe_combine_backward", "moe_router_backward", "moe_backward_workspace_size",
-            "moe_backward")
+            "moe_backward", "moe_shared_expert", "moe_ep_regroup_layout", "moe_gather_rows")
 NUM_STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "experts_up", "experts_down", "combine")
 
@@ -86,13 +86,17 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_ep.argtypes = [S, I, I, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.moe_forward_launches.argtypes = [S]
         L.moe_forward_launches.restype = ctypes.c_int
+        L.moe_shared_expert.argtypes = [S, P, P, P, P, P, P, sz, P]
+        L.moe_ep_regroup_layout.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P, P, P]
+        L.moe_gather_rows.argtypes = [P, P, ctypes.c_int64, ctypes.c_int, P, P]
         L.moe_backward_workspace_size.argtypes = [S]
         L.moe_backward_workspace_size.restype = sz
         L.moe_backward.argtypes = [S] + [P] * 18 + [P, sz, P]
         L.moe_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         for fn in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_combine_backward",
                    "moe_router_backward", "moe_forward",
-                   "moe_forward_profiled", "moe_forward_ep", "moe_backward", "moe_check_device_status"):
+                   "moe_forward_profiled", "moe_forward_ep", "moe_backward", "moe_shared_expert", "moe_ep_regroup_layout", "moe_gather_rows",
+                   "moe_check_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -227,6 +231,28 @@ def forward_profiled(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, 
                                       _ptr(y), _ptr(topk_idx), _ptr(topk_w), _ptr(counts), _ptr(ws),
                                       ws.numel() if ws is not None else 0, _stream(stream), handles),
            "moe_forward_profiled")
+
+
+def shared_expert(shape, x, W1s, W3s, W2s, Y_shared, ws, stream=None):
+    """The shared expert alone (moe_shared_expert): Y_shared [T, d] fp32."""
+    _check(lib().moe_shared_expert(ctypes.byref(shape), _ptr(x), _ptr(W1s), _ptr(W3s), _ptr(W2s), _ptr(Y_shared),
+                                   _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)), "moe_shared_expert")
+
+
+def ep_regroup_layout(n_src, E_local, recv_counts, offsets_local, to_expert_major, to_source_major, stream=None):
+    """Expert-major order of rows received from n_src ranks (moe_ep_regroup_layout)."""
+    _check(lib().moe_ep_regroup_layout(int(n_src), int(E_local), _ptr(recv_counts), _ptr(offsets_local),
+                                       _ptr(to_expert_major), _ptr(to_source_major), _stream(stream)),
+           "moe_ep_regroup_layout")
+
+
+def gather_rows(src, index, dst, stream=None):
+    """dst[r] = src[index[r]] for every row of dst (moe_gather_rows, bf16 rows)."""
+    rows = int(dst.shape[0])
+    if rows == 0:
+        return
+    _check(lib().moe_gather_rows(_ptr(src), _ptr(index), rows, int(dst.shape[1]), _ptr(dst), _stream(stream)),
+           "moe_gather_rows")
 
 
 def backward_workspace_size(shape: MoeShape) -> int:

@@ -18,7 +18,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
 
 SOURCES = ["moe_api.cu", "router.cu", "permute.cu", "grouped_gemm.cu", "combine.cu", "monitor.cu", "backward.cu",
-           "grouped_gemm_bwd.cu"]
+           "grouped_gemm_bwd.cu", "ep.cu"]
 HEADERS = ["ptx.cuh", "common.cuh", "moe_internal.h", "backward.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -435,6 +435,56 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   return MOE_OK;
 }
 
+// The shared expert alone over the T tokens of x (no routed rows): the tile
+// list holds only its tiles, and both grouped GEMMs walk them.
+moe_status run_shared_only(const moe_shape& s, const Layout& L, void* ws, const void* x, const void* W1s,
+                           const void* W3s, const void* W2s, float* Y_shared, uint32_t* status, cudaStream_t st) {
+  int4* tiles = at<int4>(ws, L.tiles);
+  int32_t* ntiles = at<int32_t>(ws, L.ntiles);
+  int* sched = at<int>(ws, L.sched);
+  uint16_t* H = at<uint16_t>(ws, L.H);
+  const int64_t Tk = s.T * s.k;
+  MOE_CUDA(launch_build_tiles(at<int32_t>(ws, L.offsets), s.E, s.T, Shard{0, 0}, true, tiles, ntiles, sched, st,
+                              nullptr));
+  const int sms = num_sms();
+  CUtensorMap a_s, w1_s, w3_s, h_map, w2_s;
+  if (!map_2d(&a_s, x, s.d, s.T, kGemmBK, kTileM) || !map_3d(&w1_s, W1s, s.shared_inter, s.d, 1, kGemmBK) ||
+      !map_3d(&w3_s, W3s, s.shared_inter, s.d, 1, kGemmBK) || !map_2d(&h_map, H, L.Hld, L.Hrows, kGemmBK, kTileM) ||
+      !map_3d(&w2_s, W2s, s.d, s.shared_inter, 1, kGemmBK))
+    return MOE_ERR_CUDA;
+  GemmParams p1{};
+  p1.tiles = tiles;
+  p1.ntiles = ntiles;
+  p1.max_mtiles = L.max_mtiles;
+  p1.tile_set = kTilesShared;
+  p1.E = s.E;
+  p1.n_nb = (L.Hld + gemm_block_n_swiglu() - 1) / gemm_block_n_swiglu();
+  p1.K_routed = p1.K_shared = s.d;
+  p1.N_routed = 0;
+  p1.N_shared = s.shared_inter;
+  p1.out_routed = p1.out_shared = H;
+  p1.out_shared_row_offset = Tk;
+  p1.ld_out = L.Hld;
+  p1.status = status;
+  p1.sched_counter = sched + 1;
+  MOE_CUDA(launch_grouped_swiglu(a_s, a_s, w1_s, w1_s, w3_s, w3_s, p1,
+                                 (int)std::min<int64_t>(sms, (int64_t)L.max_mtiles * p1.n_nb), st));
+  GemmParams p2 = p1;
+  p2.sched_counter = sched + 3;
+  p2.n_nb = (s.d + gemm_block_n_down() - 1) / gemm_block_n_down();
+  p2.K_routed = p2.K_shared = s.shared_inter;
+  p2.N_routed = 0;
+  p2.N_shared = s.d;
+  p2.a_shared_row_offset = (int)Tk;
+  p2.out_routed = nullptr;
+  p2.out_shared = Y_shared;
+  p2.out_shared_row_offset = 0;
+  p2.ld_out = s.d;
+  MOE_CUDA(launch_grouped_down(h_map, w2_s, w2_s, p2, (int)std::min<int64_t>(sms, (int64_t)L.max_mtiles * p2.n_nb),
+                               st));
+  return MOE_OK;
+}
+
 // ------------------------------------------------------------ backward pass
 // Workspace of moe_backward: the forward's layout (routing, dispatch, x_perm,
 // H, Y_perm) and the backward's own buffers after it.
@@ -946,6 +996,45 @@ moe_status moe_forward_ep(const moe_shape* shape, int ep_rank, int ep_size, cons
                           void* stream) {
   return forward_impl(shape, x, Wg, bias, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, y, topk_idx_out, topk_w_out,
                       counts_out, ws, ws_bytes, stream, nullptr, ep_rank, ep_size);
+}
+
+moe_status moe_shared_expert(const moe_shape* shape, const void* x, const void* W1s, const void* W3s,
+                             const void* W2s, float* Y_shared, void* ws, size_t ws_bytes, void* stream) {
+  moe_status v = validate_shape(shape);
+  if (v != MOE_OK) return v;
+  const moe_shape& s = *shape;
+  if (s.shared_inter <= 0) return MOE_ERR_INVALID_ARG;
+  if (!x || !W1s || !W3s || !W2s || !Y_shared) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, W1s, W3s, W2s, Y_shared};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(s);
+  if (!ws_ok(ws, ws_bytes, L.total)) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
+  if (s.T == 0) return MOE_OK;
+  return run_shared_only(s, L, ws, x, W1s, W3s, W2s, Y_shared, status, st);
+}
+
+moe_status moe_ep_regroup_layout(int n_src, int E_local, const int32_t* recv_counts, int32_t* offsets_local,
+                                 int32_t* to_expert_major, int32_t* to_source_major, void* stream) {
+  if (n_src < 1 || E_local < 1 || (int64_t)n_src * E_local > 1024) return MOE_ERR_INVALID_ARG;
+  if (!recv_counts || !offsets_local || !to_expert_major || !to_source_major) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(recv_counts) || !aligned16(offsets_local) || !aligned16(to_expert_major) ||
+      !aligned16(to_source_major))
+    return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(launch_ep_regroup(recv_counts, n_src, E_local, offsets_local, to_expert_major, to_source_major,
+                             static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_gather_rows(const void* src, const int32_t* index, int64_t rows, int d, void* dst, void* stream) {
+  if (rows < 0 || d <= 0 || d % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!src || !index || !dst || !aligned16(src) || !aligned16(index) || !aligned16(dst)) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(launch_gather_rows(src, index, rows, d, dst, num_sms(), static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
 }
 
 size_t moe_backward_workspace_size(const moe_shape* shape) {

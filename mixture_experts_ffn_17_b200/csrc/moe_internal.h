@@ -158,6 +158,11 @@ cudaError_t launch_grouped_swiglu_fp8(const CUtensorMap& tmA_r, const CUtensorMa
 cudaError_t launch_grouped_down_fp8(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const GemmParams& p, int grid,
                                     cudaStream_t stream);
 
+// ep.cu: expert-major order of rows received from n_src ranks (source-major,
+// each source's rows in expert order); n_src * E_local <= 1024.
+cudaError_t launch_ep_regroup(const int32_t* recv_counts, int n_src, int E_local, int32_t* offsets_local,
+                              int32_t* to_expert_major, int32_t* to_source_major, cudaStream_t stream);
+
 // combine.cu
 // offsets != nullptr: only permuted rows of experts [shard.e_lo, shard.e_hi)
 // are added.  topk_w == nullptr: every row has weight 1.

@@ -87,3 +87,195 @@ def forward(shape, rank: int, world: int, x, Wg, bias, w: EpWeights, y, ws, grou
     B.forward_ep(shape, rank, world, x, Wg, bias, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s, y, ws,
                  topk_idx=topk_idx, topk_w=topk_w, counts=counts, stream=stream)
     return all_reduce_partial(y, group)
+
+
+# --------------------------------------------------------------------------
+# All-to-all flavour.
+#
+# Here every rank holds its own batch of tokens and E/world routed experts;
+# the shared expert is replicated and runs on each rank's own tokens.  A
+# token's hidden state travels to the ranks that hold its selected experts
+# and the expert outputs travel back (n4n.ai page, "Why 256 experts with top-8
+# routing?", device-limited routing and the all-to-all it bounds; "Training
+# infrastructure that made this possible": that all-to-all overlapped with
+# computation).  Per rank:
+#   1. route its tokens over all E experts and permute them (moe_router_topk,
+#      moe_permute): the rows for rank q's experts form one contiguous block of
+#      the expert-major x_perm;
+#   2. exchange the per-expert row counts, then the rows (all-to-all);
+#   3. regroup the received rows expert-major (moe_ep_regroup_layout,
+#      moe_gather_rows), run the local experts (moe_grouped_swiglu), and put
+#      the outputs back in the received order;
+#   4. send them back (all-to-all); they arrive in the rank's own x_perm order,
+#      i.e. as its Y_perm;
+#   5. the shared expert on its own tokens (moe_shared_expert) and the combine
+#      (moe_combine) give the rank's y.
+# With several token chunks, chunk c+1's rows travel while chunk c's experts
+# compute, and chunk c's outputs travel back while chunk c+1's compute.
+# Every arithmetic step runs in the library's kernels; this module moves
+# tensors between ranks.
+# --------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class A2AWeights:
+    """One rank's weights in the all-to-all flavour: routed experts
+    [e_lo, e_hi) and the whole shared expert (replicated)."""
+    W1: torch.Tensor
+    W3: torch.Tensor
+    W2: torch.Tensor
+    W1s: Optional[torch.Tensor]
+    W3s: Optional[torch.Tensor]
+    W2s: Optional[torch.Tensor]
+
+
+def shard_weights_a2a(W1, W3, W2, W1s, W3s, W2s, rank: int, world: int) -> A2AWeights:
+    E = W1.shape[0]
+    if E % world or (E // world) % 32:
+        raise ValueError(f"E={E} over {world} ranks: each rank's expert count must be a multiple of 32")
+    lo, hi = rank * (E // world), (rank + 1) * (E // world)
+    return A2AWeights(W1[lo:hi].contiguous(), W3[lo:hi].contiguous(), W2[lo:hi].contiguous(), W1s, W3s, W2s)
+
+
+class A2ARank:
+    """One rank's steps of the all-to-all layer for one batch of its tokens.
+    `shape` is the whole layer's shape for this batch (T = the rank's tokens,
+    E = all experts)."""
+
+    def __init__(self, shape, rank: int, world: int, w: A2AWeights, device, stream=None):
+        self.shape, self.rank, self.world, self.w = shape, rank, world, w
+        self.stream = stream
+        T, d, E, k = shape.T, shape.d, shape.E, shape.k
+        self.El = E // world
+        dev = device
+        self.ws = B.alloc_workspace(shape, dev)
+        self.idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.tw = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(E, dtype=torch.int32, device=dev)
+        self.offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        self.perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+        self.row_of = torch.empty(T * k, dtype=torch.int32, device=dev)
+        self.x_perm = torch.empty(T * k, d, dtype=torch.bfloat16, device=dev)
+        self.Y_shared = (torch.empty(T, d, dtype=torch.float32, device=dev) if shape.shared_inter > 0 else None)
+
+    # step 1
+    def dispatch(self, x, Wg, bias) -> torch.Tensor:
+        """Route and permute; returns the send counts [world, E_local] (device)."""
+        s = self.shape
+        B.router_topk(s, x, Wg, bias, self.idx, self.tw, None, self.ws, stream=self.stream)
+        B.permute(s, self.idx, self.counts, self.offsets, self.perm, self.row_of, x, self.x_perm, self.ws,
+                  stream=self.stream)
+        return self.counts.view(self.world, self.El)
+
+    # step 3
+    def compute(self, x_recv: torch.Tensor, recv_counts: torch.Tensor) -> torch.Tensor:
+        """Rows received from every rank (source-major) and their counts
+        [world, E_local] -> this rank's expert outputs in the same order."""
+        s = self.shape
+        R = int(x_recv.shape[0])
+        dev = x_recv.device
+        y_send = torch.empty(R, s.d, dtype=torch.bfloat16, device=dev)
+        if R == 0:
+            return y_send
+        offs = torch.empty(self.El + 1, dtype=torch.int32, device=dev)
+        to_em = torch.empty(R, dtype=torch.int32, device=dev)
+        to_sm = torch.empty(R, dtype=torch.int32, device=dev)
+        B.ep_regroup_layout(self.world, self.El, recv_counts.contiguous(), offs, to_em, to_sm, stream=self.stream)
+        x_loc = torch.empty(R, s.d, dtype=torch.bfloat16, device=dev)
+        B.gather_rows(x_recv, to_em, x_loc, stream=self.stream)
+        shape_loc = B.make_shape(T=R, d=s.d, E=self.El, k=1, inter=s.inter, shared_inter=0)
+        ws_loc = B.alloc_workspace(shape_loc, dev)
+        Y_loc = torch.empty(R, s.d, dtype=torch.bfloat16, device=dev)
+        B.grouped_swiglu(shape_loc, x_loc, x_loc, offs, self.w.W1, self.w.W3, self.w.W2, None, None, None, None, None,
+                         None, Y_loc, None, ws_loc, stream=self.stream)
+        B.gather_rows(Y_loc, to_sm, y_send, stream=self.stream)
+        return y_send
+
+    # step 5
+    def combine(self, x, Y_perm: torch.Tensor, y: torch.Tensor):
+        s = self.shape
+        if self.Y_shared is not None:
+            B.shared_expert(s, x, self.w.W1s, self.w.W3s, self.w.W2s, self.Y_shared, self.ws, stream=self.stream)
+        B.combine(s, Y_perm, self.Y_shared, self.row_of, self.tw, y, stream=self.stream)
+        return y
+
+
+def _splits(counts_2d: torch.Tensor):
+    return [int(v) for v in counts_2d.sum(dim=1).tolist()]
+
+
+class ProcessGroupTransport:
+    """all_to_all_single over a torch.distributed group (NCCL on GPUs, gloo on
+    CPU).  Rows are dim 0; split sizes are host lists."""
+
+    def __init__(self, group=None):
+        self.group = group
+
+    def all_to_all(self, send: torch.Tensor, send_splits, recv_splits, async_op: bool = False):
+        import torch.distributed as dist
+        out = send.new_empty((sum(recv_splits),) + tuple(send.shape[1:]))
+        work = dist.all_to_all_single(out, send.contiguous(), list(recv_splits), list(send_splits), group=self.group,
+                                      async_op=async_op)
+        return out, work
+
+    def exchange_counts(self, send_counts: torch.Tensor) -> torch.Tensor:
+        """send_counts [world, E_local]: row q is what this rank sends to rank
+        q; returns [world, E_local], row s is what rank s sends here."""
+        n = send_counts.shape[0]
+        out, _ = self.all_to_all(send_counts.contiguous(), [1] * n, [1] * n)
+        return out
+
+
+def forward_all_to_all(shape, rank: int, world: int, x, Wg, bias, w: A2AWeights, y, transport=None, chunks: int = 2,
+                       stream=None) -> torch.Tensor:
+    """This rank's y (its own tokens) through the all-to-all layer, with the
+    tokens split into `chunks` batches whose exchanges overlap the other
+    batches' expert GEMMs.  Every rank of the group calls it with the same
+    `chunks` (the collectives run in the same order everywhere)."""
+    transport = transport or ProcessGroupTransport()
+    T = shape.T
+    bounds = [T * c // chunks for c in range(chunks + 1)]
+    parts = []
+    for c in range(chunks):
+        sl = slice(bounds[c], bounds[c + 1])
+        sh = B.make_shape(T=bounds[c + 1] - bounds[c], d=shape.d, E=shape.E, k=shape.k, inter=shape.inter,
+                          shared_inter=shape.shared_inter, route=shape.route, n_group=shape.n_group,
+                          topk_group=shape.topk_group, group_topn=shape.group_topn, route_scale=shape.route_scale,
+                          y_dtype=shape.y_dtype)
+        parts.append((sl, A2ARank(sh, rank, world, w, x.device, stream)))
+    sends, recvs, xs = [], [], []
+    for sl, st in parts:
+        sends.append(st.dispatch(x[sl], Wg, bias))
+    for c, (sl, st) in enumerate(parts):
+        recvs.append(transport.exchange_counts(sends[c]))
+    for c, (sl, st) in enumerate(parts):
+        xs.append(transport.all_to_all(st.x_perm, _splits(sends[c]), _splits(recvs[c]), async_op=True))
+    rets = []
+    for c, (sl, st) in enumerate(parts):
+        x_recv, work = xs[c]
+        if work is not None:
+            work.wait()
+        y_send = st.compute(x_recv, recvs[c])
+        rets.append(transport.all_to_all(y_send, _splits(recvs[c]), _splits(sends[c]), async_op=True))
+    for c, (sl, st) in enumerate(parts):
+        Y_perm, work = rets[c]
+        if work is not None:
+            work.wait()
+        st.combine(x[sl], Y_perm, y[sl])
+    return y
+
+
+def simulate_all_to_all(shape, xs, Wg, bias, weights, ys, stream=None):
+    """All ranks of the all-to-all layer in one process (one GPU), the
+    exchanges done by slicing: rank r's tokens xs[r] and weights weights[r]
+    -> ys[r].  The same per-rank steps as forward_all_to_all, in lock step."""
+    world = len(xs)
+    states = [A2ARank(shape, r, world, weights[r], xs[r].device, stream) for r in range(world)]
+    send = [st.dispatch(xs[r], Wg, bias) for r, st in enumerate(states)]
+    recv = [torch.stack([send[s][r] for s in range(world)]) for r in range(world)]
+    blocks = [list(torch.split(states[s].x_perm, _splits(send[s]))) for s in range(world)]
+    x_recv = [torch.cat([blocks[s][r] for s in range(world)]) for r in range(world)]
+    y_send = [st.compute(x_recv[r], recv[r]) for r, st in enumerate(states)]
+    back = [list(torch.split(y_send[r], _splits(recv[r]))) for r in range(world)]
+    for r, st in enumerate(states):
+        st.combine(xs[r], torch.cat([back[q][r] for q in range(world)]), ys[r])
+    return ys

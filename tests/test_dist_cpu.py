@@ -134,3 +134,41 @@ def test_ep_slice_rejects_uneven_splits():
     with pytest.raises(ValueError):
         ep.ep_slice(256, 2048, 2, 2)
     assert ep.ep_slice(256, 2048, 7, 8) == ep.EpSlice(224, 256, 1792, 2048)
+
+
+def test_all_to_all_exchange_plumbing_gloo():
+    # the all-to-all flavour's transport with host tensors, world size 2: the
+    # per-expert counts, then variable-sized row blocks each way and back
+    outs = _run_ranks("""
+        import torch, torch.distributed as dist
+        import bench
+        from mixture_experts_ffn_17_b200 import expert_parallel as ep
+        d = bench.Dist(backend="gloo", timeout_s=60)
+        r, n, El = d.rank, d.world, 3
+        g = torch.Generator().manual_seed(10 + r)
+        counts = torch.randint(0, 4, (n, El), generator=g, dtype=torch.int32)   # rows this rank sends q, per expert
+        rows = int(counts.sum())
+        # row i of the send buffer encodes (source rank, i)
+        send = torch.stack([torch.full((5,), 1000.0 * r + i) for i in range(rows)]) if rows else torch.zeros(0, 5)
+        tr = ep.ProcessGroupTransport()
+        recv_counts = tr.exchange_counts(counts)
+        all_counts = [torch.zeros_like(counts) for _ in range(n)]
+        dist.all_gather(all_counts, counts)
+        assert torch.equal(recv_counts, torch.stack([all_counts[s][r] for s in range(n)]))
+        ss, rs = ep._splits(counts), ep._splits(recv_counts)
+        got, _ = tr.all_to_all(send, ss, rs)
+        # block s of what arrives is source s's block for this rank, in its order
+        at = 0
+        for s in range(n):
+            first = int(all_counts[s][:r].sum())
+            for j in range(rs[s]):
+                assert float(got[at + j, 0]) == 1000.0 * s + first + j
+            at += rs[s]
+        back, _ = tr.all_to_all(got, rs, ss)
+        assert torch.equal(back, send)
+        print("RESULT", r, rows, int(recv_counts.sum()))
+        d.close()
+    """)
+    for rc, o, e in outs:
+        assert rc == 0, e
+    assert sum(1 for _, o, _ in outs for l in o.splitlines() if l.startswith("RESULT")) == 2
