@@ -98,8 +98,16 @@ struct WgradParams {
   uint32_t* status;
 };
 
+// bf16 outputs (out_bf16): 3D bf16 maps [groups, M, ncols] with [1 x 128 x 64]
+// boxes, 128-byte swizzle, of out1, out2 (routed) and out1_shared,
+// out2_shared (groups = 1); the pointers in WgradParams then go unused.
+struct WgradOutMaps {
+  CUtensorMap m[4];
+};
+
 cudaError_t launch_wgrad(int mode, const CUtensorMap& tmA_r, const CUtensorMap& tmA_s, const CUtensorMap& tmB_r,
-                         const CUtensorMap& tmB_s, const WgradParams& p, int grid, cudaStream_t stream);
+                         const CUtensorMap& tmB_s, const WgradOutMaps& om, const WgradParams& p, int grid,
+                         cudaStream_t stream);
 
 // bf16 copy of a row-major fp32 [rows, cols] matrix into rows of ld_out
 // elements, the columns past cols zeroed.

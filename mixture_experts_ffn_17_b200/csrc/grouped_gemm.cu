@@ -987,6 +987,16 @@ constexpr int kPairF8Stages = MOE_PAIR_F8_STAGES;
 constexpr uint32_t kPairF8RawBytes = 64 * 128;                         // one raw box
 constexpr uint32_t kPairF8StageBytes = kPairABytes + kPairF8RawBytes;  // 24 KB
 constexpr int kPairF8ConvStages = MOE_PAIR_F8_CONV_STAGES;
+// Converted buffer c = K step % kPairF8ConvStages is free once the MMA that
+// read it kPairF8ConvStages steps earlier has completed.  With both rings of
+// one depth that MMA's commit to the stage's `empty` barrier is what lets the
+// producer reload stage s, and the converters start on step kg only after its
+// raw codes landed in stage s, i.e. after that commit: the separate `cempty`
+// hand-off is then redundant.
+#ifndef MOE_PAIR_F8_ONE_COMMIT
+#define MOE_PAIR_F8_ONE_COMMIT 1
+#endif
+constexpr bool kPairF8OneCommit = MOE_PAIR_F8_ONE_COMMIT && kPairF8ConvStages == kPairF8Stages;
 constexpr uint32_t kPairF8ConvBytes = 2 * kF8BoxBytes;  // 16 KB: two bf16 [64 K x 64 N] boxes
 constexpr int kPairF8EpiWarps = 4;
 constexpr int kPairF8Threads = 64 + 32 * kPairF8EpiWarps + 32 * kConvWarps;
@@ -1129,7 +1139,10 @@ __global__ void __launch_bounds__(kPairF8Threads, 1)
             ptx::mma_bf16_pair(tmem + sl * kSlotCols, ptx::sdesc_sw128(a0 + kk * 32, 16, 1024),
                                ptx::sdesc_sw128(b0 + kk * 2048, kF8BoxBytes, 1024), idesc, (kb | kk) != 0 ? 1u : 0u);
           ptx::mma_commit_pair(&empty[s], 0x3);
-          ptx::mma_commit_pair(&cempty[c], 0x3);
+          // with rings of one depth, converted buffer c is stage s: the
+          // converters' wait for the stage's raw codes already orders them
+          // after this commit, so no second commit is needed
+          if (!kPairF8OneCommit) ptx::mma_commit_pair(&cempty[c], 0x3);
         }
         if (!ok) break;
         ptx::mma_commit_pair(&tfull[sl], 0x3);
@@ -1218,7 +1231,7 @@ __global__ void __launch_bounds__(kPairF8Threads, 1)
         const int s = kg % S;
         const int c = kg % CS;
         if (!ptx::wait_bounded(&rfull[s], (kg / S) & 1, abort_flag) ||
-            !ptx::wait_bounded(&cempty[c], ((kg / CS) & 1) ^ 1, abort_flag)) {
+            (!kPairF8OneCommit && !ptx::wait_bounded(&cempty[c], ((kg / CS) & 1) ^ 1, abort_flag))) {
           raise_status(p.status, abort_flag, kStatusTimeout);
           ok = false;
           break;

@@ -30,7 +30,9 @@
 // MN-major ([64 rows x 64 features] boxes of the row-major activations).  The
 // last K step of a group usually holds rows of the next expert: warp 1 zeroes
 // those rows of both operands in shared memory before the MMA reads them.  A
-// group without rows writes zeros.  Each output element is produced by one
+// group without rows writes zeros.  bf16 gradients leave through shared
+// memory in TMA stores (a lane holds one output row, so direct stores would
+// touch 32 lines per warp instruction); fp32 gradients are stored directly.  Each output element is produced by one
 // CTA, in a fixed order: the results are deterministic, with no atomics.
 #include <algorithm>
 #include <cstdint>
@@ -335,12 +337,16 @@ __global__ void __launch_bounds__(kThreads, 1) dgrad_kernel(const __grid_constan
 }
 
 // ------------------------------------------------------------------ wgrad
-constexpr int kWgStages = 4;
+constexpr int kWgStages = 3;
 constexpr uint32_t kWgBox = 64 * 64 * 2;            // [64 K rows x 64 features] bf16, 8 KB
 constexpr uint32_t kWgABytes = 2 * kWgBox;          // 128 output rows
 constexpr uint32_t kWgBBytes = 4 * kWgBox;          // 256 output columns
 constexpr uint32_t kWgStageBytes = kWgABytes + kWgBBytes;
-constexpr size_t wgrad_smem_bytes() { return 1024 + kWgStages * kWgStageBytes + 256; }
+// bf16 output tile staged for the TMA stores: four [128 rows x 64 columns]
+// boxes, 128-byte swizzled like the output tensor maps
+constexpr uint32_t kWgOutBox = 128 * 64 * 2;
+constexpr uint32_t kWgOutBytes = 4 * kWgOutBox;
+constexpr size_t wgrad_smem_bytes() { return 1024 + kWgStages * kWgStageBytes + kWgOutBytes + 256; }
 static_assert(wgrad_smem_bytes() <= 232448, "shared memory budget (wgrad)");
 
 struct WgTile {
@@ -378,11 +384,13 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
                                                             const __grid_constant__ CUtensorMap tmA_s,
                                                             const __grid_constant__ CUtensorMap tmB_r,
                                                             const __grid_constant__ CUtensorMap tmB_s,
+                                                            const __grid_constant__ WgradOutMaps om,
                                                             const WgradParams p) {
   constexpr int S = kWgStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stage0 = align_1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(stage0 + S * kWgStageBytes);
+  uint8_t* stg = stage0 + S * kWgStageBytes;  // staged bf16 output tile
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg + kWgOutBytes);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
@@ -539,8 +547,15 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
       WgTile t;
       wg_tile_at(p, tile, t);
       const int sl = tl & 1;
-      if (!ptx::wait_bounded(&tfull[sl], use[sl] & 1, abort_flag)) {
-        raise_status(p.status, abort_flag, kStatusTimeout);
+      const bool got = ptx::wait_bounded(&tfull[sl], use[sl] & 1, abort_flag);
+      if (!got) raise_status(p.status, abort_flag, kStatusTimeout);
+      if (p.out_bf16) {
+        // the epilogue warps meet on a named barrier below, so they leave the
+        // loop together or not at all; this barrier is also where the
+        // previous tile's TMA stores are known to have read the staging buffer
+        if (threadIdx.x == 64) ptx::bulk_wait_read_all();
+        if (!ptx::named_barrier_and(1, 32 * kEpiWarps, got)) break;
+      } else if (!got) {
         break;
       }
       ptx::tc_fence_after();
@@ -564,6 +579,47 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
       ptx::mbar_arrive(&tempty[sl]);
       ++use[sl];
       ++tl;
+      if (p.out_bf16) {
+        // bf16 gradients: the tile goes through shared memory and leaves in
+        // four TMA stores (full lines, rows past the matrix clipped by the
+        // tensor map)
+        const bool issuer = threadIdx.x == 64;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tc = part * 128 + i * 32;  // column within the tile
+          uint8_t* box = stg + (tc / 64) * kWgOutBox + row * 128;
+          const int j0 = (tc % 64) / 8;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint32_t* w8 = buf[i] + 8 * v;
+            *reinterpret_cast<uint4*>(box + (((j0 + v) ^ (row & 7)) << 4)) =
+                make_uint4(ptx::pack_bf16x2(__uint_as_float(w8[0]), __uint_as_float(w8[1])),
+                           ptx::pack_bf16x2(__uint_as_float(w8[2]), __uint_as_float(w8[3])),
+                           ptx::pack_bf16x2(__uint_as_float(w8[4]), __uint_as_float(w8[5])),
+                           ptx::pack_bf16x2(__uint_as_float(w8[6]), __uint_as_float(w8[7])));
+          }
+        }
+        ptx::fence_proxy_async();
+        ptx::named_barrier(1, 32 * kEpiWarps);
+        if (issuer) {
+          const int m0 = t.mb * 128, g = t.shared ? 0 : t.group;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            int mi, col;
+            if (MODE == kWgradW13) {
+              mi = (t.shared ? 2 : 0) + (b >> 1);  // boxes 0-1: dW1, 2-3: dW3
+              col = t.nb * 128 + 64 * (b & 1);
+            } else {
+              mi = t.shared ? 2 : 0;
+              col = t.nb * 256 + 64 * b;
+            }
+            if (col < (t.shared ? p.ncols_shared : p.ncols_routed))
+              ptx::tma_store_3d(&om.m[mi], stg + b * kWgOutBox, col, m0, g);
+          }
+          ptx::bulk_commit_group();
+        }
+        continue;
+      }
       const int M = t.shared ? p.M_shared : p.M_routed;
       const int m = t.mb * 128 + row;
       if (m >= M) continue;
@@ -585,23 +641,15 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
         if (col >= ncols) continue;
         const uint32_t* v32 = buf[i];
         const int64_t off = mat + (int64_t)m * ncols + col;
-        if (p.out_bf16) {
-          uint4* out = reinterpret_cast<uint4*>(static_cast<uint16_t*>(base) + off);
+        float4* out = reinterpret_cast<float4*>(static_cast<float*>(base) + off);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            out[v] = make_uint4(ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 0]), __uint_as_float(v32[8 * v + 1])),
-                                ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 2]), __uint_as_float(v32[8 * v + 3])),
-                                ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 4]), __uint_as_float(v32[8 * v + 5])),
-                                ptx::pack_bf16x2(__uint_as_float(v32[8 * v + 6]), __uint_as_float(v32[8 * v + 7])));
-        } else {
-          float4* out = reinterpret_cast<float4*>(static_cast<float*>(base) + off);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            out[v] = make_float4(__uint_as_float(v32[4 * v]), __uint_as_float(v32[4 * v + 1]),
-                                 __uint_as_float(v32[4 * v + 2]), __uint_as_float(v32[4 * v + 3]));
-        }
+        for (int v = 0; v < 8; ++v)
+          out[v] = make_float4(__uint_as_float(v32[4 * v]), __uint_as_float(v32[4 * v + 1]),
+                               __uint_as_float(v32[4 * v + 2]), __uint_as_float(v32[4 * v + 3]));
       }
     }
+    // the last tile's stores complete before the CTA exits
+    if (p.out_bf16 && threadIdx.x == 64) ptx::bulk_wait_all();
   }
 
   ptx::tc_fence_before();
@@ -659,7 +707,8 @@ cudaError_t launch_dgrad(int mode, const DgradMaps& maps, const DgradParams& p, 
 }
 
 cudaError_t launch_wgrad(int mode, const CUtensorMap& tmA_r, const CUtensorMap& tmA_s, const CUtensorMap& tmB_r,
-                         const CUtensorMap& tmB_s, const WgradParams& p, int grid, cudaStream_t stream) {
+                         const CUtensorMap& tmB_s, const WgradOutMaps& om, const WgradParams& p, int grid,
+                         cudaStream_t stream) {
   const size_t smem = wgrad_smem_bytes();
   auto kernel = mode == kWgradW13 ? wgrad_kernel<kWgradW13> : wgrad_kernel<kWgradPlain>;
   cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -667,7 +716,7 @@ cudaError_t launch_wgrad(int mode, const CUtensorMap& tmA_r, const CUtensorMap& 
   const int total = p.n_routed * p.mb_routed * p.nb_routed + (p.has_shared ? p.mb_shared * p.nb_shared : 0);
   grid = std::min(grid, total);
   if (grid <= 0) return cudaSuccess;
-  err = launch_chained(kernel, dim3(grid), dim3(kThreads), smem, stream, tmA_r, tmA_s, tmB_r, tmB_s, p);
+  err = launch_chained(kernel, dim3(grid), dim3(kThreads), smem, stream, tmA_r, tmA_s, tmB_r, tmB_s, om, p);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

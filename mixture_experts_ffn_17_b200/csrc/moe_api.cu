@@ -746,7 +746,16 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
     q.out2_shared = dW3s;
     q.out_bf16 = gbf16 ? 1 : 0;
     q.status = status;
-    MOE_CUDA(launch_wgrad(kWgradW13, ax_r, ax_s, bg, bg, q, sms, st));
+    WgradOutMaps om{};
+    om.m[0] = om.m[1] = om.m[2] = om.m[3] = ax_r;  // placeholders for fp32 gradients (stored directly)
+    if (gbf16) {
+      if (!map_3d(&om.m[0], dW1, s.inter, s.d, s.E, 128) || !map_3d(&om.m[1], dW3, s.inter, s.d, s.E, 128))
+        return MOE_ERR_CUDA;
+      if (sh && (!map_3d(&om.m[2], dW1s, s.shared_inter, s.d, 1, 128) ||
+                 !map_3d(&om.m[3], dW3s, s.shared_inter, s.d, 1, 128)))
+        return MOE_ERR_CUDA;
+    }
+    MOE_CUDA(launch_wgrad(kWgradW13, ax_r, ax_s, bg, bg, om, q, sms, st));
   }
   {
     CUtensorMap ah, bo_r, bo_s;
@@ -771,7 +780,13 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
     q.out1_shared = dW2s;
     q.out_bf16 = gbf16 ? 1 : 0;
     q.status = status;
-    MOE_CUDA(launch_wgrad(kWgradPlain, ah, ah, bo_r, bo_s, q, sms, st));
+    WgradOutMaps om{};
+    om.m[0] = om.m[1] = om.m[2] = om.m[3] = ah;
+    if (gbf16) {
+      if (!map_3d(&om.m[0], dW2, s.d, s.inter, s.E, 128)) return MOE_ERR_CUDA;
+      if (sh && !map_3d(&om.m[2], dW2s, s.d, s.shared_inter, 1, 128)) return MOE_ERR_CUDA;
+    }
+    MOE_CUDA(launch_wgrad(kWgradPlain, ah, ah, bo_r, bo_s, om, q, sms, st));
   }
   {
     CUtensorMap al, bx;
@@ -788,7 +803,10 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
     q.out1_shared = dWg;
     q.out_bf16 = gbf16 ? 1 : 0;
     q.status = status;
-    MOE_CUDA(launch_wgrad(kWgradPlain, al, al, bx, bx, q, sms, st));
+    WgradOutMaps om{};
+    om.m[0] = om.m[1] = om.m[2] = om.m[3] = al;
+    if (gbf16 && !map_3d(&om.m[2], dWg, s.d, s.E, 1, 128)) return MOE_ERR_CUDA;
+    MOE_CUDA(launch_wgrad(kWgradPlain, al, al, bx, bx, om, q, sms, st));
   }
   return MOE_OK;
 }

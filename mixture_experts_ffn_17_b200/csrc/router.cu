@@ -40,6 +40,13 @@ constexpr int kRouterStages = MOE_ROUTER_STAGES;
 
 constexpr int kRouterAccBufs = 4;    // TMEM buffers: the MMA may run this many K chunks ahead of the drain
 constexpr int kRouterDrainCols = 16; // accumulator columns per drain warp
+// K chunks (64 deep each) a drain lane sums in fp32 before widening the sum
+// to fp64 once: the widening runs on the XU pipe (16 per clock per SM) and
+// bounds the kernel when done for every chunk.
+#ifndef MOE_ROUTER_FP32_CHUNKS
+#define MOE_ROUTER_FP32_CHUNKS 4
+#endif
+constexpr int kRouterFp32Chunks = MOE_ROUTER_FP32_CHUNKS;
 
 template <int EB>
 struct RouterSmem {
@@ -156,8 +163,12 @@ __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
     const int c0 = ((warp - 2) >> 2) * kRouterDrainCols;  // first accumulator column it drains
     const int row = q * 32 + lane;
     double acc[kRouterDrainCols];
+    float part32[kRouterDrainCols];
 #pragma unroll
-    for (int j = 0; j < kRouterDrainCols; ++j) acc[j] = 0.0;
+    for (int j = 0; j < kRouterDrainCols; ++j) {
+      acc[j] = 0.0;
+      part32[j] = 0.0f;
+    }
     bool ok = true;
     for (int kb = 0; kb < nk; ++kb) {
       const int b = kb % kRouterAccBufs;
@@ -173,8 +184,20 @@ __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
       ptx::tmem_ld_wait(r);
       ptx::tc_fence_before();
       ptx::mbar_arrive(&tempty[b]);
+      if (kRouterFp32Chunks == 1) {
 #pragma unroll
-      for (int i = 0; i < kRouterDrainCols; ++i) acc[i] += (double)__uint_as_float(r[i]);
+        for (int i = 0; i < kRouterDrainCols; ++i) acc[i] += (double)__uint_as_float(r[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < kRouterDrainCols; ++i) part32[i] += __uint_as_float(r[i]);
+        if ((kb + 1) % kRouterFp32Chunks == 0 || kb + 1 == nk) {
+#pragma unroll
+          for (int i = 0; i < kRouterDrainCols; ++i) {
+            acc[i] += (double)part32[i];
+            part32[i] = 0.0f;
+          }
+        }
+      }
     }
     if (ok && m0 + row < T) {
       if (part == nullptr) {
