@@ -28,8 +28,9 @@
 // count known only on the device.  Tile = (group, 128 output rows, 256 output
 // columns); K runs over the group's rows in steps of 64, both operands
 // MN-major ([64 rows x 64 features] boxes of the row-major activations).  The
-// last K step of a group usually holds rows of the next expert: warp 1 zeroes
-// those rows of both operands in shared memory before the MMA reads them.  A
+// last K step of a group usually holds rows of the next expert: only its
+// 16-row MMA slices with rows of the group are issued, and warp 1 zeroes the
+// rest of the last one in the A operand before the MMA reads it.  A
 // group without rows writes zeros.  bf16 gradients leave through shared
 // memory in TMA stores (a lane holds one output row, so direct stores would
 // touch 32 lines per warp instruction); fp32 gradients are stored directly.  Each output element is produced by one
@@ -337,15 +338,17 @@ __global__ void __launch_bounds__(kThreads, 1) dgrad_kernel(const __grid_constan
 }
 
 // ------------------------------------------------------------------ wgrad
-constexpr int kWgStages = 3;
+constexpr int kWgStages = 2;
 constexpr uint32_t kWgBox = 64 * 64 * 2;            // [64 K rows x 64 features] bf16, 8 KB
 constexpr uint32_t kWgABytes = 2 * kWgBox;          // 128 output rows
 constexpr uint32_t kWgBBytes = 4 * kWgBox;          // 256 output columns
 constexpr uint32_t kWgStageBytes = kWgABytes + kWgBBytes;
 // bf16 output tile staged for the TMA stores: four [128 rows x 64 columns]
-// boxes, 128-byte swizzled like the output tensor maps
+// boxes, 128-byte swizzled like the output tensor maps; two such buffers, so
+// one tile's stores overlap the next tile's staging
 constexpr uint32_t kWgOutBox = 128 * 64 * 2;
-constexpr uint32_t kWgOutBytes = 4 * kWgOutBox;
+constexpr uint32_t kWgOutTile = 4 * kWgOutBox;
+constexpr uint32_t kWgOutBytes = 2 * kWgOutTile;
 constexpr size_t wgrad_smem_bytes() { return 1024 + kWgStages * kWgStageBytes + kWgOutBytes + 256; }
 static_assert(wgrad_smem_bytes() <= 232448, "shared memory budget (wgrad)");
 
@@ -501,12 +504,19 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
           break;
         }
         uint8_t* st = stage0 + s * kWgStageBytes;
-        const int valid = t.rows - kb * kBK;  // rows of this K step inside the group
-        if (valid < kBK) {
-          // 6 boxes x (64 - valid) rows x 8 16-byte chunks; a whole 128-byte
-          // row is zeroed, so the swizzle of its chunks does not matter
-          const int zr = kBK - valid;
-          for (int i = lane; i < 6 * zr * 8; i += 32) {
+        // rows of this K step inside the group: only the 16-row MMA slices
+        // that hold some are issued; the rest of the last such slice (rows
+        // of the next group) is zeroed in A, which the MMA multiplies with B
+        // (every B row a slice can reach holds finite values: written rows,
+        // or zero fill past the end of the tensor)
+        const int valid = t.rows - kb * kBK;
+        const int n_mma = valid < kBK ? (valid + 15) / 16 : kBK / 16;
+        const int zend = n_mma * 16;
+        if (valid < zend) {
+          // 2 A boxes x (zend - valid) rows x 8 16-byte chunks; a whole
+          // 128-byte row is zeroed, so the swizzle of its chunks does not matter
+          const int zr = zend - valid;
+          for (int i = lane; i < 2 * zr * 8; i += 32) {
             const int box = i / (zr * 8);
             const int rem = i - box * zr * 8;
             const int rr = valid + rem / 8, ch = rem & 7;
@@ -519,8 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
           ptx::tc_fence_after();
           const uint32_t a0 = ptx::smem_u32(st);
           const uint32_t b0 = a0 + kWgABytes;
-#pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
+          for (int kk = 0; kk < n_mma; ++kk)
             ptx::mma_bf16(tmem + sl * kSlotCols, ptx::sdesc_sw128(a0 + kk * 2048, kWgBox, 1024),
                           ptx::sdesc_sw128(b0 + kk * 2048, kWgBox, 1024), idesc, (kb | kk) != 0 ? 1u : 0u);
           ptx::mma_commit(&empty[s]);
@@ -551,9 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
       if (!got) raise_status(p.status, abort_flag, kStatusTimeout);
       if (p.out_bf16) {
         // the epilogue warps meet on a named barrier below, so they leave the
-        // loop together or not at all; this barrier is also where the
-        // previous tile's TMA stores are known to have read the staging buffer
-        if (threadIdx.x == 64) ptx::bulk_wait_read_all();
+        // loop together or not at all; this barrier is also where the stores
+        // of two tiles ago are known to have read this tile's staging buffer
+        // (the previous tile's may still be in flight from the other one)
+        if (threadIdx.x == 64) ptx::bulk_wait_read_one_pending();
         if (!ptx::named_barrier_and(1, 32 * kEpiWarps, got)) break;
       } else if (!got) {
         break;
@@ -587,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int tc = part * 128 + i * 32;  // column within the tile
-          uint8_t* box = stg + (tc / 64) * kWgOutBox + row * 128;
+          uint8_t* box = stg + (tl & 1) * kWgOutTile + (tc / 64) * kWgOutBox + row * 128;
           const int j0 = (tc % 64) / 8;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -614,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
               col = t.nb * 256 + 64 * b;
             }
             if (col < (t.shared ? p.ncols_shared : p.ncols_routed))
-              ptx::tma_store_3d(&om.m[mi], stg + b * kWgOutBox, col, m0, g);
+              ptx::tma_store_3d(&om.m[mi], stg + (tl & 1) * kWgOutTile + b * kWgOutBox, col, m0, g);
           }
           ptx::bulk_commit_group();
         }

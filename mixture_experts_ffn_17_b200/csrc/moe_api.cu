@@ -721,10 +721,20 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
 
   // ---- weight gradients
   {
-    CUtensorMap ax_r, ax_s, bg;
+    // the routed dG | dU rows and the shared expert's get maps of their own,
+    // each ending at its last row: the last MMA slice of a group reads zero
+    // fill past it, never another region's rows (whose columns past its own
+    // width are not written)
+    CUtensorMap ax_r, ax_s, bg_r, bg_s;
     if (!map_rows(&ax_r, x_perm, s.d, Tk, 64) || !map_rows(&ax_s, x, s.d, T, 64) ||
-        !map_rows(&bg, dGU, 2 * (uint64_t)Hld, B.rows, 64))
+        !map_rows(&bg_r, dGU, 2 * (uint64_t)Hld, Tk, 64))
       return MOE_ERR_CUDA;
+    if (sh) {
+      const uint16_t* dgu_shared = static_cast<const uint16_t*>(dGU) + Tk * 2 * (int64_t)Hld;
+      if (!map_rows(&bg_s, dgu_shared, 2 * (uint64_t)Hld, T, 64)) return MOE_ERR_CUDA;
+    } else {
+      bg_s = bg_r;
+    }
     WgradParams q{};
     q.offsets = offsets;
     q.n_routed = s.E;
@@ -737,7 +747,7 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
     q.ncols_routed = s.inter;
     q.ncols_shared = s.shared_inter;
     q.a_shared_row0 = 0;
-    q.b_shared_row0 = (int)Tk;
+    q.b_shared_row0 = 0;
     q.shared_rows = s.T;
     q.u_off = Hld;
     q.out1 = dW1;
@@ -755,7 +765,7 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
                  !map_3d(&om.m[3], dW3s, s.shared_inter, s.d, 1, 128)))
         return MOE_ERR_CUDA;
     }
-    MOE_CUDA(launch_wgrad(kWgradW13, ax_r, ax_s, bg, bg, om, q, sms, st));
+    MOE_CUDA(launch_wgrad(kWgradW13, ax_r, ax_s, bg_r, bg_s, om, q, sms, st));
   }
   {
     CUtensorMap ah, bo_r, bo_s;

@@ -117,6 +117,12 @@ __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bul
 // shared-memory source (the buffer may then be rewritten).
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// The same, except that the most recently committed group may still be
+// reading (one store in flight while the next buffer is filled).
+__device__ __forceinline__ void bulk_wait_read_one_pending() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
 // Wait until every bulk group this thread committed has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
