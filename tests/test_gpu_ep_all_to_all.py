@@ -35,7 +35,7 @@ def _rank_tokens(base, r):
     """Rank r's own batch: the base workload's weights, tokens from another seed."""
     w = workloads.make(base.cfg.replace(seed=base.cfg.seed + 101 * (r + 1)))
     return to_device(workloads.Workload(base.cfg, w.x, base.Wg, base.W1, base.W3, base.W2, base.W1s, base.W3s,
-                                        base.W2s))
+                                        base.W2s, bias=base.bias))
 
 
 def _check(base, world, mutate=None):
@@ -48,7 +48,7 @@ def _check(base, world, mutate=None):
     weights = [ep.shard_weights_a2a(wdev.W1, wdev.W3, wdev.W2, wdev.W1s, wdev.W3s, wdev.W2s, r, world)
                for r in range(world)]
     ys = [torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda") for _ in range(world)]
-    ep.simulate_all_to_all(shape, [w.x for w in ranks], wdev.Wg, None, weights, ys)
+    ep.simulate_all_to_all(shape, [w.x for w in ranks], wdev.Wg, wdev.bias, weights, ys)
     torch.cuda.synchronize()
     received = []
     for r, w in enumerate(ranks):
@@ -70,6 +70,13 @@ def _check(base, world, mutate=None):
 def test_all_to_all_ranks_match_the_layer(world, E):
     base = workloads.make_small("prefill", T=160, d=512, E=E, k=4, inter=256, shared_inter=256)
     _check(base, world)
+
+
+def test_all_to_all_group_routing_with_bias():
+    # sigmoid group-limited routing with the selection bias (8 groups of 16,
+    # top-4 groups, x 2.5), bf16 experts, 2 ranks
+    base = workloads.make_small("fp8", T=160, d=512, E=128, k=8, inter=256, shared_inter=256, fp8=False)
+    _check(base, 2)
 
 
 def test_all_to_all_rank_without_rows_and_no_shared_expert():
