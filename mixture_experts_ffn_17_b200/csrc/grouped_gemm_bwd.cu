@@ -338,7 +338,21 @@ __global__ void __launch_bounds__(kThreads, 1) dgrad_kernel(const __grid_constan
 }
 
 // ------------------------------------------------------------------ wgrad
-constexpr int kWgStages = 2;
+// operand ring depth and output staging buffers (build knobs): the short K
+// loops of the weight gradients (2-3 steps per tile at prefill) wait on L2
+// latency unless enough stages are in flight
+#ifndef MOE_WGRAD_STAGES
+#define MOE_WGRAD_STAGES 3
+#endif
+#ifndef MOE_WGRAD_OUT_BUFS
+#define MOE_WGRAD_OUT_BUFS 1
+#endif
+constexpr int kWgStages = MOE_WGRAD_STAGES;
+// 2: two whole-tile buffers (one tile's stores overlap the next tile's
+// staging); 1: one whole-tile buffer; 0: one half-tile buffer that the tile's
+// two 128-column halves take in turn (frees 32 KB for the operand ring)
+constexpr int kWgOutBufs = MOE_WGRAD_OUT_BUFS;
+static_assert(kWgOutBufs >= 0 && kWgOutBufs <= 2, "output staging: 0 (half tile), 1 or 2 tiles");
 constexpr uint32_t kWgBox = 64 * 64 * 2;            // [64 K rows x 64 features] bf16, 8 KB
 constexpr uint32_t kWgABytes = 2 * kWgBox;          // 128 output rows
 constexpr uint32_t kWgBBytes = 4 * kWgBox;          // 256 output columns
@@ -348,7 +362,7 @@ constexpr uint32_t kWgStageBytes = kWgABytes + kWgBBytes;
 // one tile's stores overlap the next tile's staging
 constexpr uint32_t kWgOutBox = 128 * 64 * 2;
 constexpr uint32_t kWgOutTile = 4 * kWgOutBox;
-constexpr uint32_t kWgOutBytes = 2 * kWgOutTile;
+constexpr uint32_t kWgOutBytes = kWgOutBufs == 0 ? kWgOutTile / 2 : kWgOutBufs * kWgOutTile;
 constexpr size_t wgrad_smem_bytes() { return 1024 + kWgStages * kWgStageBytes + kWgOutBytes + 256; }
 static_assert(wgrad_smem_bytes() <= 232448, "shared memory budget (wgrad)");
 
@@ -563,7 +577,12 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
         // loop together or not at all; this barrier is also where the stores
         // of two tiles ago are known to have read this tile's staging buffer
         // (the previous tile's may still be in flight from the other one)
-        if (threadIdx.x == 64) ptx::bulk_wait_read_one_pending();
+        if (threadIdx.x == 64) {
+          if (kWgOutBufs == 2)
+            ptx::bulk_wait_read_one_pending();
+          else
+            ptx::bulk_wait_read_all();  // 0 or 1 buffer: the previous stores must have read it
+        }
         if (!ptx::named_barrier_and(1, 32 * kEpiWarps, got)) break;
       } else if (!got) {
         break;
@@ -594,39 +613,69 @@ __global__ void __launch_bounds__(kThreads, 1) wgrad_kernel(const __grid_constan
         // four TMA stores (full lines, rows past the matrix clipped by the
         // tensor map)
         const bool issuer = threadIdx.x == 64;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int tc = part * 128 + i * 32;  // column within the tile
-          uint8_t* box = stg + (tl & 1) * kWgOutTile + (tc / 64) * kWgOutBox + row * 128;
-          const int j0 = (tc % 64) / 8;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint32_t* w8 = buf[i] + 8 * v;
-            *reinterpret_cast<uint4*>(box + (((j0 + v) ^ (row & 7)) << 4)) =
-                make_uint4(ptx::pack_bf16x2(__uint_as_float(w8[0]), __uint_as_float(w8[1])),
-                           ptx::pack_bf16x2(__uint_as_float(w8[2]), __uint_as_float(w8[3])),
-                           ptx::pack_bf16x2(__uint_as_float(w8[4]), __uint_as_float(w8[5])),
-                           ptx::pack_bf16x2(__uint_as_float(w8[6]), __uint_as_float(w8[7])));
+        const int m0 = t.mb * 128, g = t.shared ? 0 : t.group;
+        const int ncols = t.shared ? p.ncols_shared : p.ncols_routed;
+        // output box b (64 columns of the tile) -> tensor map index and column
+        auto box_target = [&](int b, int& mi, int& col) {
+          if (MODE == kWgradW13) {
+            mi = (t.shared ? 2 : 0) + (b >> 1);  // boxes 0-1: dW1, 2-3: dW3
+            col = t.nb * 128 + 64 * (b & 1);
+          } else {
+            mi = t.shared ? 2 : 0;
+            col = t.nb * 256 + 64 * b;
           }
-        }
-        ptx::fence_proxy_async();
-        ptx::named_barrier(1, 32 * kEpiWarps);
-        if (issuer) {
-          const int m0 = t.mb * 128, g = t.shared ? 0 : t.group;
+        };
+        // this thread's 128 columns (its part) as 16-byte bf16 chunks into the
+        // staging boxes at `dst` (box index relative to the part's first box)
+        auto stage_part = [&](uint8_t* dst) {
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            int mi, col;
-            if (MODE == kWgradW13) {
-              mi = (t.shared ? 2 : 0) + (b >> 1);  // boxes 0-1: dW1, 2-3: dW3
-              col = t.nb * 128 + 64 * (b & 1);
-            } else {
-              mi = t.shared ? 2 : 0;
-              col = t.nb * 256 + 64 * b;
+          for (int i = 0; i < 4; ++i) {
+            uint8_t* box = dst + (i / 2) * kWgOutBox + row * 128;
+            const int j0 = (i & 1) * 4;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint32_t* w8 = buf[i] + 8 * v;
+              *reinterpret_cast<uint4*>(box + (((j0 + v) ^ (row & 7)) << 4)) =
+                  make_uint4(ptx::pack_bf16x2(__uint_as_float(w8[0]), __uint_as_float(w8[1])),
+                             ptx::pack_bf16x2(__uint_as_float(w8[2]), __uint_as_float(w8[3])),
+                             ptx::pack_bf16x2(__uint_as_float(w8[4]), __uint_as_float(w8[5])),
+                             ptx::pack_bf16x2(__uint_as_float(w8[6]), __uint_as_float(w8[7])));
             }
-            if (col < (t.shared ? p.ncols_shared : p.ncols_routed))
-              ptx::tma_store_3d(&om.m[mi], stg + (tl & 1) * kWgOutTile + b * kWgOutBox, col, m0, g);
           }
-          ptx::bulk_commit_group();
+        };
+        if (kWgOutBufs > 0) {
+          uint8_t* tile_buf = stg + (tl % (kWgOutBufs > 0 ? kWgOutBufs : 1)) * kWgOutTile;
+          stage_part(tile_buf + part * 2 * kWgOutBox);
+          ptx::fence_proxy_async();
+          ptx::named_barrier(1, 32 * kEpiWarps);
+          if (issuer) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              int mi, col;
+              box_target(b, mi, col);
+              if (col < ncols) ptx::tma_store_3d(&om.m[mi], tile_buf + b * kWgOutBox, col, m0, g);
+            }
+            ptx::bulk_commit_group();
+          }
+        } else {
+          // the two halves of the tile through one half-tile buffer in turn
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (part == h) stage_part(stg);
+            ptx::fence_proxy_async();
+            ptx::named_barrier(1, 32 * kEpiWarps);
+            if (issuer) {
+#pragma unroll
+              for (int b = 0; b < 2; ++b) {
+                int mi, col;
+                box_target(2 * h + b, mi, col);
+                if (col < ncols) ptx::tma_store_3d(&om.m[mi], stg + b * kWgOutBox, col, m0, g);
+              }
+              ptx::bulk_commit_group();
+              if (h == 0) ptx::bulk_wait_read_all();
+            }
+            if (h == 0) ptx::named_barrier(1, 32 * kEpiWarps);
+          }
         }
         continue;
       }
