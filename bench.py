@@ -459,6 +459,27 @@ def decode_record(args, dist, dev, stream, peaks, peak_src):
     return rec
 
 
+def write_peak_gbs(dev, nbytes=4 << 30):
+    """HBM write rate on this GPU, measured live: the best of ten fills of a
+    buffer larger than L2 (CUDA events).  The copy peak of MEASURED_PEAKS.json
+    moves as many bytes in as out; a write stream alone runs at its own rate,
+    which is what a kernel that mostly writes (the weight gradients) meets."""
+    buf = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        buf.fill_(1.0)
+    torch.cuda.synchronize(dev)
+    best = float("inf")
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(10):
+        s.record()
+        buf.fill_(0.0)
+        e.record()
+        torch.cuda.synchronize(dev)
+        best = min(best, s.elapsed_time(e))
+    del buf
+    return nbytes / (best / 1e3) / 1e9
+
+
 def backward_work(cfg, counts, grad_bytes):
     """Algorithmic FLOPs and bytes of one moe_backward call (the forward it
     recomputes, then the gradients): FLOPs = the forward's + per routed and
@@ -470,8 +491,9 @@ def backward_work(cfg, counts, grad_bytes):
     flops = T * cfg.flops_per_token() + T * k * 12 * d * I + T * 12 * d * Is + 4 * T * E * d
     wbytes = touched_weight_bytes(cfg, counts)
     grads = (E * 3 * d * I + 3 * d * Is + E * d) * grad_bytes
-    nbytes = 2 * wbytes + grads + 2 * E * d * 2 + T * d * 2 + T * d * 4 + T * d * grad_bytes
-    return flops, nbytes
+    reads = 2 * wbytes + 2 * E * d * 2 + T * d * 2 + T * d * 4
+    writes = grads + T * d * grad_bytes
+    return flops, reads + writes, reads, writes
 
 
 def backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src):
@@ -501,17 +523,25 @@ def backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src):
     fws = B.alloc_workspace(B.shape_of(cfg, B.MOE_F32), dev)
     B.forward(B.shape_of(cfg, B.MOE_F32), w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s,
               y, fws, counts=counts)
-    flops, nbytes = backward_work(cfg, counts.cpu().numpy(), 2)
+    flops, nbytes, rbytes, wbytes = backward_work(cfg, counts.cpu().numpy(), 2)
     t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     d_roof = max(flops / (DATASHEET_PEAKS["bf16_tflops"] * 1e12), nbytes / (DATASHEET_PEAKS["hbm_gbs"] * 1e9))
+    w_gbs = write_peak_gbs(dev)
+    # reads at the copy peak, writes at the measured write rate, one after the other
+    t_rw = rbytes / (peaks["hbm_gbs"] * 1e9) + wbytes / (w_gbs * 1e9)
     return {"what": "moe_backward: forward recompute + dx, dWg, dW1, dW3, dW2 and the shared expert's gradients "
                     "(bf16 gradient outputs, fp32 dy)",
             "steps": K, "ms_per_step": ms, "tokens_per_s": dist.world * cfg.T / (ms / 1e3),
             "tflops": dist.world * flops / (ms / 1e3) / 1e12, "flops": flops, "bytes": nbytes,
+            "bytes_read": rbytes, "bytes_written": wbytes,
             "roofline_ms": 1e3 * max(t_tc, t_hbm), "bound": "hbm" if t_hbm >= t_tc else "tensor",
             "frac": 1e3 * max(t_tc, t_hbm) / ms, "frac_datasheet": 1e3 * d_roof / ms,
-            "peaks": peak_src, "clocks": clocks}
+            "write_gbs_measured": w_gbs, "roofline_ms_write_aware": 1e3 * max(t_tc, t_rw),
+            "frac_write_aware": 1e3 * max(t_tc, t_rw) / ms,
+            "peaks": peak_src + " (copy peak for every byte; the write-aware figure prices the gradient writes at "
+                                "the write rate measured live by a fill of 4 GiB)",
+            "clocks": clocks}
 
 
 def run_ours(args, dist):

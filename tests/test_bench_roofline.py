@@ -49,3 +49,15 @@ def test_decode_touched_weights_count_only_touched_experts():
     counts[:200] = 2
     counts[200] = 112
     assert bench.touched_weight_bytes(cfg, counts) == 202 * 3 * 7168 * 2048 * 2
+
+
+def test_backward_work_counts_two_weight_reads_and_every_gradient_write():
+    cfg = workloads.CONFIGS["prefill"]
+    counts = np.full(cfg.E, cfg.T * cfg.k // cfg.E)
+    flops, nbytes, reads, writes = bench.backward_work(cfg, counts, 2)
+    # the forward's FLOPs and twice them again (input and weight gradients)
+    assert flops == cfg.T * cfg.flops_per_token() * 3
+    weights = 257 * 3 * 7168 * 2048 * 2
+    assert reads == 2 * weights + 2 * 256 * 7168 * 2 + 4096 * 7168 * (2 + 4)
+    assert writes == weights + 256 * 7168 * 2 + 4096 * 7168 * 2     # dW*, dWg and dx in bf16
+    assert nbytes == reads + writes
