@@ -291,6 +291,25 @@ moe_status moe_backward(const moe_shape* shape, const void* x, const void* Wg, c
                         const float* dy, void* dx, void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s,
                         void* dW2s, void* ws, size_t ws_bytes, void* stream);
 
+/* The same gradient in two calls, for a training step that keeps the
+ * forward's state instead of recomputing it (the HBM holds it easily):
+ * moe_forward_train is moe_forward (y in shape->y_dtype, the same value)
+ * that also leaves in `ws` -- a moe_backward_workspace_size workspace -- the
+ * logits, the routing, the permuted rows, g and u (bf16), H and the routed
+ * expert outputs; moe_backward_saved then computes every gradient from that
+ * state (same results as moe_backward on the same inputs).  Between the two
+ * calls the workspace must not be reused, and x, Wg, the weights and the
+ * shape must be the ones the forward saw.  Arguments, layouts and errors as
+ * moe_forward / moe_backward; moe_backward_saved takes no bias (the routing
+ * is the saved one). */
+moe_status moe_forward_train(const moe_shape* shape, const void* x, const void* Wg, const float* bias,
+                             const void* W1, const void* W3, const void* W2, const void* W1s, const void* W3s,
+                             const void* W2s, void* y, void* ws, size_t ws_bytes, void* stream);
+moe_status moe_backward_saved(const moe_shape* shape, const void* x, const void* Wg, const void* W1, const void* W3,
+                              const void* W2, const void* W1s, const void* W3s, const void* W2s, const float* dy,
+                              void* dx, void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s,
+                              void* dW2s, void* ws, size_t ws_bytes, void* stream);
+
 /* The whole layer: router, dispatch, grouped experts, shared expert and
  * combine, with no host synchronisation.
  *   y [T, d] out (fp32 or bf16 per shape->y_dtype)

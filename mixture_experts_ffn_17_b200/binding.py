@@ -25,7 +25,8 @@ EXPORTED = ("moe_workspace_size", "moe_router_topk", "moe_permute", "moe_grouped
             "moe_forward", "moe_forward_profiled", "moe_check_device_status", "moe_status_string", "moe_version",
             "moe_permute_noalloc", "moe_router_topk_limited", "moe_expert_utilisation", "moe_forward_ep",
             "moe_forward_launches", "moe_combine_backward", "moe_router_backward", "moe_backward_workspace_size",
-            "moe_backward", "moe_shared_expert", "moe_ep_regroup_layout", "moe_gather_rows")
+            "moe_backward", "moe_shared_expert", "moe_ep_regroup_layout", "moe_gather_rows", "moe_forward_train",
+            "moe_backward_saved")
 NUM_STAGE_EVENTS = 6
 STAGES = ("router", "dispatch", "experts_up", "experts_down", "combine")
 
@@ -92,11 +93,13 @@ def lib() -> ctypes.CDLL:
         L.moe_backward_workspace_size.argtypes = [S]
         L.moe_backward_workspace_size.restype = sz
         L.moe_backward.argtypes = [S] + [P] * 18 + [P, sz, P]
+        L.moe_forward_train.argtypes = [S] + [P] * 10 + [P, sz, P]
+        L.moe_backward_saved.argtypes = [S] + [P] * 17 + [P, sz, P]
         L.moe_check_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         for fn in ("moe_router_topk", "moe_permute", "moe_grouped_swiglu", "moe_combine", "moe_combine_backward",
                    "moe_router_backward", "moe_forward",
                    "moe_forward_profiled", "moe_forward_ep", "moe_backward", "moe_shared_expert", "moe_ep_regroup_layout", "moe_gather_rows",
-                   "moe_check_device_status"):
+                   "moe_forward_train", "moe_backward_saved", "moe_check_device_status"):
             getattr(L, fn).restype = ctypes.c_int
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
@@ -274,6 +277,23 @@ def backward(shape, x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, dy, dx, dWg, dW1, dW
                               _ptr(W1s), _ptr(W3s), _ptr(W2s), _ptr(dy), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3),
                               _ptr(dW2), _ptr(dW1s), _ptr(dW3s), _ptr(dW2s), _ptr(ws),
                               ws.numel() if ws is not None else 0, _stream(stream)), "moe_backward")
+
+
+def forward_train(shape, x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, y, ws, stream=None):
+    """moe_forward_train: the layer's y, keeping the forward's state in the
+    backward workspace `ws` for backward_saved."""
+    _check(lib().moe_forward_train(ctypes.byref(shape), _ptr(x), _ptr(Wg), _ptr(bias), _ptr(W1), _ptr(W3), _ptr(W2),
+                                   _ptr(W1s), _ptr(W3s), _ptr(W2s), _ptr(y), _ptr(ws),
+                                   ws.numel() if ws is not None else 0, _stream(stream)), "moe_forward_train")
+
+
+def backward_saved(shape, x, Wg, W1, W3, W2, W1s, W3s, W2s, dy, dx, dWg, dW1, dW3, dW2, dW1s, dW3s, dW2s, ws,
+                   stream=None):
+    """moe_backward_saved: every gradient from the state forward_train left in `ws`."""
+    _check(lib().moe_backward_saved(ctypes.byref(shape), _ptr(x), _ptr(Wg), _ptr(W1), _ptr(W3), _ptr(W2), _ptr(W1s),
+                                    _ptr(W3s), _ptr(W2s), _ptr(dy), _ptr(dx), _ptr(dWg), _ptr(dW1), _ptr(dW3),
+                                    _ptr(dW2), _ptr(dW1s), _ptr(dW3s), _ptr(dW2s), _ptr(ws),
+                                    ws.numel() if ws is not None else 0, _stream(stream)), "moe_backward_saved")
 
 
 def check_device_status(ws, stream=None) -> tuple[int, int]:

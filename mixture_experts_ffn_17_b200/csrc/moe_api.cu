@@ -538,17 +538,19 @@ bool map_rows(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, u
   return map_2d(m, ptr, inner, outer, 64, box_outer);
 }
 
-moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, const float* bias, const void* W1,
-                         const void* W3, const void* W2, const void* W1s, const void* W3s, const void* W2s,
-                         const float* dy, void* dx, void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s,
-                         void* dW2s, void* ws, cudaStream_t st) {
+// The forward of the training pass: routing, dispatch and both expert GEMMs,
+// keeping in the backward workspace what the gradient needs (logits, routing,
+// x_perm, g and u in bf16, H, the routed expert outputs Y_perm).  y != nullptr:
+// the shared expert's output too, and the combine into y (shape.y_dtype).
+moe_status train_forward(const moe_shape& s, const void* x, const void* Wg, const float* bias, const void* W1,
+                         const void* W3, const void* W2, const void* W1s, const void* W3s, const void* W2s, void* y,
+                         void* ws, cudaStream_t st) {
   const BwdLayout B = make_bwd_layout(s);
   const Layout& L = B.f;
   const bool sh = s.shared_inter > 0;
-  const int64_t T = s.T, Tk = s.T * s.k;
+  const int64_t Tk = s.T * s.k;
   const int Hld = L.Hld;
   const int sms = num_sms();
-  const bool gbf16 = s.y_dtype == MOE_BF16;
   uint32_t* status = at<uint32_t>(ws, L.status);
   int32_t* idx = at<int32_t>(ws, L.idx);
   float* w = at<float>(ws, L.w);
@@ -564,18 +566,7 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
   int32_t* ntiles = at<int32_t>(ws, L.ntiles);
   int* sched = at<int>(ws, L.sched);
   void* GU = at<void>(ws, B.gu);
-  void* dGU = at<void>(ws, B.dgu);
-  void* dO = at<void>(ws, B.dO);
-  void* dy_b = at<void>(ws, B.dy_b);
-  float* dw = at<float>(ws, B.dw);
-  float* dl = at<float>(ws, B.dl);
-  void* dl_b = at<void>(ws, B.dl_b);
-  void* wgT = at<void>(ws, B.wgT);
-  void* dX = at<void>(ws, B.dX);
-  float* dXs = at<float>(ws, B.dXs);
 
-  // ---- forward, keeping what the gradient needs: logits, routing, x_perm,
-  // g and u (bf16), H, and the routed expert outputs Y_perm
   moe_status r = run_router(s, x, Wg, bias, idx, w, logits, at<double>(ws, L.rpart), status, st);
   if (r != MOE_OK) return r;
   MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
@@ -619,10 +610,15 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
   CUtensorMap h_map, w2_r, w2_s;
   if (!map_2d(&h_map, H, Hld, L.Hrows, kGemmBK, kTileM) || !map_3d(&w2_r, W2, s.d, s.inter, s.E, kGemmBK))
     return MOE_ERR_CUDA;
-  w2_s = w2_r;
+  if (sh && y) {
+    if (!map_3d(&w2_s, W2s, s.d, s.shared_inter, 1, kGemmBK)) return MOE_ERR_CUDA;
+  } else {
+    w2_s = w2_r;
+  }
   GemmParams p2 = p1;
   p2.out_gu = nullptr;
-  p2.tile_set = kTilesRouted;  // Y_perm only: the shared expert's output has no gradient use
+  // the gradient needs Y_perm only; the shared expert's output only for y
+  p2.tile_set = y && sh ? kTilesAll : kTilesRouted;
   p2.sched_counter = sched + 2;
   p2.n_nb = (s.d + gemm_block_n_down() - 1) / gemm_block_n_down();
   p2.K_routed = s.inter;
@@ -631,10 +627,51 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
   p2.N_shared = s.d;
   p2.a_shared_row_offset = (int)Tk;
   p2.out_routed = Y_perm;
-  p2.out_shared = nullptr;
+  p2.out_shared = y && sh ? at<float>(ws, L.Y_shared) : nullptr;
+  p2.out_shared_row_offset = 0;
   p2.ld_out = s.d;
   const int grid2 = (int)std::min<int64_t>(sms, (int64_t)B.max_mtiles * p2.n_nb);
   MOE_CUDA(launch_grouped_down(h_map, w2_r, w2_s, p2, grid2, st));
+  if (y)
+    MOE_CUDA(launch_combine(Y_perm, sh ? at<float>(ws, L.Y_shared) : nullptr, row_of, w, s.T, s.k, s.d, y,
+                            s.y_dtype == MOE_BF16, st));
+  return MOE_OK;
+}
+
+
+// The gradient from the state train_forward left in the workspace.
+moe_status train_backward(const moe_shape& s, const void* x, const void* Wg, const void* W1, const void* W3,
+                          const void* W2, const void* W1s, const void* W3s, const void* W2s, const float* dy, void* dx,
+                          void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s, void* dW2s, void* ws,
+                          cudaStream_t st) {
+  const BwdLayout B = make_bwd_layout(s);
+  const Layout& L = B.f;
+  const bool sh = s.shared_inter > 0;
+  const int64_t T = s.T, Tk = s.T * s.k;
+  const int Hld = L.Hld;
+  const int sms = num_sms();
+  const bool gbf16 = s.y_dtype == MOE_BF16;
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  int32_t* idx = at<int32_t>(ws, L.idx);
+  float* w = at<float>(ws, L.w);
+  float* logits = at<float>(ws, L.logits);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* row_of = at<int32_t>(ws, L.row_of);
+  void* x_perm = at<void>(ws, L.x_perm);
+  uint16_t* H = at<uint16_t>(ws, L.H);
+  void* Y_perm = at<void>(ws, L.Y_perm);
+  int4* tiles = at<int4>(ws, B.tiles);
+  int32_t* ntiles = at<int32_t>(ws, L.ntiles);
+  void* GU = at<void>(ws, B.gu);
+  void* dGU = at<void>(ws, B.dgu);
+  void* dO = at<void>(ws, B.dO);
+  void* dy_b = at<void>(ws, B.dy_b);
+  float* dw = at<float>(ws, B.dw);
+  float* dl = at<float>(ws, B.dl);
+  void* dl_b = at<void>(ws, B.dl_b);
+  void* wgT = at<void>(ws, B.wgT);
+  void* dX = at<void>(ws, B.dX);
+  float* dXs = at<float>(ws, B.dXs);
 
   // ---- combine and routing steps
   MOE_CUDA(launch_combine_backward(dy, Y_perm, row_of, w, s.T, s.k, s.d, dO, dw, st));
@@ -817,6 +854,47 @@ moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, cons
     om.m[0] = om.m[1] = om.m[2] = om.m[3] = al;
     if (gbf16 && !map_3d(&om.m[2], dWg, s.d, s.E, 1, 128)) return MOE_ERR_CUDA;
     MOE_CUDA(launch_wgrad(kWgradPlain, al, al, bx, bx, om, q, sms, st));
+  }
+  return MOE_OK;
+}
+
+moe_status backward_impl(const moe_shape& s, const void* x, const void* Wg, const float* bias, const void* W1,
+                         const void* W3, const void* W2, const void* W1s, const void* W3s, const void* W2s,
+                         const float* dy, void* dx, void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s,
+                         void* dW2s, void* ws, cudaStream_t st) {
+  moe_status r = train_forward(s, x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, nullptr, ws, st);
+  if (r != MOE_OK) return r;
+  return train_backward(s, x, Wg, W1, W3, W2, W1s, W3s, W2s, dy, dx, dWg, dW1, dW3, dW2, dW1s, dW3s, dW2s, ws, st);
+}
+
+// Arguments of the training calls (moe_backward, moe_forward_train,
+// moe_backward_saved): bf16 experts, the pointers each needs, alignment and
+// workspace.
+moe_status check_train_args(const moe_shape* shape, const void* const* need, int n_need, const void* const* opt,
+                            int n_opt, const void* ws, size_t ws_bytes) {
+  moe_status v = validate_backward(shape);
+  if (v != MOE_OK) return v;
+  for (int i = 0; i < n_need; ++i)
+    if (!need[i] || !aligned16(need[i])) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < n_opt; ++i)
+    if (opt[i] && !aligned16(opt[i])) return MOE_ERR_INVALID_ARG;
+  if (!ws_ok(ws, ws_bytes, make_bwd_layout(*shape).total)) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+// Every weight gradient of an empty batch is zero.
+moe_status zero_weight_grads(const moe_shape& s, void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s,
+                             void* dW2s, cudaStream_t st) {
+  const size_t gb = s.y_dtype == MOE_BF16 ? 2 : 4;
+  const size_t eI = (size_t)s.E * s.d * s.inter * gb, sI = (size_t)s.d * s.shared_inter * gb;
+  MOE_CUDA(cudaMemsetAsync(dWg, 0, (size_t)s.E * s.d * gb, st));
+  MOE_CUDA(cudaMemsetAsync(dW1, 0, eI, st));
+  MOE_CUDA(cudaMemsetAsync(dW3, 0, eI, st));
+  MOE_CUDA(cudaMemsetAsync(dW2, 0, eI, st));
+  if (s.shared_inter > 0) {
+    MOE_CUDA(cudaMemsetAsync(dW1s, 0, sI, st));
+    MOE_CUDA(cudaMemsetAsync(dW3s, 0, sI, st));
+    MOE_CUDA(cudaMemsetAsync(dW2s, 0, sI, st));
   }
   return MOE_OK;
 }
@@ -1070,6 +1148,40 @@ size_t moe_backward_workspace_size(const moe_shape* shape) {
   return make_bwd_layout(*shape).total;
 }
 
+moe_status moe_forward_train(const moe_shape* shape, const void* x, const void* Wg, const float* bias,
+                                        const void* W1, const void* W3, const void* W2, const void* W1s,
+                                        const void* W3s, const void* W2s, void* y, void* ws, size_t ws_bytes,
+                                        void* stream) {
+  if (!shape) return MOE_ERR_INVALID_ARG;
+  const bool sh = shape->shared_inter > 0;
+  const void* need[] = {x, Wg, W1, W3, W2, y, sh ? W1s : x, sh ? W3s : x, sh ? W2s : x};
+  const void* opt[] = {bias};
+  moe_status v = check_train_args(shape, need, 9, opt, 1, ws, ws_bytes);
+  if (v != MOE_OK) return v;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_CUDA(cudaMemsetAsync(at<uint32_t>(ws, make_bwd_layout(*shape).f.status), 0, 4, st));
+  if (shape->T == 0) return MOE_OK;
+  return train_forward(*shape, x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, y, ws, st);
+}
+
+moe_status moe_backward_saved(const moe_shape* shape, const void* x, const void* Wg, const void* W1,
+                                         const void* W3, const void* W2, const void* W1s, const void* W3s,
+                                         const void* W2s, const float* dy, void* dx, void* dWg, void* dW1, void* dW3,
+                                         void* dW2, void* dW1s, void* dW3s, void* dW2s, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  if (!shape) return MOE_ERR_INVALID_ARG;
+  const bool sh = shape->shared_inter > 0;
+  const void* need[] = {x, Wg, W1, W3, W2, dy, dx, dWg, dW1, dW3, dW2, sh ? W1s : x, sh ? W3s : x, sh ? W2s : x,
+                        sh ? dW1s : x, sh ? dW3s : x, sh ? dW2s : x};
+  moe_status v = check_train_args(shape, need, 17, nullptr, 0, ws, ws_bytes);
+  if (v != MOE_OK) return v;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the status word keeps what moe_forward_train raised
+  if (shape->T == 0) return zero_weight_grads(*shape, dWg, dW1, dW3, dW2, dW1s, dW3s, dW2s, st);
+  return train_backward(*shape, x, Wg, W1, W3, W2, W1s, W3s, W2s, dy, dx, dWg, dW1, dW3, dW2, dW1s, dW3s, dW2s, ws,
+                        st);
+}
+
 moe_status moe_backward(const moe_shape* shape, const void* x, const void* Wg, const float* bias, const void* W1,
                         const void* W3, const void* W2, const void* W1s, const void* W3s, const void* W2s,
                         const float* dy, void* dx, void* dWg, void* dW1, void* dW3, void* dW2, void* dW1s, void* dW3s,
@@ -1087,21 +1199,7 @@ moe_status moe_backward(const moe_shape* shape, const void* x, const void* Wg, c
   if (!ws_ok(ws, ws_bytes, B.total)) return MOE_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   MOE_CUDA(cudaMemsetAsync(at<uint32_t>(ws, B.f.status), 0, 4, st));
-  if (s.T == 0) {
-    // no tokens: every weight gradient is zero
-    const size_t gb = s.y_dtype == MOE_BF16 ? 2 : 4;
-    const size_t eI = (size_t)s.E * s.d * s.inter * gb, sI = (size_t)s.d * s.shared_inter * gb;
-    MOE_CUDA(cudaMemsetAsync(dWg, 0, (size_t)s.E * s.d * gb, st));
-    MOE_CUDA(cudaMemsetAsync(dW1, 0, eI, st));
-    MOE_CUDA(cudaMemsetAsync(dW3, 0, eI, st));
-    MOE_CUDA(cudaMemsetAsync(dW2, 0, eI, st));
-    if (sh) {
-      MOE_CUDA(cudaMemsetAsync(dW1s, 0, sI, st));
-      MOE_CUDA(cudaMemsetAsync(dW3s, 0, sI, st));
-      MOE_CUDA(cudaMemsetAsync(dW2s, 0, sI, st));
-    }
-    return MOE_OK;
-  }
+  if (s.T == 0) return zero_weight_grads(s, dWg, dW1, dW3, dW2, dW1s, dW3s, dW2s, st);  // no tokens
   return backward_impl(s, x, Wg, bias, W1, W3, W2, W1s, W3s, W2s, dy, dx, dWg, dW1, dW3, dW2, dW1s, dW3s, dW2s, ws,
                        st);
 }

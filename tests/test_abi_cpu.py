@@ -229,3 +229,26 @@ def test_backward_validation_without_gpu():
     # without a shared expert its weights and gradients may be NULL
     s0 = B.make_shape(T=128, d=512, E=32, k=4, inter=256, shared_inter=0)
     assert B.backward_workspace_size(s0) > 0
+
+
+def test_training_calls_validation_without_gpu():
+    L = B.lib()
+    s = B.make_shape(T=128, d=512, E=32, k=4, inter=256, shared_inter=256)
+    n = B.backward_workspace_size(s)
+    keep, p = _fake()
+    nul = None
+    # moe_forward_train: x Wg bias W1 W3 W2 W1s W3s W2s y | ws n stream
+    fa = [p, p, nul, p, p, p, p, p, p, p, p, n, nul]
+    for i in (0, 1, 3, 6, 9):
+        a = list(fa); a[i] = nul
+        assert L.moe_forward_train(ctypes.byref(s), *a) == B.MOE_ERR_INVALID_ARG, i
+    a = list(fa); a[11] = B.workspace_size(s)          # the forward's workspace is too small
+    assert L.moe_forward_train(ctypes.byref(s), *a) == B.MOE_ERR_WORKSPACE
+    # moe_backward_saved: x Wg W1 W3 W2 W1s W3s W2s dy | dx dWg dW1 dW3 dW2 dW1s dW3s dW2s | ws n stream
+    ba = [p] * 17 + [p, n, nul]
+    for i in (0, 8, 9, 13, 16):
+        a = list(ba); a[i] = nul
+        assert L.moe_backward_saved(ctypes.byref(s), *a) == B.MOE_ERR_INVALID_ARG, i
+    s8 = B.make_shape(T=128, d=512, E=32, k=4, inter=256, shared_inter=256, w_dtype=B.MOE_E4M3)
+    assert L.moe_forward_train(ctypes.byref(s8), *fa) == B.MOE_ERR_UNSUPPORTED
+    assert L.moe_backward_saved(ctypes.byref(s8), *ba) == B.MOE_ERR_UNSUPPORTED

@@ -11,7 +11,7 @@ from mixture_experts_ffn_17_b200 import binding as B
 from mixture_experts_ffn_17_b200 import build as libbuild
 from mixture_experts_ffn_17_b200 import workloads
 
-from gpu_util import to_device
+from gpu_util import run_forward, to_device
 from parity import TOL_BF16, dec, to_np
 
 pytestmark = pytest.mark.gpu
@@ -283,3 +283,27 @@ def test_backward_bf16_gradients_and_determinism():
     for name in h:
         # the bf16 gradients are the fp32 ones rounded once
         assert torch.equal(h[name], g32[name].to(torch.bfloat16)), name
+
+
+@pytest.mark.parametrize("shared", [384, 0])
+def test_training_step_with_saved_state_matches_recomputing_calls(shared):
+    # moe_forward_train + moe_backward_saved give moe_forward's y and
+    # moe_backward's gradients, bit for bit (same kernels, same order)
+    w = _medium(T=700, shared_inter=shared)
+    cfg = w.cfg
+    dy = torch.randn(cfg.T, cfg.d, generator=torch.Generator(device="cuda").manual_seed(11), device="cuda")
+    ref, _ = _backward(w, dy)
+    y_ref, *_ = run_forward(w)
+    shape = B.shape_of(cfg, B.MOE_F32)
+    ws = B.alloc_backward_workspace(shape)
+    y = torch.empty_like(y_ref)
+    B.forward_train(shape, w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.W1s, w.W3s, w.W2s, y, ws)
+    z = lambda *sz: torch.full(sz, float("nan"), dtype=torch.float32, device="cuda")
+    g = {k: z(*v.shape) for k, v in ref.items()}
+    B.backward_saved(shape, w.x, w.Wg, w.W1, w.W3, w.W2, w.W1s, w.W3s, w.W2s, dy, g["dx"], g["dWg"], g["dW1"],
+                     g["dW3"], g["dW2"], g.get("dW1s"), g.get("dW3s"), g.get("dW2s"), ws)
+    rc, raw = B.check_device_status(ws)
+    assert rc == B.MOE_OK, (rc, raw)
+    assert torch.equal(y, y_ref)
+    for name in ref:
+        assert torch.equal(g[name], ref[name]), name

@@ -85,3 +85,46 @@ def test_forward_replays_in_a_cuda_graph(case):
         assert torch.equal(y_graph, y_eager), (rep, (y_graph - y_eager).abs().max().item())
         assert torch.isfinite(y_graph).all()
     del g
+
+
+def test_backward_replays_in_a_cuda_graph():
+    # moe_backward makes no host synchronisation either: a captured call
+    # replayed on new output gradients equals eager calls bit for bit
+    w = to_device(workloads.make_small("prefill", T=600, d=1024, E=64, k=6, inter=512, shared_inter=384))
+    cfg = w.cfg
+    shape = B.shape_of(cfg, B.MOE_BF16)
+    ws = B.alloc_backward_workspace(shape)
+    e = lambda *sz: torch.empty(sz, dtype=torch.bfloat16, device="cuda")
+    grads = [e(cfg.T, cfg.d), e(cfg.E, cfg.d), e(cfg.E, cfg.d, cfg.inter), e(cfg.E, cfg.d, cfg.inter),
+             e(cfg.E, cfg.inter, cfg.d), e(cfg.d, cfg.shared_inter), e(cfg.d, cfg.shared_inter),
+             e(cfg.shared_inter, cfg.d)]
+    dy_static = torch.zeros(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+
+    def call(dy, out):
+        B.backward(shape, w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.W1s, w.W3s, w.W2s, dy, *out, ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call(dy_static, grads)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call(dy_static, grads)
+    gen = torch.Generator(device="cuda").manual_seed(77)
+    for rep in range(2):
+        dy = torch.randn(cfg.T, cfg.d, generator=gen, device="cuda")
+        dy_static.copy_(dy)
+        g.replay()
+        torch.cuda.synchronize()
+        got = [t.clone() for t in grads]
+        eager = [torch.empty_like(t) for t in grads]
+        call(dy, eager)
+        torch.cuda.synchronize()
+        rc, raw = B.check_device_status(ws)
+        assert rc == B.MOE_OK, (rc, raw)
+        for a, b in zip(got, eager):
+            assert torch.equal(a, b), rep
+        assert all(torch.isfinite(t.float()).all() for t in got)
+    del g
