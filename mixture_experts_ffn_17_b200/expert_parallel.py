@@ -230,7 +230,12 @@ def forward_all_to_all(shape, rank: int, world: int, x, Wg, bias, w: A2AWeights,
     """This rank's y (its own tokens) through the all-to-all layer, with the
     tokens split into `chunks` batches whose exchanges overlap the other
     batches' expert GEMMs.  Every rank of the group calls it with the same
-    `chunks` (the collectives run in the same order everywhere)."""
+    `chunks` (the collectives run in the same order everywhere).  `stream`
+    (default: the current one) orders the kernels and the collectives alike:
+    torch.distributed enqueues its work after the current stream's."""
+    if stream is not None:
+        with torch.cuda.stream(stream):
+            return forward_all_to_all(shape, rank, world, x, Wg, bias, w, y, transport, chunks, None)
     transport = transport or ProcessGroupTransport()
     T = shape.T
     bounds = [T * c // chunks for c in range(chunks + 1)]
