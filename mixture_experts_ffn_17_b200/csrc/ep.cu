@@ -63,7 +63,6 @@ __global__ void __launch_bounds__(kEpThreads)
   __shared__ int32_t total;
   __shared__ int32_t src_start[kEpThreads];  // source-major start of segment (s, e) at s * E_local + e
   __shared__ int32_t em_start[kEpThreads];   // expert-major start of the same segment
-  __shared__ int32_t exp_start[kEpThreads];  // offsets_local
   grid_dependency_wait();
   const int i = threadIdx.x;
   const int nseg = n_src * E_local;
@@ -77,7 +76,6 @@ __global__ void __launch_bounds__(kEpThreads)
     for (int s = 0; s < n_src; ++s) te += max(cnt[s * E_local + i], 0);
   const int32_t es = block_exclusive_scan(te, warp_tot, &total);
   if (i < E_local) {
-    exp_start[i] = es;
     offsets_local[i] = es;
     int32_t run = es;
     for (int s = 0; s < n_src; ++s) {

@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) dgrad_kernel(const __grid_constan
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_bf16(kTileM, 256, false, false);
-      int kg = 0, tl = 0;
+      int kg = 0;
       uint32_t use[2] = {0u, 0u};
       int next = 0;
       bool ok = true;
@@ -227,7 +227,6 @@ __global__ void __launch_bounds__(kThreads, 1) dgrad_kernel(const __grid_constan
           ++use[sl];
         }
         next = (next + ti.halves) & 1;
-        ++tl;
       }
       ptx::mma_commit(done);
       if (!ptx::wait_bounded(done, 0, &never)) raise_status(p.status, abort_flag, kStatusTimeout);
