@@ -14,13 +14,14 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from mixture_experts_ffn_17_b200 import binding as B
 from mixture_experts_ffn_17_b200 import build as libbuild
 from mixture_experts_ffn_17_b200 import expert_parallel as ep
 from mixture_experts_ffn_17_b200 import workloads
 
 from gpu_util import oracle_full, route_with_exemptions, run_forward, to_device
-from parity import TOL_BF16, max_rel_err, to_np
+from parity import TOL_BF16, dec, max_rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -120,3 +121,39 @@ def test_chunked_driver_on_a_one_rank_nccl_group():
     y1, *_ = run_forward(base)
     rms = float(y1.double().pow(2).mean().sqrt())
     assert float((y - y1).abs().max()) <= 1e-3 * rms
+
+
+def test_all_to_all_v3_decode_eight_ranks():
+    # V3 shapes: 256 experts over 8 simulated ranks (32 each), each rank with
+    # its own decode batch of 64 tokens; every rank's y against the whole layer
+    # on one GPU, rank 0's against the fp64 oracle on all its tokens
+    from gpu_util import oracle_sampled
+    base_cfg = workloads.CONFIGS["decode"]
+    world = 8
+    base = workloads.make(base_cfg, device="cuda")
+    ranks = []
+    for r in range(world):
+        g = torch.Generator(device="cuda").manual_seed(base_cfg.seed + 17 * (r + 1))
+        z = torch.randn(base_cfg.T, base_cfg.d, generator=g, device="cuda")
+        x = (z / z.pow(2).mean(dim=1, keepdim=True).sqrt()).to(torch.bfloat16)
+        ranks.append(workloads.Workload(base_cfg, x, base.Wg, base.W1, base.W3, base.W2, base.W1s, base.W3s,
+                                        base.W2s))
+    shape = B.shape_of(base_cfg)
+    weights = [ep.shard_weights_a2a(base.W1, base.W3, base.W2, base.W1s, base.W3s, base.W2s, r, world)
+               for r in range(world)]
+    ys = [torch.empty(base_cfg.T, base_cfg.d, dtype=torch.float32, device="cuda") for _ in range(world)]
+    ep.simulate_all_to_all(shape, [w.x for w in ranks], base.Wg, None, weights, ys)
+    torch.cuda.synchronize()
+    for r, w in enumerate(ranks):
+        y1, idx, _, _, _ = run_forward(w)
+        rms = float(y1.double().pow(2).mean().sqrt())
+        assert float((ys[r] - y1).abs().max()) <= 1e-3 * rms, r
+    w = ranks[0]
+    lg = oracle.logits(dec(w.x), dec(w.Wg))
+    _, idx, _, _, _ = run_forward(w)
+    _, _, merged, report, n_near = route_with_exemptions(w, lg, to_np(idx))
+    assert len(report) <= n_near
+    y_o = oracle_sampled(w, lg, merged, np.arange(base_cfg.T))
+    err = max_rel_err(to_np(ys[0]).astype(np.float64), y_o)
+    print(f"all-to-all, 8 ranks, V3 decode shapes: rank 0 max|err|/rms = {err:.2e}")
+    assert err <= TOL_BF16, err
