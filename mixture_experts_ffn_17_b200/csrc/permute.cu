@@ -199,6 +199,13 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// MOE_PAIR_LAST_ALL=1: a segment with full 256-row tiles also puts its last
+// tile, however short, on the pair list (right after its full tiles, while
+// its weights are still in L2) instead of the one-CTA list.
+#ifndef MOE_PAIR_LAST_ALL
+#define MOE_PAIR_LAST_ALL 0
+#endif
+
 // Tile lists for the grouped GEMMs: one int4 {group, row_start, rows,
 // row tiles of the group's segment} per
 // 256-row tile of each expert segment of [e_lo, e_hi) (group e, rows in
@@ -222,8 +229,11 @@ __global__ void build_tiles_kernel(const int32_t* __restrict__ offsets, int E, i
     start = offsets[e];
     cnt = offsets[e + 1] - start;
     const int rem = cnt % kTileRows;
-    mt_full = split ? cnt / kTileRows + (rem > kPairMinRows) : 0;
-    mt_part = split ? (rem != 0 && rem <= kPairMinRows) : (cnt + kTileRows - 1) / kTileRows;
+    // a segment's last tile goes on the pair list when it is nearly full, or
+    // (MOE_PAIR_LAST_ALL) whenever the segment also has full tiles there
+    const bool last_pair = rem > kPairMinRows || (MOE_PAIR_LAST_ALL && rem > 0 && cnt >= kTileRows);
+    mt_full = split ? cnt / kTileRows + last_pair : 0;
+    mt_part = split ? (rem != 0 && !last_pair) : (cnt + kTileRows - 1) / kTileRows;
   }
   // one scan of both counts: full tiles in the high word, partial in the low
   const long long mine_t = ((long long)mt_full << 32) | (unsigned)mt_part;

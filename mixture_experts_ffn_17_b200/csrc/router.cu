@@ -38,9 +38,18 @@ constexpr int kRouterBK = 64;
 #endif
 constexpr int kRouterStages = MOE_ROUTER_STAGES;
 
-constexpr int kRouterAccBufs = 4;    // TMEM buffers: the MMA may run this many K chunks ahead of the drain
-constexpr int kRouterDrainCols = 16; // accumulator columns per drain warp
-// K chunks (64 deep each) a drain lane sums in fp32 before widening the sum
+constexpr int kRouterAccBufs = 4;    // TMEM buffers: the MMA may run this many K groups ahead of the drain
+#ifndef MOE_ROUTER_DRAIN_COLS
+#define MOE_ROUTER_DRAIN_COLS 16
+#endif
+constexpr int kRouterDrainCols = MOE_ROUTER_DRAIN_COLS;  // accumulator columns per drain warp
+// K chunks (64 deep each) the tensor core accumulates into one TMEM buffer
+// before the drain reads it (a K group).
+#ifndef MOE_ROUTER_MMA_CHUNKS
+#define MOE_ROUTER_MMA_CHUNKS 1
+#endif
+constexpr int kRouterMmaChunks = MOE_ROUTER_MMA_CHUNKS;
+// K groups a drain lane sums in fp32 before widening the sum
 // to fp64 once: the widening runs on the XU pipe (16 per clock per SM) and
 // bounds the kernel when done for every chunk.
 #ifndef MOE_ROUTER_FP32_CHUNKS
@@ -52,11 +61,24 @@ template <int EB>
 struct RouterSmem {
   static constexpr int kDrainWarps = 4 * (EB / kRouterDrainCols);
   static constexpr int kThreads = 64 + 32 * kDrainWarps;
+  static_assert(kThreads <= 1024, "too many drain warps for one CTA");
   static constexpr uint32_t kABytes = kRouterBM * kRouterBK * 2;
   static constexpr uint32_t kBBytes = EB * kRouterBK * 2;
-  static constexpr uint32_t kTmemCols = kRouterAccBufs * EB <= 128 ? 128 : 256;
+  static constexpr uint32_t kAccCols = kRouterAccBufs * EB;
+  static_assert(kAccCols <= 512, "TMEM holds 512 columns");
+  static constexpr uint32_t kTmemCols = kAccCols <= 128 ? 128 : (kAccCols <= 256 ? 256 : 512);
   static constexpr size_t kBytes = 1024 + kRouterStages * (kABytes + kBBytes) + 256;
 };
+
+// A drain lane's columns of one finished K group, read from TMEM.
+__device__ __forceinline__ void drain_load(uint32_t taddr, uint32_t (&r)[16]) {
+  ptx::tmem_ld16(taddr, r);
+  ptx::tmem_ld_wait(r);
+}
+__device__ __forceinline__ void drain_load(uint32_t taddr, uint32_t (&r)[32]) {
+  ptx::tmem_ld32(taddr, r);
+  ptx::tmem_ld_wait(r);
+}
 
 template <int EB>
 __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
@@ -138,9 +160,12 @@ __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
       for (int kb = 0; kb < nk; ++kb) {
         const int s = kb % S;
         const uint32_t ph = (kb / S) & 1;
-        const int b = kb % kRouterAccBufs;
-        const uint32_t use = kb / kRouterAccBufs;
-        if (!ptx::wait_bounded(&tempty[b], (use & 1) ^ 1, abort_flag) ||
+        const int gi = kb / kRouterMmaChunks;  // K group
+        const bool first = kb % kRouterMmaChunks == 0;
+        const bool last = (kb + 1) % kRouterMmaChunks == 0 || kb + 1 == nk;
+        const int b = gi % kRouterAccBufs;
+        const uint32_t use = gi / kRouterAccBufs;
+        if ((first && !ptx::wait_bounded(&tempty[b], (use & 1) ^ 1, abort_flag)) ||
             !ptx::wait_bounded(&full[s], ph, abort_flag)) {
           raise_status(status, abort_flag, kStatusTimeout);
           break;
@@ -151,9 +176,9 @@ __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kRouterBK / 16; ++kk)
           ptx::mma_bf16(tmem + b * EB, ptx::sdesc_sw128(a0 + kk * 32, 16, 1024),
-                        ptx::sdesc_sw128(b0 + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+                        ptx::sdesc_sw128(b0 + kk * 32, 16, 1024), idesc, (kk > 0 || !first) ? 1u : 0u);
         ptx::mma_commit(&empty[s]);
-        ptx::mma_commit(&tfull[b]);
+        if (last) ptx::mma_commit(&tfull[b]);
       }
       ptx::mma_commit(done);
       if (!ptx::wait_bounded(done, 0, &never)) raise_status(status, abort_flag, kStatusTimeout);
@@ -170,7 +195,8 @@ __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
       part32[j] = 0.0f;
     }
     bool ok = true;
-    for (int kb = 0; kb < nk; ++kb) {
+    const int ng = (nk + kRouterMmaChunks - 1) / kRouterMmaChunks;  // K groups
+    for (int kb = 0; kb < ng; ++kb) {
       const int b = kb % kRouterAccBufs;
       const uint32_t use = kb / kRouterAccBufs;
       if (!ptx::wait_bounded(&tfull[b], use & 1, abort_flag)) {
@@ -180,8 +206,7 @@ __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
       }
       ptx::tc_fence_after();
       uint32_t r[kRouterDrainCols];
-      ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + b * EB + c0, r);
-      ptx::tmem_ld_wait(r);
+      drain_load(tmem + ((uint32_t)(q * 32) << 16) + b * EB + c0, r);
       ptx::tc_fence_before();
       ptx::mbar_arrive(&tempty[b]);
       if (kRouterFp32Chunks == 1) {
@@ -190,7 +215,7 @@ __global__ void __launch_bounds__(RouterSmem<EB>::kThreads, 1)
       } else {
 #pragma unroll
         for (int i = 0; i < kRouterDrainCols; ++i) part32[i] += __uint_as_float(r[i]);
-        if ((kb + 1) % kRouterFp32Chunks == 0 || kb + 1 == nk) {
+        if ((kb + 1) % kRouterFp32Chunks == 0 || kb + 1 == ng) {
 #pragma unroll
           for (int i = 0; i < kRouterDrainCols; ++i) {
             acc[i] += (double)part32[i];
@@ -399,7 +424,12 @@ cudaError_t launch_topk_nv(const float* logits, const float* bias, const uint8_t
 
 }  // namespace
 
+#ifndef MOE_ROUTER_EB
+#define MOE_ROUTER_EB 64
+#endif
+
 int router_expert_block(int E) {
+  if (MOE_ROUTER_EB >= 128 && E % 128 == 0) return 128;
   if (E % 64 == 0) return 64;
   if (E % 32 == 0) return 32;
   return 0;
@@ -420,6 +450,9 @@ int router_splits(int64_t T, int d, int E, int sms) {
 cudaError_t launch_router_logits(const CUtensorMap& tm_x, const CUtensorMap& tm_wg, int T, int d, int E, int splits,
                                  float* logits, double* part, uint32_t* status, cudaStream_t stream) {
   switch (router_expert_block(E)) {
+#if MOE_ROUTER_EB >= 128
+    case 128: return launch_router_logits<128>(tm_x, tm_wg, T, d, E, splits, logits, part, status, stream);
+#endif
     case 64: return launch_router_logits<64>(tm_x, tm_wg, T, d, E, splits, logits, part, status, stream);
     case 32: return launch_router_logits<32>(tm_x, tm_wg, T, d, E, splits, logits, part, status, stream);
     default: return cudaErrorInvalidValue;
