@@ -116,10 +116,8 @@ struct TileInfo {
 // the slot: the half-subpartition layout of the 64-row tcgen05.mma.
 __device__ __forceinline__ bool narrow_half(const TileInfo& ti, int h) { return ti.rows - h * kTileM <= kTileM / 2; }
 
-// The part of the tile list this launch walks: `count` tile-list rows.  A
-// launch over the whole list interleaves the shared expert's rows evenly among
-// the routed ones (the shared weights stay in L2 while routed tiles keep HBM
-// busy); the routed-only and shared-only launches walk their range in order.
+// The part of the tile list this launch walks: `count` tile-list rows from
+// `begin` (the whole list, the routed tiles only, or the shared expert's).
 struct TileSpan {
   int begin, count, routed, shared;
 };
@@ -135,19 +133,15 @@ __device__ __forceinline__ TileSpan tile_span(const GemmParams& p) {
   return t;
 }
 
-__device__ __forceinline__ int tile_row(const GemmParams& p, const TileSpan& sp, int q, bool interleave) {
-  if (!interleave || p.tile_set != kTilesAll || sp.shared == 0) return sp.begin + q;
-  const int stride = sp.count / sp.shared;  // >= 1; shared row j sits at slot (j+1)*stride-1
-  const int before = min(sp.shared, (q + 1) / stride);
-  if ((q + 1) % stride == 0 && (q + 1) / stride <= sp.shared) return sp.routed + (q + 1) / stride - 1;
-  return q - before;
-}
-
-__device__ __forceinline__ bool tile_at(const GemmParams& p, const TileSpan& sp, int tile, int BN, TileInfo& ti,
-                                        bool interleave = true) {
+// Work item `tile` = row tile q (in list order: the routed experts' tiles,
+// then the shared expert's) x column block nb, column blocks of a row tile
+// consecutive.  The shared expert's tiles run back to back at the end, so
+// its weights stay in L2 across its row tiles without being held there for
+// the whole launch.
+__device__ __forceinline__ bool tile_at(const GemmParams& p, const TileSpan& sp, int tile, int BN, TileInfo& ti) {
   const int q = tile / p.n_nb;
   ti.nb = tile - q * p.n_nb;
-  const int4 e = p.tiles[tile_row(p, sp, q, interleave)];
+  const int4 e = p.tiles[sp.begin + q];
   ti.group = e.x;
   ti.row0 = e.y;
   ti.rows = e.z;
@@ -312,7 +306,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
                              : MOE_GEMM_A_POLICY == 1 ? ptx::policy_evict_normal()
                                                       : ptx::policy_evict_last();
       const uint64_t pol_w = ptx::policy_evict_first();  // each weight tile is read once
-      const uint64_t pol_ws = ptx::policy_evict_last();  // the shared expert's weights serve every row tile
+
       int kg = 0, ns = 0;
       bool ok = !p.debug_withhold_loads;
       while (ok) {
@@ -331,9 +325,12 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         if (tile < 0) break;
         TileInfo ti;
         if (!tile_at(p, span, tile, BN, ti)) continue;
-        // weights of an expert with several row tiles are read again by each
-        // of them: keep them in L2 (evict-normal) instead of streaming them
-        const uint64_t pol_b = ti.shared ? pol_ws : (ti.seg_tiles > 1 ? pol_a : pol_w);
+        // weights of a group with several row tiles (the shared expert, an
+        // expert with many rows) are read again by each of them: keep them in
+        // L2 (evict-normal) instead of streaming them (evict-first); evict-last
+        // would keep them past their last row tile, at the expense of the
+        // weights that stream after them
+        const uint64_t pol_b = (ti.shared || ti.seg_tiles > 1) ? pol_a : pol_w;
         const CUtensorMap* mA = ti.shared ? &tmA_s : &tmA_r;
         const CUtensorMap* mB = ti.shared ? &tmB_s : &tmB_r;
         const CUtensorMap* mC = ti.shared ? &tmC_s : &tmC_r;
@@ -733,21 +730,6 @@ static_assert(kPairStages * kPairStageBytes + 1024 + 256 <= 232448, "shared memo
 
 constexpr size_t pair_smem_bytes() { return 1024 + kPairStages * kPairStageBytes + 256; }
 
-// The shared expert's tiles in the CTA-pair list: after the routed tiles (0)
-// or spread among them (1); its weights loaded evict-normal (0) or
-// evict-last (1).  The pair kernel runs when hot experts have several row
-// tiles each: each such expert's weights (58.7 MB at V3 shapes) should stay
-// in L2 while its row tiles pass, and shared-expert tiles spread among them,
-// with their own 58.7 MB held evict-last, crowd them out.
-#ifndef MOE_PAIR_INTERLEAVE_SHARED
-#define MOE_PAIR_INTERLEAVE_SHARED 0
-#endif
-#ifndef MOE_PAIR_SHARED_EVICT_LAST
-#define MOE_PAIR_SHARED_EVICT_LAST 0
-#endif
-constexpr bool kPairInterleaveShared = MOE_PAIR_INTERLEAVE_SHARED != 0;
-constexpr bool kPairSharedEvictLast = MOE_PAIR_SHARED_EVICT_LAST != 0;
-
 template <Mode M>
 __global__ void __launch_bounds__(kPairThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
@@ -814,15 +796,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       const uint64_t pol_a = ptx::policy_evict_normal();
       const uint64_t pol_w = ptx::policy_evict_first();
-      const uint64_t pol_ws = kPairSharedEvictLast ? ptx::policy_evict_last() : ptx::policy_evict_normal();
       int kg = 0;
       bool ok = !p.debug_withhold_loads;
       for (int tile = cluster; ok && tile < total; tile += clusters) {
         TileInfo ti;
-        if (!tile_at(p, span, tile, BN, ti, kPairInterleaveShared)) continue;
-        // weights of an expert with several row tiles are read again by each
-        // of them: keep them in L2 (evict-normal) instead of streaming them
-        const uint64_t pol_b = ti.shared ? pol_ws : (ti.seg_tiles > 1 ? pol_a : pol_w);
+        if (!tile_at(p, span, tile, BN, ti)) continue;
+        // weights read again by later row tiles stay in L2 (as above)
+        const uint64_t pol_b = (ti.shared || ti.seg_tiles > 1) ? pol_a : pol_w;
         const CUtensorMap* mA = ti.shared ? &tmA_s : &tmA_r;
         // SwiGLU: CTA 0 loads W1's columns, CTA 1 the same columns of W3
         const CUtensorMap* mB = (M == Mode::kSwiGLU && rank == 1) ? (ti.shared ? &tmC_s : &tmC_r)
@@ -860,7 +840,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       bool ok = true;
       for (int tile = cluster; ok && tile < total; tile += clusters) {
         TileInfo ti;
-        if (!tile_at(p, span, tile, BN, ti, kPairInterleaveShared)) continue;
+        if (!tile_at(p, span, tile, BN, ti)) continue;
         const int nk = (ti.shared ? p.K_shared : p.K_routed) / kBK;
         const int sl = tl & 1;
         if (!ptx::wait_bounded(&tempty[sl], ((tl >> 1) & 1) ^ 1, abort_flag)) {
@@ -902,7 +882,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     int tl = 0;
     for (int tile = cluster; tile < total; tile += clusters) {
       TileInfo ti;
-      if (!tile_at(p, span, tile, BN, ti, kPairInterleaveShared)) continue;
+      if (!tile_at(p, span, tile, BN, ti)) continue;
       const int sl = tl & 1;
       if (!ptx::wait_bounded(&tfull[sl], (tl >> 1) & 1, abort_flag)) {
         raise_status(p.status, abort_flag, kStatusTimeout);
