@@ -425,7 +425,7 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   if (ev) MOE_CUDA(cudaEventRecord(ev[1], st));
   MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
                           perm, row_of, status, st));
-  MOE_CUDA(launch_gather_rows(x, perm, s.T * s.k, s.d, x_perm, num_sms(), st, offsets, shard.e_lo, shard.e_hi));
+  MOE_CUDA(launch_scatter_rows(x, row_of, s.T, s.k, s.d, x_perm, num_sms(), st, offsets, shard.e_lo, shard.e_hi));
   r = run_experts(sl, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared, status, st,
                   shard, ev ? ev + 2 : nullptr);
   if (r != MOE_OK) return r;
@@ -571,7 +571,7 @@ moe_status train_forward(const moe_shape& s, const void* x, const void* Wg, cons
   if (r != MOE_OK) return r;
   MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
                           perm, row_of, status, st));
-  MOE_CUDA(launch_gather_rows(x, perm, Tk, s.d, x_perm, sms, st, offsets, 0, s.E));
+  MOE_CUDA(launch_scatter_rows(x, row_of, s.T, s.k, s.d, x_perm, sms, st, offsets, 0, s.E));
   MOE_CUDA(launch_build_tiles(offsets, s.E, s.T, whole_layer(s), true, tiles, ntiles, sched, st, nullptr));
 
   CUtensorMap a_r, a_s, w1_r, w1_s, w3_r, w3_s;
@@ -987,8 +987,8 @@ moe_status moe_permute(const moe_shape* shape, const int32_t* topk_idx, int32_t*
   MOE_CUDA(launch_permute(topk_idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
                           perm_token, row_of, status, st));
   // only the rows the scatter wrote: entries with an out-of-range index are
-  // skipped, so perm_token holds offsets[E] <= T*k tokens
-  if (x) MOE_CUDA(launch_gather_rows(x, perm_token, s.T * s.k, s.d, x_perm, num_sms(), st, offsets, 0, s.E));
+  // skipped (row_of = -1), so offsets[E] <= T*k rows are filled
+  if (x) MOE_CUDA(launch_scatter_rows(x, row_of, s.T, s.k, s.d, x_perm, num_sms(), st, offsets, 0, s.E));
   return MOE_OK;
 }
 
@@ -1306,7 +1306,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_shape* shape, const int32_t*
   int32_t* base = hist + per;
   MOE_CUDA(launch_permute(topk_idx, s.T, s.k, s.E, hist, base, counts, offsets, perm_token, row_of, status, st));
   // only the rows the scatter wrote: entries with an out-of-range index are
-  // skipped, so perm_token holds offsets[E] <= T*k tokens
-  if (x) MOE_CUDA(launch_gather_rows(x, perm_token, s.T * s.k, s.d, x_perm, num_sms(), st, offsets, 0, s.E));
+  // skipped (row_of = -1), so offsets[E] <= T*k rows are filled
+  if (x) MOE_CUDA(launch_scatter_rows(x, row_of, s.T, s.k, s.d, x_perm, num_sms(), st, offsets, 0, s.E));
   return MOE_OK;
 }

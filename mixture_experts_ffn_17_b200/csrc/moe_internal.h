@@ -85,6 +85,11 @@ cudaError_t launch_permute(const int32_t* idx, int64_t T, int k, int E, int32_t*
 cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t rows, int d, void* x_perm,
                                int num_sms, cudaStream_t stream, const int32_t* offsets = nullptr, int e_lo = 0,
                                int e_hi = 0);
+// x_perm[row_of[t*k + j]] = x[t] in token order (each x row read once) for the
+// rows [offsets[e_lo], offsets[e_hi]); the same rows and values as
+// launch_gather_rows over that range.
+cudaError_t launch_scatter_rows(const void* x, const int32_t* row_of, int64_t T, int k, int d, void* x_perm,
+                                int num_sms, cudaStream_t stream, const int32_t* offsets, int e_lo, int e_hi);
 // Also zeroes the grouped GEMMs' tile counters (kNumSchedCounters ints).
 constexpr int kNumSchedCounters = 4;
 // tiles_pair != nullptr: full 256-row tiles go to that list (ntiles[2], [3])

@@ -206,6 +206,47 @@ __global__ void __launch_bounds__(256)
 #define MOE_PAIR_LAST_ALL 0
 #endif
 
+// The same copy in token order: x_perm[row_of[t*k + j], :] = x[t, :] for the
+// rows of [offsets[e_lo], offsets[e_hi]) (every row when e_lo = 0, e_hi = E;
+// an entry with an out-of-range expert has row_of = -1 and is skipped).  Each
+// x row is read once and written k times, where the permuted-order gather
+// reads it k times far apart (x no longer in L2 by then).  A work item is
+// one token's row, or a column part of it when there are few tokens.
+__global__ void __launch_bounds__(256)
+    scatter_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ row_of, int T, int k,
+                        int vec_per_row, int parts, uint4* __restrict__ x_perm, const int32_t* __restrict__ offsets,
+                        int e_lo, int e_hi) {
+  grid_dependency_wait();
+  const int64_t r_lo = offsets[e_lo], r_hi = offsets[e_hi];
+  const int vpp = (vec_per_row + parts - 1) / parts;
+  const int64_t items = (int64_t)T * parts;
+  for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+    const int t = (int)(it / parts);
+    const int v_begin = (int)(it - (int64_t)t * parts) * vpp;
+    const int v_end = min(vec_per_row, v_begin + vpp);
+    const uint4* src = x + (size_t)t * vec_per_row;
+    const int32_t* rows = row_of + (size_t)t * k;
+    for (int v0 = v_begin + threadIdx.x; v0 < v_end; v0 += kGatherUnroll * blockDim.x) {
+      uint4 buf[kGatherUnroll];
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        const int v = v0 + u * blockDim.x;
+        if (v < v_end) buf[u] = __ldg(src + v);
+      }
+      for (int j = 0; j < k; ++j) {
+        const int64_t r = __ldg(rows + j);
+        if (r < r_lo || r >= r_hi) continue;
+        uint4* dst = x_perm + (size_t)r * vec_per_row;
+#pragma unroll
+        for (int u = 0; u < kGatherUnroll; ++u) {
+          const int v = v0 + u * blockDim.x;
+          if (v < v_end) dst[v] = buf[u];
+        }
+      }
+    }
+  }
+}
+
 // Tile lists for the grouped GEMMs: one int4 {group, row_start, rows,
 // row tiles of the group's segment} per
 // 256-row tile of each expert segment of [e_lo, e_hi) (group e, rows in
@@ -319,6 +360,23 @@ cudaError_t launch_gather_rows(const void* x, const int32_t* perm_token, int64_t
   const int64_t g = std::min<int64_t>(rows, (int64_t)num_sms * 16);
   const cudaError_t err = launch_chained(gather_rows_kernel, dim3((unsigned)g), dim3(256), 0, stream,
                                          static_cast<const uint4*>(x), perm_token, rows, d / 8,
+                                         static_cast<uint4*>(x_perm), offsets, e_lo, e_hi);
+  return err != cudaSuccess ? err : cudaGetLastError();
+}
+
+cudaError_t launch_scatter_rows(const void* x, const int32_t* row_of, int64_t T, int k, int d, void* x_perm,
+                                int num_sms, cudaStream_t stream, const int32_t* offsets, int e_lo, int e_hi) {
+  if (T == 0) return cudaSuccess;
+  const int vec = d / 8;
+  // enough work items to cover the device: split rows into column parts when
+  // tokens are few (at least 32 vectors per part)
+  const int64_t want = (int64_t)num_sms * 4;
+  int parts = (int)std::min<int64_t>((want + T - 1) / T, std::max(1, vec / 32));
+  if (parts < 1) parts = 1;
+  const int64_t items = T * parts;
+  const int64_t g = std::min<int64_t>(items, (int64_t)num_sms * 16);
+  const cudaError_t err = launch_chained(scatter_rows_kernel, dim3((unsigned)g), dim3(256), 0, stream,
+                                         static_cast<const uint4*>(x), row_of, (int)T, k, vec, parts,
                                          static_cast<uint4*>(x_perm), offsets, e_lo, e_hi);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
