@@ -357,8 +357,9 @@ int moe_forward_launches(const moe_shape* shape);
 /* moe_forward plus per-stage timing: records the caller's CUDA events
  * (cudaEvent_t handles, created with timing enabled) on `stream` at the stage
  * boundaries, without synchronising:
- *   [0] start  [1] after the router  [2] after dispatch (permutation, row
- *   gather, tile list)  [3] after the grouped SwiGLU up-projection
+ *   [0] start  [1] after the router  [2] after dispatch (permutation, x rows
+ *   copied into permuted order, tile list)  [3] after the grouped SwiGLU
+ *   up-projection
  *   [4] after the grouped down-projection  [5] after the combine.
  * Same results and launches as moe_forward.  Profiling aid; the pages have no
  * counterpart. */
