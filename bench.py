@@ -459,27 +459,6 @@ def decode_record(args, dist, dev, stream, peaks, peak_src):
     return rec
 
 
-def write_peak_gbs(dev, nbytes=4 << 30):
-    """HBM write rate on this GPU, measured live: the best of ten fills of a
-    buffer larger than L2 (CUDA events).  The copy peak of MEASURED_PEAKS.json
-    moves as many bytes in as out; a write stream alone runs at its own rate,
-    which is what a kernel that mostly writes (the weight gradients) meets."""
-    buf = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
-    for _ in range(3):
-        buf.fill_(1.0)
-    torch.cuda.synchronize(dev)
-    best = float("inf")
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for _ in range(10):
-        s.record()
-        buf.fill_(0.0)
-        e.record()
-        torch.cuda.synchronize(dev)
-        best = min(best, s.elapsed_time(e))
-    del buf
-    return nbytes / (best / 1e3) / 1e9
-
-
 def backward_work(cfg, counts, grad_bytes):
     """Algorithmic FLOPs and bytes of one moe_backward call (the forward it
     recomputes, then the gradients): FLOPs = the forward's + per routed and
@@ -496,7 +475,7 @@ def backward_work(cfg, counts, grad_bytes):
     return flops, reads + writes, reads, writes
 
 
-def backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src, w_gbs):
+def backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src):
     """moe_backward (the training pass: forward recompute and every gradient,
     bf16 gradient outputs) on the same weights, timed like the forward."""
     from mixture_experts_ffn_17_b200 import binding as B
@@ -544,25 +523,19 @@ def backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src, w_gbs):
     t_tc = flops / (peaks["bf16_tflops_sustained"] * 1e12)
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
     d_roof = max(flops / (DATASHEET_PEAKS["bf16_tflops"] * 1e12), nbytes / (DATASHEET_PEAKS["hbm_gbs"] * 1e9))
-    # reads at the copy peak, writes at the write rate measured at the start of
-    # the run, one after the other
-    t_rw = rbytes / (peaks["hbm_gbs"] * 1e9) + wbytes / (w_gbs * 1e9)
+    roof_ms = 1e3 * max(t_tc, t_hbm)
     return {"what": "moe_backward: forward recompute + dx, dWg, dW1, dW3, dW2 and the shared expert's gradients "
                     "(bf16 gradient outputs, fp32 dy)",
             "steps": K, "ms_per_step": ms, "tokens_per_s": dist.world * cfg.T / (ms / 1e3),
             "tflops": dist.world * flops / (ms / 1e3) / 1e12, "flops": flops, "bytes": nbytes,
             "bytes_read": rbytes, "bytes_written": wbytes,
-            "roofline_ms": 1e3 * max(t_tc, t_hbm), "bound": "hbm" if t_hbm >= t_tc else "tensor",
-            "frac": 1e3 * max(t_tc, t_hbm) / ms, "frac_datasheet": 1e3 * d_roof / ms,
-            "write_gbs_measured": w_gbs, "roofline_ms_write_aware": 1e3 * max(t_tc, t_rw),
-            "frac_write_aware": 1e3 * max(t_tc, t_rw) / ms,
+            "roofline_ms": roof_ms, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "frac": roof_ms / ms, "frac_datasheet": 1e3 * d_roof / ms,
             "train_step": {"what": "moe_forward_train (y, the forward's state kept) + moe_backward_saved",
                            "ms_per_step": ms_step, "tokens_per_s": dist.world * cfg.T / (ms_step / 1e3),
                            "forward_train_ms": ms_fwd_train, "backward_saved_ms_derived": ms_step - ms_fwd_train,
-                           "roofline_ms_write_aware": 1e3 * max(t_tc, t_rw),
-                           "frac_write_aware": 1e3 * max(t_tc, t_rw) / ms_step, "clocks": clocks_step},
-            "peaks": peak_src + " (copy peak for every byte; the write-aware figure prices the gradient writes at "
-                                "the write rate measured live, before any timed work, by fills of 4 GiB)",
+                           "roofline_ms": roof_ms, "frac": roof_ms / ms_step, "clocks": clocks_step},
+            "peaks": peak_src + " (HBM copy peak for every byte read or written: plain and bulk stores reach it too)",
             "clocks": clocks}
 
 
@@ -584,8 +557,6 @@ def run_ours(args, dist):
     counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream(dev)
     fwd_args = (shape, w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s, y, ws)
-    # the HBM write rate for the backward record, before any timed work
-    write_gbs = write_peak_gbs(dev) if args.workload == "prefill" and not args.no_backward else None
 
     for _ in range(args.warmup):
         B.forward(*fwd_args, counts=counts)
@@ -663,7 +634,7 @@ def run_ours(args, dist):
         line["cpu_baseline"] = run_cpu_baseline(args, w, cfg)
     if args.workload == "prefill" and not args.no_backward:
         fwd_args = None
-        line["backward"] = backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src, write_gbs)
+        line["backward"] = backward_record(args, dist, dev, stream, w, cfg, peaks, peak_src)
         torch.cuda.empty_cache()
     if args.workload == "prefill" and not (args.tokens or args.experts or args.no_decode):
         # the decode batch of the same layer shapes, in the same run (its own
