@@ -33,8 +33,11 @@ def built():
 
 
 def _check_v3(name, sample_size, tol=TOL_BF16):
-    cfg = workloads.CONFIGS[name]
-    w = workloads.make(cfg, device="cuda")
+    return _check_workload(name, workloads.make(workloads.CONFIGS[name], device="cuda"), sample_size, tol)
+
+
+def _check_workload(name, w, sample_size, tol=TOL_BF16):
+    cfg = w.cfg
     y, idx, tw, counts, ws = run_forward(w)
     idx_d = to_np(idx)
     lg = oracle_logits(w)
@@ -88,3 +91,25 @@ def test_v3_skewed_sampled():
 def test_v3_fp8_group_routing_sampled():
     c, _ = _check_v3("fp8", SAMPLE, tol=TOL_FP8)
     assert (c > 0).sum() > 200
+
+
+# The largest batches the library takes are bounded by T*k + T < 2**31 rows,
+# not by the V3 configs: a narrow layer (d=256, 64 experts, inter 128) at
+# T = 200,000 tokens (1.6M routed rows, 12x the skewed batch) runs the
+# permutation, the tile lists and both grouped-GEMM schedulers far past the V3
+# sizes, near-uniform and Zipf-skewed (segments of tens of thousands of rows,
+# CTA pairs), against the oracle on all tokens' routing and a sampled output.
+LARGE = dict(T=200_000, d=256, E=64, k=8, inter=128, shared_inter=128)
+
+
+def test_large_batch_narrow_layer_uniform():
+    w = workloads.make_small("prefill", device="cuda", **LARGE)
+    c, _ = _check_workload("large uniform", w, SAMPLE)
+    assert c.sum() == LARGE["T"] * LARGE["k"] and (c > 0).all()
+
+
+def test_large_batch_narrow_layer_skewed():
+    w = workloads.make_small("skewed", device="cuda", **LARGE)
+    c, _ = _check_workload("large skewed", w, SAMPLE)
+    assert c.sum() == LARGE["T"] * LARGE["k"]
+    assert c.max() > 100 * 256                # segments of hundreds of 256-row tiles
