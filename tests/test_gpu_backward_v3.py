@@ -39,8 +39,20 @@ def _close(d, o, what):
 
 
 def test_v3_prefill_backward_sampled():
-    cfg = workloads.CONFIGS["prefill"]
-    w = workloads.make(cfg, device="cuda")
+    _check_backward_sampled(workloads.make(workloads.CONFIGS["prefill"], device="cuda"))
+
+
+def test_large_batch_narrow_layer_skewed_backward():
+    # 100,000 tokens of a narrow layer with Zipf routing: the weight gradients
+    # of the hot experts contract over tens of thousands of rows (a K loop of
+    # hundreds of 64-row steps per tile), far past the V3 prefill segments
+    w = workloads.make_small("skewed", device="cuda", T=100_000, d=256, E=64, k=8, inter=128, shared_inter=128)
+    c = _check_backward_sampled(w)
+    assert c.max() > 20_000
+
+
+def _check_backward_sampled(w):
+    cfg = w.cfg
     dy = torch.randn(cfg.T, cfg.d, generator=torch.Generator(device="cuda").manual_seed(314), device="cuda")
     shape = B.shape_of(cfg, B.MOE_BF16)
     ws = B.alloc_backward_workspace(shape)
@@ -94,3 +106,4 @@ def test_v3_prefill_backward_sampled():
         dl = obw.routing_backward(lg[t, merged[t]], wts[t], dw_t, cfg.route, cfg.route_scale)
         dx_t += dl @ Wg[merged[t]]
         _close(to_np(g["dx"][t].float()), dx_t, f"dx[{t}]")
+    return c
