@@ -113,3 +113,11 @@ def test_large_batch_narrow_layer_skewed():
     c, _ = _check_workload("large skewed", w, SAMPLE)
     assert c.sum() == LARGE["T"] * LARGE["k"]
     assert c.max() > 100 * 256                # segments of hundreds of 256-row tiles
+
+
+def test_large_batch_narrow_layer_fp8_group_routing():
+    # the FP8 recipe (e4m3 experts with 128x128 block scales, sigmoid
+    # group-limited routing with a selection bias) at the same large batch
+    w = workloads.make_small("fp8", device="cuda", **LARGE)
+    c, _ = _check_workload("large fp8", w, SAMPLE, tol=TOL_FP8)
+    assert c.sum() == LARGE["T"] * LARGE["k"]
