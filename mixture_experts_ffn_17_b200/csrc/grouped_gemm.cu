@@ -18,8 +18,10 @@
 //             swizzle: the weights' natural [K, N] row-major layout) into a
 //             3-stage ring (the K depth and stage count are build-time knobs,
 //             MOE_GEMM_BK / MOE_GEMM_STAGES; 64 x 3 measured fastest);
-//   warp 1    single-thread tcgen05.mma issuer, M=128 (M=64 for a half of
-//             at most 64 rows), K=16 per instruction, fp32 accumulators in
+//   warp 1    single-thread tcgen05.mma issuer, M=128 (a half of at most
+//             64 rows: transposed, the weights as an M=128 operand and the
+//             rows as an N=16-64 operand; M=64 with FP8 weights), K=16 per
+//             instruction, fp32 accumulators in
 //             TMEM: two 256-column slots handed out round-robin (a one-half
 //             tile takes one, a two-half tile both), so one-half tiles overlap
 //             their epilogue with the next main loop;
@@ -116,6 +118,25 @@ struct TileInfo {
 // the slot: the half-subpartition layout of the 64-row tcgen05.mma.
 __device__ __forceinline__ bool narrow_half(const TileInfo& ti, int h) { return ti.rows - h * kTileM <= kTileM / 2; }
 
+// With bf16 weights a half of at most 64 rows is computed transposed instead:
+// D^T = W^T x^T, the weight tile (already in shared memory as MN-major boxes)
+// as the M=128 operand and the half's rows (its K-major A box) as an N operand
+// of the rows rounded up to 16.  Per K=16 slice that is two M=128 MMAs of N
+// 16-64 (one per 128 output columns) instead of one M=64 N=256 MMA: about an
+// eighth of the tensor work for the 1-16 rows of a prefill segment's tail or a
+// decode segment.  D^T sits in the half's slot: lane = output column, columns
+// [0, N) for output columns 0-127 of the tile and [128, 128 + N) for 128-255.
+__device__ __forceinline__ int transposed_cols(const TileInfo& ti, int h) {
+  return ((ti.rows - h * kTileM + 15) / 16) * 16;
+}
+
+// With FP8 weights the converted B buffer has its own layout and the narrow
+// half stays an M=64 MMA.
+template <bool F8>
+__device__ __forceinline__ bool transposed_half(const TileInfo& ti, int h) {
+  return !F8 && narrow_half(ti, h);
+}
+
 // The part of the tile list this launch walks: `count` tile-list rows from
 // `begin` (the whole list, the routed tiles only, or the shared expert's).
 struct TileSpan {
@@ -163,6 +184,9 @@ struct SlotRing {
     if (sl) ++u1; else ++u0;
   }
 };
+
+// One fp32 rounded to nearest-even bf16, as its 16 bits.
+__device__ __forceinline__ uint16_t bf16_bits(float v) { return (uint16_t)(ptx::pack_bf16x2(v, 0.0f) & 0xFFFFu); }
 
 // e4m3 codes (4 per word) * scale -> 4 bf16 (two packed words).  The e4m3 ->
 // f16 widening is exact; the product is rounded once to bf16.
@@ -435,8 +459,17 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
             const uint64_t bd = ptx::sdesc_sw128(b0 + kk * 2048, BoxBytes, 1024);
             for (int h = 0; h < ti.halves; ++h) {
               const uint64_t ad = ptx::sdesc(a0 + h * ABytes + kk * 32, 16, ASBO, ASwz);
-              ptx::mma_bf16(tmem + ((ring.next + h) & 1) * kSlotCols, ad, bd, narrow_half(ti, h) ? idesc_narrow : idesc,
-                            acc);
+              const uint32_t dslot = tmem + ((ring.next + h) & 1) * kSlotCols;
+              if (transposed_half<F8>(ti, h)) {
+                // transposed: the weight boxes 0-1 and 2-3 (MN-major) as M=128
+                // operands, the half's rows (K-major) as the N operand
+                const uint32_t idt = ptx::idesc_bf16(kTileM, transposed_cols(ti, h), true, false);
+                ptx::mma_bf16(dslot, bd, ad, idt, acc);
+                ptx::mma_bf16(dslot + 128, ptx::sdesc_sw128(b0 + 2 * BoxBytes + kk * 2048, BoxBytes, 1024), ad, idt,
+                              acc);
+              } else {
+                ptx::mma_bf16(dslot, ad, bd, narrow_half(ti, h) ? idesc_narrow : idesc, acc);
+              }
             }
           }
           ptx::mma_commit(&empty[s]);
@@ -480,6 +513,56 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         const bool narrow = narrow_half(ti, h);
         const int r = h * kTileM + (narrow ? (lane < 16 ? q * 16 + lane : kTileM) : row);  // row within the tile
         const bool valid = r < ti.rows && (!narrow || lane < 16);
+        if (transposed_half<F8>(ti, h)) {
+          // transposed half: this lane holds output column f (and f + 128) of
+          // the tile for the half's rows; each part takes 32 of its <= 64 rows
+          const int f = q * 32 + lane;
+          const int r0 = part * 32;
+          uint32_t da[32], db[32];
+          ptx::tmem_ld32(tbase + r0, da);
+          ptx::tmem_ld32(tbase + 128 + r0, db);
+          ptx::tmem_ld_wait2(da, db);
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&tempty[sl]);
+          const int nr = ti.rows - h * kTileM - r0;  // rows of this part (may be <= 0)
+          const int64_t grow0 = (int64_t)ti.row0 + h * kTileM + r0 + (ti.shared ? p.out_shared_row_offset : 0);
+          if (M == Mode::kSwiGLU) {
+            uint16_t* base = static_cast<uint16_t*>(ti.shared ? p.out_shared : p.out_routed);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nr) {
+                const float g = __uint_as_float(da[j]), u = __uint_as_float(db[j]);
+                const int64_t hrow = grow0 + j;
+                base[hrow * p.ld_out + n0 + f] = bf16_bits(g / (1.0f + __expf(-g)) * u);
+                if (p.out_gu) {
+                  uint16_t* gu_row = static_cast<uint16_t*>(p.out_gu) + hrow * 2 * p.ld_out + n0 + f;
+                  gu_row[0] = bf16_bits(g);
+                  gu_row[p.ld_out] = bf16_bits(u);
+                }
+              }
+            }
+          } else {
+            const int N = ti.shared ? p.N_shared : p.N_routed;
+            const bool c0ok = n0 + f < N, c1ok = n0 + 128 + f < N;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (j < nr) {
+                const int64_t orow = grow0 + j;
+                if (ti.shared) {
+                  float* out = static_cast<float*>(p.out_shared) + orow * p.ld_out + n0 + f;
+                  if (c0ok) out[0] = __uint_as_float(da[j]);
+                  if (c1ok) out[128] = __uint_as_float(db[j]);
+                } else {
+                  uint16_t* out = static_cast<uint16_t*>(p.out_routed) + orow * p.ld_out + n0 + f;
+                  if (c0ok) out[0] = bf16_bits(__uint_as_float(da[j]));
+                  if (c1ok) out[128] = bf16_bits(__uint_as_float(db[j]));
+                }
+              }
+            }
+          }
+          ring.bump(sl);
+          continue;
+        }
         if constexpr (!F8) {
           // Drain first: this warp's whole share of the slot (128 fp32 per
           // lane: g and u of two 32-column chunks, or four W2 chunks) is read
