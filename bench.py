@@ -52,6 +52,8 @@ def parse_args():
     p.add_argument("--tokens", type=int, default=None, help="override T (profiling small cases)")
     p.add_argument("--experts", type=int, default=None, help="override E (profiling small cases)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-other", action="store_true",
+                   help="leave out the skewed and FP8 records that the default prefill run adds")
     p.add_argument("--cpu-sample", type=int, default=16, help="tokens the CPU baseline runs through the oracle")
     p.add_argument("--ref-sample", type=int, default=2, help="tokens per step of the reference arm")
     p.add_argument("--no-e2e", action="store_true")
@@ -459,6 +461,40 @@ def decode_record(args, dist, dev, stream, peaks, peak_src):
     return rec
 
 
+def workload_record(name, args, dist, dev, stream, peaks, peak_src):
+    """Another workload of the layer (its own weights) timed in the same run:
+    the burst and a sustained leg against its own layer roofline, with clocks,
+    so that one bench line carries every config's measurement."""
+    from mixture_experts_ffn_17_b200 import binding as B
+    from mixture_experts_ffn_17_b200 import workloads
+    cfg = workloads.CONFIGS[name]
+    w = workloads.make(cfg, device=dev)
+    shape = B.shape_of(cfg, B.MOE_F32)
+    ws = B.alloc_workspace(shape, dev)
+    y = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device=dev)
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    fwd_args = (shape, w.x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s, y, ws)
+    for _ in range(max(args.warmup, 3)):
+        B.forward(*fwd_args, counts=counts)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"{name}: device status after warm-up (raw {raw})")
+    K = args.steps
+    ms, clocks = time_loop(lambda i: B.forward(*fwd_args, counts=counts), K, stream, dev, dist)
+    roof = layer_roofline(cfg, counts.cpu().numpy(), ms, peaks, peak_src)
+    rec = {"workload": config_of(cfg, args)["workload"], "steps": K, "ms_per_step": ms,
+           "tokens_per_s": dist.world * cfg.T / (ms / 1e3), "tflops": dist.world * roof["flops"] / (ms / 1e3) / 1e12,
+           "roofline_layer": roof, "clocks": clocks}
+    if args.sustain_s > 0:
+        rec["sustained"] = sustained_leg(B, fwd_args, counts, cfg, K, ms, args.sustain_s, stream, dev, dist, peaks,
+                                         peak_src)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"{name}: device status after the timed steps (raw {raw})")
+    rec["gpu_launches_per_step"] = B.forward_launches(shape)
+    return rec
+
+
 def backward_work(cfg, counts, grad_bytes):
     """Algorithmic FLOPs and bytes of one moe_backward call (the forward it
     recomputes, then the gradients): FLOPs = the forward's + per routed and
@@ -643,6 +679,12 @@ def run_ours(args, dist):
         torch.cuda.empty_cache()
         line["decode"] = decode_record(args, dist, dev, stream, peaks, peak_src)
         line["config"]["workload"] += "; decode record: " + line["decode"]["workload"]
+        if not args.no_other:
+            # the two other configs of the layer, each with its own weights
+            for other in ("skewed", "fp8"):
+                torch.cuda.empty_cache()
+                line[other] = workload_record(other, args, dist, dev, stream, peaks, peak_src)
+                line["config"]["workload"] += f"; {other} record: " + line[other]["workload"]
     if dist.rank == 0:
         print(json.dumps(line), flush=True)
 
