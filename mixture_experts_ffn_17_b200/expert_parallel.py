@@ -119,21 +119,30 @@ def forward(shape, rank: int, world: int, x, Wg, bias, w: EpWeights, y, ws, grou
 @dataclasses.dataclass
 class A2AWeights:
     """One rank's weights in the all-to-all flavour: routed experts
-    [e_lo, e_hi) and the whole shared expert (replicated)."""
+    [e_lo, e_hi) (e4m3 codes with their 128 x 128 block scales s1, s3, s2, or
+    bf16 with no scales) and the whole shared expert (replicated, bf16)."""
     W1: torch.Tensor
     W3: torch.Tensor
     W2: torch.Tensor
     W1s: Optional[torch.Tensor]
     W3s: Optional[torch.Tensor]
     W2s: Optional[torch.Tensor]
+    s1: Optional[torch.Tensor] = None
+    s3: Optional[torch.Tensor] = None
+    s2: Optional[torch.Tensor] = None
 
 
-def shard_weights_a2a(W1, W3, W2, W1s, W3s, W2s, rank: int, world: int) -> A2AWeights:
+def shard_weights_a2a(W1, W3, W2, W1s, W3s, W2s, rank: int, world: int, s1=None, s3=None, s2=None) -> A2AWeights:
+    """Rank `rank`'s routed experts (and, for e4m3 experts, their block scales
+    [E, ., .]) of the full layer's weights; the shared expert is kept whole."""
     E = W1.shape[0]
     if E % world or (E // world) % 32:
         raise ValueError(f"E={E} over {world} ranks: each rank's expert count must be a multiple of 32")
+    if (s1 is None) != (s3 is None) or (s1 is None) != (s2 is None):
+        raise ValueError("e4m3 experts need all three block-scale tensors")
     lo, hi = rank * (E // world), (rank + 1) * (E // world)
-    return A2AWeights(W1[lo:hi].contiguous(), W3[lo:hi].contiguous(), W2[lo:hi].contiguous(), W1s, W3s, W2s)
+    ex = lambda t: None if t is None else t[lo:hi].contiguous()
+    return A2AWeights(ex(W1), ex(W3), ex(W2), W1s, W3s, W2s, ex(s1), ex(s3), ex(s2))
 
 
 class A2ARank:
@@ -182,11 +191,11 @@ class A2ARank:
         B.ep_regroup_layout(self.world, self.El, recv_counts.contiguous(), offs, to_em, to_sm, stream=self.stream)
         x_loc = torch.empty(R, s.d, dtype=torch.bfloat16, device=dev)
         B.gather_rows(x_recv, to_em, x_loc, stream=self.stream)
-        shape_loc = B.make_shape(T=R, d=s.d, E=self.El, k=1, inter=s.inter, shared_inter=0)
+        shape_loc = B.make_shape(T=R, d=s.d, E=self.El, k=1, inter=s.inter, shared_inter=0, w_dtype=s.w_dtype)
         ws_loc = B.alloc_workspace(shape_loc, dev)
         Y_loc = torch.empty(R, s.d, dtype=torch.bfloat16, device=dev)
-        B.grouped_swiglu(shape_loc, x_loc, x_loc, offs, self.w.W1, self.w.W3, self.w.W2, None, None, None, None, None,
-                         None, Y_loc, None, ws_loc, stream=self.stream)
+        B.grouped_swiglu(shape_loc, x_loc, x_loc, offs, self.w.W1, self.w.W3, self.w.W2, self.w.s1, self.w.s3,
+                         self.w.s2, None, None, None, Y_loc, None, ws_loc, stream=self.stream)
         B.gather_rows(Y_loc, to_sm, y_send, stream=self.stream)
         return y_send
 
@@ -245,7 +254,7 @@ def forward_all_to_all(shape, rank: int, world: int, x, Wg, bias, w: A2AWeights,
         sh = B.make_shape(T=bounds[c + 1] - bounds[c], d=shape.d, E=shape.E, k=shape.k, inter=shape.inter,
                           shared_inter=shape.shared_inter, route=shape.route, n_group=shape.n_group,
                           topk_group=shape.topk_group, group_topn=shape.group_topn, route_scale=shape.route_scale,
-                          y_dtype=shape.y_dtype)
+                          w_dtype=shape.w_dtype, y_dtype=shape.y_dtype)
         parts.append((sl, A2ARank(sh, rank, world, w, x.device, stream)))
     sends, recvs, xs = [], [], []
     for sl, st in parts:

@@ -21,7 +21,7 @@ from mixture_experts_ffn_17_b200 import expert_parallel as ep
 from mixture_experts_ffn_17_b200 import workloads
 
 from gpu_util import oracle_full, route_with_exemptions, run_forward, to_device
-from parity import TOL_BF16, dec, max_rel_err, to_np
+from parity import TOL_BF16, TOL_FP8, dec, max_rel_err, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -36,17 +36,18 @@ def _rank_tokens(base, r):
     """Rank r's own batch: the base workload's weights, tokens from another seed."""
     w = workloads.make(base.cfg.replace(seed=base.cfg.seed + 101 * (r + 1)))
     return to_device(workloads.Workload(base.cfg, w.x, base.Wg, base.W1, base.W3, base.W2, base.W1s, base.W3s,
-                                        base.W2s, bias=base.bias))
+                                        base.W2s, bias=base.bias, s1=base.s1, s3=base.s3, s2=base.s2))
 
 
-def _check(base, world, mutate=None):
+def _check(base, world, mutate=None, tol=TOL_BF16):
     cfg = base.cfg
     ranks = [_rank_tokens(base, r) for r in range(world)]
     wdev = to_device(base)
     if mutate:
         mutate(wdev, ranks)
     shape = B.shape_of(cfg)
-    weights = [ep.shard_weights_a2a(wdev.W1, wdev.W3, wdev.W2, wdev.W1s, wdev.W3s, wdev.W2s, r, world)
+    weights = [ep.shard_weights_a2a(wdev.W1, wdev.W3, wdev.W2, wdev.W1s, wdev.W3s, wdev.W2s, r, world,
+                                    wdev.s1, wdev.s3, wdev.s2)
                for r in range(world)]
     ys = [torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda") for _ in range(world)]
     ep.simulate_all_to_all(shape, [w.x for w in ranks], wdev.Wg, wdev.bias, weights, ys)
@@ -62,7 +63,7 @@ def _check(base, world, mutate=None):
         if report:
             y_o, *_ = oracle_full(w, force_idx=merged)
         err = max_rel_err(to_np(ys[r]).astype(np.float64), y_o)
-        assert err <= TOL_BF16, (r, err)
+        assert err <= tol, (r, err)
         received.append(to_np(counts))
     return received
 
@@ -78,6 +79,34 @@ def test_all_to_all_group_routing_with_bias():
     # top-4 groups, x 2.5), bf16 experts, 2 ranks
     base = workloads.make_small("fp8", T=160, d=512, E=128, k=8, inter=256, shared_inter=256, fp8=False)
     _check(base, 2)
+
+
+def test_all_to_all_fp8_experts_group_routing():
+    # e4m3 routed experts with 128 x 128 block scales (each rank holds its
+    # experts' codes and scales), bf16 shared expert, group routing, 2 ranks
+    base = workloads.make_small("fp8", T=160, d=512, E=128, k=8, inter=256, shared_inter=256)
+    assert base.cfg.fp8 and base.s1 is not None
+    _check(base, 2, tol=TOL_FP8)
+
+
+def test_all_to_all_fp8_chunked_driver_on_a_one_rank_nccl_group():
+    import torch.distributed as dist
+    base = to_device(workloads.make_small("fp8", T=300, d=512, E=64, k=6, inter=256, shared_inter=256, n_group=8,
+                                          topk_group=3))
+    cfg = base.cfg
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        w = ep.shard_weights_a2a(base.W1, base.W3, base.W2, base.W1s, base.W3s, base.W2s, 0, 1,
+                                 base.s1, base.s3, base.s2)
+        y = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+        ep.forward_all_to_all(B.shape_of(cfg), 0, 1, base.x, base.Wg, base.bias, w, y, chunks=2)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    y1, *_ = run_forward(base)
+    rms = float(y1.double().pow(2).mean().sqrt())
+    assert float((y - y1).abs().max()) <= 1e-3 * rms
 
 
 def test_all_to_all_rank_without_rows_and_no_shared_expert():
