@@ -35,7 +35,9 @@
 //             swizzled N-major layout the MMA reads, through a 2-deep ring.
 //             The tensor cores take A and B of one type and the activations
 //             stay bf16, so the weights are widened in shared memory and the
-//             MMA runs kind::f16.
+//             MMA runs kind::f16.  When no tile can hold more than one half
+//             (batches of at most 128 tokens) the FP8 stages hold one A half,
+//             and the rings are 4 raw + 3 converted stages deep.
 //
 // Kernel A (SwiGLU):  N = 128 columns of W1 and the same 128 of W3 per tile,
 //                     one N=256 MMA per K step over [W1 | W3] (g and u side by
@@ -84,9 +86,21 @@ constexpr uint32_t kF8ConvBytes = 4 * kF8BoxBytes;      // 32 KB
 constexpr int kConvWarps = 8;
 constexpr int kSchedDepth = 4;  // tile indices the producer may publish ahead
 
+// FP8 weights at small batches (every routed tile one 128-row half, which
+// the host knows when T <= 128): a stage holds one A half and the raw codes,
+// so deeper rings fit -- each raw stage is held through the HBM latency and
+// the widening, each converted buffer until its MMAs complete, and at such
+// batches no MMA work hides them.  4 raw + 3 converted stages measured best
+// (of 5 + 2, 4 + 3, 3 + 4, 2 + 5 in the same 224 KB).
+constexpr int kF8NStages = 4;
+constexpr int kF8NConvStages = 3;
+constexpr uint32_t kF8NStageBytes = kF8ABytes + 2 * kF8RawBox;  // 32 KB
+
 static_assert(kStages * kStageBytes + 1024 + 256 <= 232448, "shared memory budget");
 static_assert(kF8Stages * kF8StageBytes + kF8ConvStages * kF8ConvBytes + 1024 + 256 <= 232448,
               "shared memory budget (FP8)");
+static_assert(kF8NStages * kF8NStageBytes + kF8NConvStages * kF8ConvBytes + 1024 + 256 <= 232448,
+              "shared memory budget (FP8, one-half stages)");
 
 enum class Mode { kSwiGLU, kDown };
 
@@ -101,9 +115,11 @@ struct Cfg<Mode::kDown> {
   static constexpr int BN = 256;  // columns of W2 per tile
 };
 
-template <bool F8>
+template <bool F8, bool N1 = false>
 constexpr size_t smem_bytes() {
-  return F8 ? 1024 + kF8Stages * kF8StageBytes + kF8ConvStages * kF8ConvBytes + 256
+  return F8 ? 1024 + (N1 ? kF8NStages * kF8NStageBytes + kF8NConvStages * kF8ConvBytes
+                         : kF8Stages * kF8StageBytes + kF8ConvStages * kF8ConvBytes) +
+                  256
             : 1024 + kStages * kStageBytes + 256;
 }
 
@@ -130,8 +146,9 @@ __device__ __forceinline__ int transposed_cols(const TileInfo& ti, int h) {
   return ((ti.rows - h * kTileM + 15) / 16) * 16;
 }
 
-// With FP8 weights the converted B buffer has its own layout and the narrow
-// half stays an M=64 MMA.
+// With FP8 weights the narrow half stays an M=64 MMA: the converted B buffer
+// has the bf16 boxes' layout, so the transposed MMA would apply, but it
+// measured slower there (the four FP8 epilogue warps take both row chunks).
 template <bool F8>
 __device__ __forceinline__ bool transposed_half(const TileInfo& ti, int h) {
   return !F8 && narrow_half(ti, h);
@@ -208,7 +225,19 @@ __device__ __forceinline__ uint2 e4m3x4_to_bf16x4(uint32_t q, float scale) {
       "cvt.f32.f16 %3, h1;\n\t}\n"
       : "=f"(a0), "=f"(a1), "=f"(b0), "=f"(b1)
       : "r"(h01), "r"(h23));
-  return make_uint2(ptx::pack_bf16x2(a0 * scale, a1 * scale), ptx::pack_bf16x2(b0 * scale, b1 * scale));
+  // the products of a pair in one packed multiply (the same rounding as two)
+  float p0, p1, p2, p3;
+  asm("{\n\t.reg .b64 a, b, s, pa, pb;\n\t"
+      "mov.b64 a, {%4, %5};\n\t"
+      "mov.b64 b, {%6, %7};\n\t"
+      "mov.b64 s, {%8, %8};\n\t"
+      "mul.rn.f32x2 pa, a, s;\n\t"
+      "mul.rn.f32x2 pb, b, s;\n\t"
+      "mov.b64 {%0, %1}, pa;\n\t"
+      "mov.b64 {%2, %3}, pb;\n\t}\n"
+      : "=f"(p0), "=f"(p1), "=f"(p2), "=f"(p3)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(scale));
+  return make_uint2(ptx::pack_bf16x2(p0, p1), ptx::pack_bf16x2(p2, p3));
 }
 
 // Epilogue warps: two per TMEM lane quarter with bf16 weights (each drains
@@ -223,21 +252,23 @@ constexpr int kernel_threads() {
   return 64 + 32 * epi_warps<F8>() + (F8 ? 32 * kConvWarps : 0);
 }
 
-template <Mode M, bool F8>
+template <Mode M, bool F8, bool N1 = false>
 __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
                         const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
                         const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s,
                         const GemmParams p) {
-  constexpr int S = F8 ? kF8Stages : kStages;
+  static_assert(!N1 || F8, "one-half stages are an FP8 layout");
+  constexpr int S = F8 ? (N1 ? kF8NStages : kF8Stages) : kStages;
   constexpr int BK = F8 ? kF8BK : kBK;
   constexpr uint32_t ABytes = F8 ? kF8ABytes : kABytes;
-  constexpr uint32_t StageBytes = F8 ? kF8StageBytes : kStageBytes;
+  constexpr uint32_t StageBytes = F8 ? (N1 ? kF8NStageBytes : kF8StageBytes) : kStageBytes;
+  constexpr int AHalves = N1 ? 1 : 2;  // A halves a stage has room for
   constexpr uint32_t BoxBytes = F8 ? kF8BoxBytes : kBoxBytes;
   constexpr uint32_t ASwz = F8 ? ptx::kSwizzle128B : kASwizzle;
   constexpr uint32_t ASBO = F8 ? 1024 : kASBO;
   constexpr int BN = Cfg<M>::BN;
-  constexpr int CS = kF8ConvStages;
+  constexpr int CS = N1 ? kF8NConvStages : kF8ConvStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stage0 = align_1024(smem_raw);
   uint8_t* conv0 = stage0 + S * StageBytes;  // FP8: converted bf16 B ring
@@ -349,6 +380,10 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         if (tile < 0) break;
         TileInfo ti;
         if (!tile_at(p, span, tile, BN, ti)) continue;
+        if (N1 && ti.halves == 2) {  // a launch with one-half stages got a longer tile: not computed
+          raise_status(p.status, abort_flag, kStatusBounds);
+          continue;
+        }
         // weights of a group with several row tiles (the shared expert, an
         // expert with many rows) are read again by each of them: keep them in
         // L2 (evict-normal) instead of streaming them (evict-first); evict-last
@@ -387,7 +422,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
           ptx::mbar_arrive_expect_tx(&full[s], bytes);
           ptx::tma_load_2d(st, mA, &full[s], kb * BK, arow, pol_a);
           if (ti.halves == 2) ptx::tma_load_2d(st + ABytes, mA, &full[s], kb * BK, arow + kTileM, pol_a);
-          uint8_t* sb = st + 2 * ABytes;
+          uint8_t* sb = st + AHalves * ABytes;
           if (F8) {
             // raw codes: box 0 = W1 (or W2 columns n0..n0+127), box 1 = W3 (or W2 n0+128..)
             if (M == Mode::kSwiGLU) {
@@ -429,7 +464,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         const int tile = next_tile(ns, ok);
         if (tile < 0) break;
         TileInfo ti;
-        if (!tile_at(p, span, tile, BN, ti)) continue;
+        if (!tile_at(p, span, tile, BN, ti) || (N1 && ti.halves == 2)) continue;
         const int nk = (ti.shared ? p.K_shared : p.K_routed) / BK;
         for (int h = 0; h < ti.halves; ++h) {
           const int sl = (ring.next + h) & 1;
@@ -499,7 +534,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
       const int tile = next_tile(ns, ok);
       if (tile < 0) break;
       TileInfo ti;
-      if (!tile_at(p, span, tile, BN, ti)) continue;
+      if (!tile_at(p, span, tile, BN, ti) || (N1 && ti.halves == 2)) continue;
       const int n0 = ti.nb * BN;
       for (int h = 0; h < ti.halves; ++h) {
         const int sl = (ring.next + h) & 1;
@@ -736,7 +771,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
       const int tile = next_tile(ns, ok);
       if (tile < 0) break;
       TileInfo ti;
-      if (!tile_at(p, span, tile, BN, ti)) continue;
+      if (!tile_at(p, span, tile, BN, ti) || (N1 && ti.halves == 2)) continue;
       const int nk = p.K_routed / BK;
       const int n0 = ti.nb * BN;
       const int ksb = p.K_routed / 128, nsb = p.N_routed / 128;  // scale blocks per expert
@@ -749,7 +784,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
           ok = false;
           break;
         }
-        const uint8_t* raw = stage0 + s * kF8StageBytes + 2 * kF8ABytes;
+        const uint8_t* raw = stage0 + s * StageBytes + AHalves * kF8ABytes;
         uint8_t* conv = conv0 + c * kF8ConvBytes;
         const int kblk = (kb * BK) / 128;
         const int64_t sbase = ((int64_t)(ti.group - p.group_base) * ksb + kblk) * nsb;
@@ -1405,17 +1440,17 @@ cudaError_t launch_pair(const CUtensorMap& a_r, const CUtensorMap& a_s, const CU
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
-template <Mode M, bool F8>
+template <Mode M, bool F8, bool N1 = false>
 cudaError_t launch(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtensorMap& b_r, const CUtensorMap& b_s,
                    const CUtensorMap& c_r, const CUtensorMap& c_s, const GemmParams& p, int grid,
                    cudaStream_t stream) {
-  const size_t smem = smem_bytes<F8>();
+  const size_t smem = smem_bytes<F8, N1>();
   cudaError_t err =
-      cudaFuncSetAttribute(grouped_gemm_kernel<M, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(grouped_gemm_kernel<M, F8, N1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   if (grid <= 0) return cudaSuccess;
-  cudaError_t e = launch_chained(grouped_gemm_kernel<M, F8>, grid, dim3(kernel_threads<F8>()), smem, stream, a_r, a_s,
-                                 b_r, b_s, c_r, c_s, p);
+  cudaError_t e = launch_chained(grouped_gemm_kernel<M, F8, N1>, grid, dim3(kernel_threads<F8>()), smem, stream,
+                                 a_r, a_s, b_r, b_s, c_r, c_s, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1460,13 +1495,15 @@ cudaError_t launch_grouped_down_pair_fp8(const CUtensorMap& tmA, const CUtensorM
 
 cudaError_t launch_grouped_swiglu_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,
                                       const CUtensorMap& tmW3_r, const GemmParams& p, int grid,
-                                      cudaStream_t stream) {
-  return launch<Mode::kSwiGLU, true>(tmA_r, tmA_r, tmW1_r, tmW1_r, tmW3_r, tmW3_r, p, grid, stream);
+                                      cudaStream_t stream, bool one_half) {
+  return one_half ? launch<Mode::kSwiGLU, true, true>(tmA_r, tmA_r, tmW1_r, tmW1_r, tmW3_r, tmW3_r, p, grid, stream)
+                  : launch<Mode::kSwiGLU, true>(tmA_r, tmA_r, tmW1_r, tmW1_r, tmW3_r, tmW3_r, p, grid, stream);
 }
 
 cudaError_t launch_grouped_down_fp8(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const GemmParams& p, int grid,
-                                    cudaStream_t stream) {
-  return launch<Mode::kDown, true>(tmA, tmA, tmW2_r, tmW2_r, tmW2_r, tmW2_r, p, grid, stream);
+                                    cudaStream_t stream, bool one_half) {
+  return one_half ? launch<Mode::kDown, true, true>(tmA, tmA, tmW2_r, tmW2_r, tmW2_r, tmW2_r, p, grid, stream)
+                  : launch<Mode::kDown, true>(tmA, tmA, tmW2_r, tmW2_r, tmW2_r, tmW2_r, p, grid, stream);
 }
 
 }  // namespace moe

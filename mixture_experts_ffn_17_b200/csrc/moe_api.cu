@@ -180,6 +180,12 @@ int num_sms() {
 // measured no faster than the one-CTA path (T=8192 layer: 9.53 vs 9.61 ms), so
 // they run only when forced.  MOE_PAIR_TILES=1 / 0 in the environment forces
 // pairs on / off.
+// FP8 batches whose segments all fit one 128-row half (T <= 128) launch the
+// FP8 kernels with one-A-half stages and deeper rings (0: the general layout)
+#ifndef MOE_F8_ONE_HALF_STAGES
+#define MOE_F8_ONE_HALF_STAGES 1
+#endif
+
 bool use_pair_tiles(const moe_shape& s) {
   const char* v = std::getenv("MOE_PAIR_TILES");
   if (v && v[0] == '1') return true;
@@ -212,8 +218,11 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
                        const int32_t* offsets, const void* W1, const void* W3, const void* W2, const float* s1,
                        const float* s3, const float* s2, const void* W1s, const void* W3s, const void* W2s,
                        void* Y_perm, float* Y_shared, uint32_t* status, cudaStream_t st, const Shard& shard,
-                       const cudaEvent_t* ev = nullptr) {
+                       const cudaEvent_t* ev = nullptr, bool short_segments = false) {
   const bool f8 = s.w_dtype == MOE_E4M3;
+  // FP8 launches with one-half stages and a deeper ring when no segment can
+  // exceed one 128-row half (see launch_grouped_swiglu_fp8)
+  const bool f8_one_half = f8 && short_segments && MOE_F8_ONE_HALF_STAGES;
   const bool sh = s.shared_inter > 0;
   const int64_t Tk = s.T * s.k;
   int4* tiles = at<int4>(ws, L.tiles);
@@ -281,7 +290,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
       qp.ntiles = ntiles + 2;
       MOE_CUDA(launch_grouped_swiglu_pair_fp8(a8_r, w18_r, w38_r, qp, sms, st));
     }
-    MOE_CUDA(launch_grouped_swiglu_fp8(a8_r, w18_r, w38_r, q, grid1, st));
+    MOE_CUDA(launch_grouped_swiglu_fp8(a8_r, w18_r, w38_r, q, grid1, st, f8_one_half));
     if (sh) {
       q = p1;
       q.tile_set = kTilesShared;
@@ -345,7 +354,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
       qp.ntiles = ntiles + 2;
       MOE_CUDA(launch_grouped_down_pair_fp8(h8_map, w28_r, qp, sms, st));
     }
-    MOE_CUDA(launch_grouped_down_fp8(h8_map, w28_r, q, grid2, st));
+    MOE_CUDA(launch_grouped_down_fp8(h8_map, w28_r, q, grid2, st, f8_one_half));
     if (sh) {
       q = p2;
       q.tile_set = kTilesShared;
@@ -426,8 +435,9 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   MOE_CUDA(launch_permute(idx, s.T, s.k, s.E, at<int32_t>(ws, L.hist), at<int32_t>(ws, L.base), counts, offsets,
                           perm, row_of, status, st));
   MOE_CUDA(launch_scatter_rows(x, row_of, s.T, s.k, s.d, x_perm, num_sms(), st, offsets, shard.e_lo, shard.e_hi));
+  // the router picks k distinct experts per token, so no segment exceeds T rows
   r = run_experts(sl, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared, status, st,
-                  shard, ev ? ev + 2 : nullptr);
+                  shard, ev ? ev + 2 : nullptr, s.T <= kTileM);
   if (r != MOE_OK) return r;
   MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16, st,
                           whole ? nullptr : offsets, whole ? nullptr : &shard));
@@ -1012,8 +1022,9 @@ moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const void*
   uint32_t* status = at<uint32_t>(ws, L.status);
   MOE_CUDA(cudaMemsetAsync(status, 0, 4, st));
   if (s.T == 0) return MOE_OK;
+  // caller-given offsets: segments are bounded only by the T*k rows
   return run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm,
-                     sh ? Y_shared : nullptr, status, st, whole_layer(s));
+                     sh ? Y_shared : nullptr, status, st, whole_layer(s), nullptr, s.T * s.k <= kTileM);
 }
 
 moe_status moe_combine(const moe_shape* shape, const void* Y_perm, const float* Y_shared, const int32_t* row_of,

@@ -156,12 +156,15 @@ cudaError_t launch_grouped_down_pair_fp8(const CUtensorMap& tmA, const CUtensorM
 cudaError_t launch_grouped_down(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
                                 const GemmParams& p, int grid, cudaStream_t stream);
 // FP8 (e4m3 + 128x128 block scales) routed experts; the tensor maps of W are
-// uint8 [E, K, N] with [1 x 64 x 128] boxes and no swizzle.
+// uint8 [E, K, N] with [1 x 64 x 128] boxes and no swizzle.  one_half: every
+// routed tile holds at most 128 rows (the caller knows it, e.g. T <= 128 with
+// distinct experts per token), so the kernel's stages hold one A half and its
+// ring is deeper; a longer tile is then skipped and raises kStatusBounds.
 cudaError_t launch_grouped_swiglu_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,
                                       const CUtensorMap& tmW3_r, const GemmParams& p, int grid,
-                                      cudaStream_t stream);
+                                      cudaStream_t stream, bool one_half);
 cudaError_t launch_grouped_down_fp8(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const GemmParams& p, int grid,
-                                    cudaStream_t stream);
+                                    cudaStream_t stream, bool one_half);
 
 // ep.cu: expert-major order of rows received from n_src ranks (source-major,
 // each source's rows in expert order); n_src * E_local <= 1024.

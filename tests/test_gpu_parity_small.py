@@ -393,6 +393,23 @@ def test_forward_fp8_no_shared_expert():
     _check_forward(_fp8(T=300, shared_inter=0), tol=TOL_FP8)
 
 
+def test_forward_fp8_small_batch():
+    # T <= 128: no expert segment can pass one 128-row half, so the FP8
+    # kernels run with one-A-half stages and a deeper ring
+    _check_forward(_fp8(T=100), tol=TOL_FP8)
+    _check_forward(_fp8(T=1, shared_inter=0), tol=TOL_FP8)
+
+
+def test_grouped_swiglu_fp8_short_segments():
+    # T*k <= 128 rows through moe_grouped_swiglu (one-half stages): segments
+    # of 65 (past the 64-row narrow half), 1, 16, 17, 0 and 21 rows
+    w = _fp8(T=120, k=1, E=32, n_group=4, topk_group=2, d=512, inter=256)
+    counts = [65, 1, 16, 17, 0, 21]
+    idx = np.repeat(np.arange(len(counts), dtype=np.int32), counts)
+    np.random.default_rng(7).shuffle(idx)
+    _experts_case(w, idx[:, None])
+
+
 # --------------------------------------------------- device-limited routing
 def test_router_limited_matches_oracle():
     w = _medium()

@@ -93,6 +93,14 @@ def test_v3_fp8_group_routing_sampled():
     assert (c > 0).sum() > 200
 
 
+def test_v3_fp8_decode_batch_all_tokens():
+    # e4m3 experts and group routing at a decode batch (T=64): segments of a
+    # few rows, each widening whole weight tiles; every token against the oracle
+    w = workloads.make(workloads.CONFIGS["fp8"].replace(T=64), device="cuda")
+    c, _ = _check_workload("fp8 decode batch", w, None, tol=TOL_FP8)
+    assert c.sum() == 64 * 8 and c.max() <= 64
+
+
 # The largest batches the library takes are bounded by T*k + T < 2**31 rows,
 # not by the V3 configs: a narrow layer (d=256, 64 experts, inter 128) at
 # T = 200,000 tokens (1.6M routed rows, 12x the skewed batch) runs the
