@@ -775,9 +775,27 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
       const int nk = p.K_routed / BK;
       const int n0 = ti.nb * BN;
       const int ksb = p.K_routed / 128, nsb = p.N_routed / 128;  // scale blocks per expert
+      // the block scales of K step kb (one 128 x 128 block per box)
+      auto load_scales = [&](int kb, float* sc) {
+        const int kblk = (kb * BK) / 128;
+        const int64_t sbase = ((int64_t)(ti.group - p.group_base) * ksb + kblk) * nsb;
+        if (M == Mode::kSwiGLU) {
+          sc[0] = p.scale_b[sbase + n0 / 128];
+          sc[1] = p.scale_c[sbase + n0 / 128];
+        } else {
+          sc[0] = p.scale_b[sbase + n0 / 128];
+          sc[1] = n0 + 128 < p.N_routed ? p.scale_b[sbase + n0 / 128 + 1] : 0.0f;  // past the last column
+        }
+      };
+      float sc_next[2];
+      load_scales(0, sc_next);
       for (int kb = 0; kb < nk; ++kb, ++kg) {
         const int s = kg % S;
         const int c = kg % CS;
+        // this step's scales were loaded one step ahead; the next step's load
+        // is issued before the waits, so its latency overlaps them
+        const float sc[2] = {sc_next[0], sc_next[1]};
+        if (kb + 1 < nk) load_scales(kb + 1, sc_next);
         if (!ptx::wait_bounded(&full[s], (kg / S) & 1, abort_flag) ||
             !ptx::wait_bounded(&cempty[c], ((kg / CS) & 1) ^ 1, abort_flag)) {
           raise_status(p.status, abort_flag, kStatusTimeout);
@@ -786,16 +804,6 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         }
         const uint8_t* raw = stage0 + s * StageBytes + AHalves * kF8ABytes;
         uint8_t* conv = conv0 + c * kF8ConvBytes;
-        const int kblk = (kb * BK) / 128;
-        const int64_t sbase = ((int64_t)(ti.group - p.group_base) * ksb + kblk) * nsb;
-        float sc[2];
-        if (M == Mode::kSwiGLU) {
-          sc[0] = p.scale_b[sbase + n0 / 128];
-          sc[1] = p.scale_c[sbase + n0 / 128];
-        } else {
-          sc[0] = p.scale_b[sbase + n0 / 128];
-          sc[1] = n0 + 128 < p.N_routed ? p.scale_b[sbase + n0 / 128 + 1] : 0.0f;  // past the last column
-        }
 #pragma unroll
         for (int i = 0; i < 128 / (4 * kConvWarps); ++i) {
           const int rr = (cw * (128 / kConvWarps)) + i * 4 + sub_row;  // 0..127
