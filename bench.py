@@ -492,7 +492,41 @@ def workload_record(name, args, dist, dev, stream, peaks, peak_src):
     if rc != B.MOE_OK:
         raise B.MoeError(rc, f"{name}: device status after the timed steps (raw {raw})")
     rec["gpu_launches_per_step"] = B.forward_launches(shape)
+    if cfg.fp8:
+        del ws
+        rec["decode_batch"] = decode_batch_record(B, cfg, w, 64, args, dist, dev, stream, peaks, peak_src)
     return rec
+
+
+def decode_batch_record(B, cfg, w, T, args, dist, dev, stream, peaks, peak_src):
+    """The same weights at a decode batch (the workload's first T tokens),
+    burst only: the touched experts' weight bytes over the step time against
+    HBM, as the decode record measures the bf16 layer."""
+    cs = cfg.replace(T=T)
+    shape = B.shape_of(cs, B.MOE_F32)
+    ws = B.alloc_workspace(shape, dev)
+    x = w.x[:T].contiguous()
+    y = torch.empty(T, cs.d, dtype=torch.float32, device=dev)
+    counts = torch.empty(cs.E, dtype=torch.int32, device=dev)
+    fwd_args = (shape, x, w.Wg, w.bias, w.W1, w.W3, w.W2, w.s1, w.s3, w.s2, w.W1s, w.W3s, w.W2s, y, ws)
+    for _ in range(max(args.warmup, 3)):
+        B.forward(*fwd_args, counts=counts)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"{cs.name} T={T}: device status after warm-up (raw {raw})")
+    K = max(args.steps, 50)
+    ms, clocks = time_loop(lambda i: B.forward(*fwd_args, counts=counts), K, stream, dev, dist)
+    c = counts.cpu().numpy()
+    wbytes = touched_weight_bytes(cs, c)
+    rc, raw = B.check_device_status(ws)
+    if rc != B.MOE_OK:
+        raise B.MoeError(rc, f"{cs.name} T={T}: device status after the timed steps (raw {raw})")
+    return {"workload": config_of(cs, args)["workload"], "steps": K, "ms_per_step": ms,
+            "tokens_per_s": dist.world * T / (ms / 1e3), "touched_experts": touched_experts(c),
+            "touched_weight_bytes": wbytes, "touched_weight_gbs": wbytes / (ms / 1e3) / 1e9,
+            "hbm_frac": wbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "hbm_frac_datasheet": wbytes / (ms / 1e3) / 1e9 / DATASHEET_PEAKS["hbm_gbs"],
+            "roofline_layer": layer_roofline(cs, c, ms, peaks, peak_src), "clocks": clocks}
 
 
 def backward_work(cfg, counts, grad_bytes):
