@@ -37,7 +37,8 @@
 //             stay bf16, so the weights are widened in shared memory and the
 //             MMA runs kind::f16.  When no tile can hold more than one half
 //             (batches of at most 128 tokens) the FP8 stages hold one A half,
-//             and the rings are 4 raw + 3 converted stages deep.
+//             and the rings are 4 raw + 3 converted stages deep; at most 64
+//             rows (64 tokens): a 64-row A box and 5 + 3 stages.
 //
 // Kernel A (SwiGLU):  N = 128 columns of W1 and the same 128 of W3 per tile,
 //                     one N=256 MMA per K step over [W1 | W3] (g and u side by
@@ -95,12 +96,23 @@ constexpr int kSchedDepth = 4;  // tile indices the producer may publish ahead
 constexpr int kF8NStages = 4;
 constexpr int kF8NConvStages = 3;
 constexpr uint32_t kF8NStageBytes = kF8ABytes + 2 * kF8RawBox;  // 32 KB
+// ... and when no tile can hold more than 64 rows (batches of at most 64
+// tokens) the A box is 64 rows, the stage 24 KB, and the ring 5 deep
+#ifndef MOE_F8N2_STAGES
+#define MOE_F8N2_STAGES 5
+#endif
+constexpr int kF8N2Stages = MOE_F8N2_STAGES;
+constexpr uint32_t kF8N2ABytes = kF8ABytes / 2;
+constexpr uint32_t kF8N2StageBytes = kF8N2ABytes + 2 * kF8RawBox;  // 24 KB
 
 static_assert(kStages * kStageBytes + 1024 + 256 <= 232448, "shared memory budget");
 static_assert(kF8Stages * kF8StageBytes + kF8ConvStages * kF8ConvBytes + 1024 + 256 <= 232448,
               "shared memory budget (FP8)");
 static_assert(kF8NStages * kF8NStageBytes + kF8NConvStages * kF8ConvBytes + 1024 + 256 <= 232448,
               "shared memory budget (FP8, one-half stages)");
+static_assert(kF8N2Stages * kF8N2StageBytes + kF8NConvStages * kF8ConvBytes + 1024 + 256 <= 232448,
+              "shared memory budget (FP8, 64-row stages)");
+static_assert(kF8N2StageBytes % 1024 == 0, "64-row stages keep the 1024-byte alignment of the A boxes");
 
 enum class Mode { kSwiGLU, kDown };
 
@@ -115,9 +127,12 @@ struct Cfg<Mode::kDown> {
   static constexpr int BN = 256;  // columns of W2 per tile
 };
 
-template <bool F8, bool N1 = false>
+// N1 (FP8 only): 0 the general layout, 1 stages of one 128-row A half,
+// 2 stages of one 64-row A box
+template <bool F8, int N1 = 0>
 constexpr size_t smem_bytes() {
-  return F8 ? 1024 + (N1 ? kF8NStages * kF8NStageBytes + kF8NConvStages * kF8ConvBytes
+  return F8 ? 1024 + (N1 == 2 ? kF8N2Stages * kF8N2StageBytes + kF8NConvStages * kF8ConvBytes
+                     : N1 ? kF8NStages * kF8NStageBytes + kF8NConvStages * kF8ConvBytes
                          : kF8Stages * kF8StageBytes + kF8ConvStages * kF8ConvBytes) +
                   256
             : 1024 + kStages * kStageBytes + 256;
@@ -252,17 +267,18 @@ constexpr int kernel_threads() {
   return 64 + 32 * epi_warps<F8>() + (F8 ? 32 * kConvWarps : 0);
 }
 
-template <Mode M, bool F8, bool N1 = false>
+template <Mode M, bool F8, int N1 = 0>
 __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
                         const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
                         const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s,
                         const GemmParams p) {
   static_assert(!N1 || F8, "one-half stages are an FP8 layout");
-  constexpr int S = F8 ? (N1 ? kF8NStages : kF8Stages) : kStages;
+  constexpr int S = F8 ? (N1 == 2 ? kF8N2Stages : N1 ? kF8NStages : kF8Stages) : kStages;
   constexpr int BK = F8 ? kF8BK : kBK;
-  constexpr uint32_t ABytes = F8 ? kF8ABytes : kABytes;
-  constexpr uint32_t StageBytes = F8 ? (N1 ? kF8NStageBytes : kF8StageBytes) : kStageBytes;
+  constexpr uint32_t ABytes = F8 ? (N1 == 2 ? kF8N2ABytes : kF8ABytes) : kABytes;
+  constexpr uint32_t StageBytes =
+      F8 ? (N1 == 2 ? kF8N2StageBytes : N1 ? kF8NStageBytes : kF8StageBytes) : kStageBytes;
   constexpr int AHalves = N1 ? 1 : 2;  // A halves a stage has room for
   constexpr uint32_t BoxBytes = F8 ? kF8BoxBytes : kBoxBytes;
   constexpr uint32_t ASwz = F8 ? ptx::kSwizzle128B : kASwizzle;
@@ -380,7 +396,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         if (tile < 0) break;
         TileInfo ti;
         if (!tile_at(p, span, tile, BN, ti)) continue;
-        if (N1 && ti.halves == 2) {  // a launch with one-half stages got a longer tile: not computed
+        if (N1 && ti.rows > (N1 == 2 ? kTileM / 2 : kTileM)) {  // longer than the stages hold: not computed
           raise_status(p.status, abort_flag, kStatusBounds);
           continue;
         }
@@ -464,7 +480,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
         const int tile = next_tile(ns, ok);
         if (tile < 0) break;
         TileInfo ti;
-        if (!tile_at(p, span, tile, BN, ti) || (N1 && ti.halves == 2)) continue;
+        if (!tile_at(p, span, tile, BN, ti) || (N1 && ti.rows > (N1 == 2 ? kTileM / 2 : kTileM))) continue;
         const int nk = (ti.shared ? p.K_shared : p.K_routed) / BK;
         for (int h = 0; h < ti.halves; ++h) {
           const int sl = (ring.next + h) & 1;
@@ -534,7 +550,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
       const int tile = next_tile(ns, ok);
       if (tile < 0) break;
       TileInfo ti;
-      if (!tile_at(p, span, tile, BN, ti) || (N1 && ti.halves == 2)) continue;
+      if (!tile_at(p, span, tile, BN, ti) || (N1 && ti.rows > (N1 == 2 ? kTileM / 2 : kTileM))) continue;
       const int n0 = ti.nb * BN;
       for (int h = 0; h < ti.halves; ++h) {
         const int sl = (ring.next + h) & 1;
@@ -771,7 +787,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
       const int tile = next_tile(ns, ok);
       if (tile < 0) break;
       TileInfo ti;
-      if (!tile_at(p, span, tile, BN, ti) || (N1 && ti.halves == 2)) continue;
+      if (!tile_at(p, span, tile, BN, ti) || (N1 && ti.rows > (N1 == 2 ? kTileM / 2 : kTileM))) continue;
       const int nk = p.K_routed / BK;
       const int n0 = ti.nb * BN;
       const int ksb = p.K_routed / 128, nsb = p.N_routed / 128;  // scale blocks per expert
@@ -802,7 +818,7 @@ __global__ void __launch_bounds__(kernel_threads<F8>(), 1)
           ok = false;
           break;
         }
-        const uint8_t* raw = stage0 + s * StageBytes + AHalves * kF8ABytes;
+        const uint8_t* raw = stage0 + s * StageBytes + AHalves * ABytes;
         uint8_t* conv = conv0 + c * kF8ConvBytes;
 #pragma unroll
         for (int i = 0; i < 128 / (4 * kConvWarps); ++i) {
@@ -1448,7 +1464,7 @@ cudaError_t launch_pair(const CUtensorMap& a_r, const CUtensorMap& a_s, const CU
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
-template <Mode M, bool F8, bool N1 = false>
+template <Mode M, bool F8, int N1 = 0>
 cudaError_t launch(const CUtensorMap& a_r, const CUtensorMap& a_s, const CUtensorMap& b_r, const CUtensorMap& b_s,
                    const CUtensorMap& c_r, const CUtensorMap& c_s, const GemmParams& p, int grid,
                    cudaStream_t stream) {
@@ -1503,15 +1519,19 @@ cudaError_t launch_grouped_down_pair_fp8(const CUtensorMap& tmA, const CUtensorM
 
 cudaError_t launch_grouped_swiglu_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,
                                       const CUtensorMap& tmW3_r, const GemmParams& p, int grid,
-                                      cudaStream_t stream, bool one_half) {
-  return one_half ? launch<Mode::kSwiGLU, true, true>(tmA_r, tmA_r, tmW1_r, tmW1_r, tmW3_r, tmW3_r, p, grid, stream)
-                  : launch<Mode::kSwiGLU, true>(tmA_r, tmA_r, tmW1_r, tmW1_r, tmW3_r, tmW3_r, p, grid, stream);
+                                      cudaStream_t stream, int short_rows) {
+  if (short_rows == 2)
+    return launch<Mode::kSwiGLU, true, 2>(tmA_r, tmA_r, tmW1_r, tmW1_r, tmW3_r, tmW3_r, p, grid, stream);
+  if (short_rows == 1)
+    return launch<Mode::kSwiGLU, true, 1>(tmA_r, tmA_r, tmW1_r, tmW1_r, tmW3_r, tmW3_r, p, grid, stream);
+  return launch<Mode::kSwiGLU, true>(tmA_r, tmA_r, tmW1_r, tmW1_r, tmW3_r, tmW3_r, p, grid, stream);
 }
 
 cudaError_t launch_grouped_down_fp8(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const GemmParams& p, int grid,
-                                    cudaStream_t stream, bool one_half) {
-  return one_half ? launch<Mode::kDown, true, true>(tmA, tmA, tmW2_r, tmW2_r, tmW2_r, tmW2_r, p, grid, stream)
-                  : launch<Mode::kDown, true>(tmA, tmA, tmW2_r, tmW2_r, tmW2_r, tmW2_r, p, grid, stream);
+                                    cudaStream_t stream, int short_rows) {
+  if (short_rows == 2) return launch<Mode::kDown, true, 2>(tmA, tmA, tmW2_r, tmW2_r, tmW2_r, tmW2_r, p, grid, stream);
+  if (short_rows == 1) return launch<Mode::kDown, true, 1>(tmA, tmA, tmW2_r, tmW2_r, tmW2_r, tmW2_r, p, grid, stream);
+  return launch<Mode::kDown, true>(tmA, tmA, tmW2_r, tmW2_r, tmW2_r, tmW2_r, p, grid, stream);
 }
 
 }  // namespace moe

@@ -181,9 +181,11 @@ int num_sms() {
 // they run only when forced.  MOE_PAIR_TILES=1 / 0 in the environment forces
 // pairs on / off.
 // FP8 batches whose segments all fit one 128-row half (T <= 128) launch the
-// FP8 kernels with one-A-half stages and deeper rings (0: the general layout)
+// FP8 kernels with one-A-half stages and deeper rings; with 2, those whose
+// segments fit 64 rows (T <= 64) use 64-row A boxes and deeper rings still
+// (1: only the first; 0: the general layout)
 #ifndef MOE_F8_ONE_HALF_STAGES
-#define MOE_F8_ONE_HALF_STAGES 1
+#define MOE_F8_ONE_HALF_STAGES 2
 #endif
 
 bool use_pair_tiles(const moe_shape& s) {
@@ -218,11 +220,16 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
                        const int32_t* offsets, const void* W1, const void* W3, const void* W2, const float* s1,
                        const float* s3, const float* s2, const void* W1s, const void* W3s, const void* W2s,
                        void* Y_perm, float* Y_shared, uint32_t* status, cudaStream_t st, const Shard& shard,
-                       const cudaEvent_t* ev = nullptr, bool short_segments = false) {
+                       const cudaEvent_t* ev = nullptr, int64_t max_segment = -1) {
   const bool f8 = s.w_dtype == MOE_E4M3;
-  // FP8 launches with one-half stages and a deeper ring when no segment can
-  // exceed one 128-row half (see launch_grouped_swiglu_fp8)
-  const bool f8_one_half = f8 && short_segments && MOE_F8_ONE_HALF_STAGES;
+  // FP8 launches with short stages and deeper rings when no segment can
+  // exceed one 128-row half, or 64 rows (see launch_grouped_swiglu_fp8);
+  // max_segment < 0: unknown
+  const int f8_short = !f8 || max_segment < 0 || !MOE_F8_ONE_HALF_STAGES || use_pair_tiles(s) ? 0
+                       : max_segment <= kTileM / 2 && MOE_F8_ONE_HALF_STAGES >= 2 ? 2
+                       : max_segment <= kTileM                                      ? 1
+                                                                                    : 0;
+  const int a8_rows = f8_short == 2 ? kTileM / 2 : kTileM;  // rows of the FP8 launches' A boxes
   const bool sh = s.shared_inter > 0;
   const int64_t Tk = s.T * s.k;
   int4* tiles = at<int4>(ws, L.tiles);
@@ -242,7 +249,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
     return MOE_ERR_CUDA;
   if (f8) {
     // FP8 launches use a 64-deep K stage whatever the bf16 kernel's depth
-    if (!map_2d(&a8_r, x_perm, s.d, Tk, 64, kTileM) || !map_3d_u8(&w18_r, W1, s.inter, s.d, E_w) ||
+    if (!map_2d(&a8_r, x_perm, s.d, Tk, 64, a8_rows) || !map_3d_u8(&w18_r, W1, s.inter, s.d, E_w) ||
         !map_3d_u8(&w38_r, W3, s.inter, s.d, E_w))
       return MOE_ERR_CUDA;
     w1_r = a_r;  // placeholders: the bf16 launch below only walks the shared expert's tiles
@@ -290,7 +297,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
       qp.ntiles = ntiles + 2;
       MOE_CUDA(launch_grouped_swiglu_pair_fp8(a8_r, w18_r, w38_r, qp, sms, st));
     }
-    MOE_CUDA(launch_grouped_swiglu_fp8(a8_r, w18_r, w38_r, q, grid1, st, f8_one_half));
+    MOE_CUDA(launch_grouped_swiglu_fp8(a8_r, w18_r, w38_r, q, grid1, st, f8_short));
     if (sh) {
       q = p1;
       q.tile_set = kTilesShared;
@@ -318,7 +325,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
   CUtensorMap h_map, w2_r, w2_s, h8_map, w28_r;
   if (!map_2d(&h_map, H, L.Hld, L.Hrows, kGemmBK, kTileM)) return MOE_ERR_CUDA;
   if (f8) {
-    if (!map_2d(&h8_map, H, L.Hld, L.Hrows, 64, kTileM) || !map_3d_u8(&w28_r, W2, s.d, s.inter, E_w))
+    if (!map_2d(&h8_map, H, L.Hld, L.Hrows, 64, a8_rows) || !map_3d_u8(&w28_r, W2, s.d, s.inter, E_w))
       return MOE_ERR_CUDA;
     w2_r = h_map;  // placeholder: the bf16 launch below only walks the shared expert's tiles
   } else if (!map_3d(&w2_r, W2, s.d, s.inter, E_w, kGemmBK)) {
@@ -354,7 +361,7 @@ moe_status run_experts(const moe_shape& s, const Layout& L, void* ws, const void
       qp.ntiles = ntiles + 2;
       MOE_CUDA(launch_grouped_down_pair_fp8(h8_map, w28_r, qp, sms, st));
     }
-    MOE_CUDA(launch_grouped_down_fp8(h8_map, w28_r, q, grid2, st, f8_one_half));
+    MOE_CUDA(launch_grouped_down_fp8(h8_map, w28_r, q, grid2, st, f8_short));
     if (sh) {
       q = p2;
       q.tile_set = kTilesShared;
@@ -437,7 +444,7 @@ moe_status forward_impl(const moe_shape* shape, const void* x, const void* Wg, c
   MOE_CUDA(launch_scatter_rows(x, row_of, s.T, s.k, s.d, x_perm, num_sms(), st, offsets, shard.e_lo, shard.e_hi));
   // the router picks k distinct experts per token, so no segment exceeds T rows
   r = run_experts(sl, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm, Y_shared, status, st,
-                  shard, ev ? ev + 2 : nullptr, s.T <= kTileM);
+                  shard, ev ? ev + 2 : nullptr, s.T);
   if (r != MOE_OK) return r;
   MOE_CUDA(launch_combine(Y_perm, Y_shared, row_of, w, s.T, s.k, s.d, y, s.y_dtype == MOE_BF16, st,
                           whole ? nullptr : offsets, whole ? nullptr : &shard));
@@ -1024,7 +1031,7 @@ moe_status moe_grouped_swiglu(const moe_shape* shape, const void* x, const void*
   if (s.T == 0) return MOE_OK;
   // caller-given offsets: segments are bounded only by the T*k rows
   return run_experts(s, L, ws, x, x_perm, offsets, W1, W3, W2, s1, s3, s2, W1s, W3s, W2s, Y_perm,
-                     sh ? Y_shared : nullptr, status, st, whole_layer(s), nullptr, s.T * s.k <= kTileM);
+                     sh ? Y_shared : nullptr, status, st, whole_layer(s), nullptr, s.T * s.k);
 }
 
 moe_status moe_combine(const moe_shape* shape, const void* Y_perm, const float* Y_shared, const int32_t* row_of,

@@ -156,15 +156,17 @@ cudaError_t launch_grouped_down_pair_fp8(const CUtensorMap& tmA, const CUtensorM
 cudaError_t launch_grouped_down(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const CUtensorMap& tmW2_s,
                                 const GemmParams& p, int grid, cudaStream_t stream);
 // FP8 (e4m3 + 128x128 block scales) routed experts; the tensor maps of W are
-// uint8 [E, K, N] with [1 x 64 x 128] boxes and no swizzle.  one_half: every
-// routed tile holds at most 128 rows (the caller knows it, e.g. T <= 128 with
-// distinct experts per token), so the kernel's stages hold one A half and its
-// ring is deeper; a longer tile is then skipped and raises kStatusBounds.
+// uint8 [E, K, N] with [1 x 64 x 128] boxes and no swizzle.  short_rows: 1
+// when every routed tile holds at most 128 rows, 2 when at most 64 (the caller
+// knows it, e.g. T <= 128 or 64 with distinct experts per token): the kernel's
+// stages then hold one 128-row A half, or one 64-row A box (tmA's boxes must
+// be 64 rows then), and its rings are deeper; a longer tile is skipped and
+// raises kStatusBounds.  0: the general layout.
 cudaError_t launch_grouped_swiglu_fp8(const CUtensorMap& tmA_r, const CUtensorMap& tmW1_r,
                                       const CUtensorMap& tmW3_r, const GemmParams& p, int grid,
-                                      cudaStream_t stream, bool one_half);
+                                      cudaStream_t stream, int short_rows);
 cudaError_t launch_grouped_down_fp8(const CUtensorMap& tmA, const CUtensorMap& tmW2_r, const GemmParams& p, int grid,
-                                    cudaStream_t stream, bool one_half);
+                                    cudaStream_t stream, int short_rows);
 
 // ep.cu: expert-major order of rows received from n_src ranks (source-major,
 // each source's rows in expert order); n_src * E_local <= 1024.

@@ -408,6 +408,13 @@ def test_grouped_swiglu_fp8_short_segments():
     idx = np.repeat(np.arange(len(counts), dtype=np.int32), counts)
     np.random.default_rng(7).shuffle(idx)
     _experts_case(w, idx[:, None])
+    # T*k <= 64 rows (64-row A boxes when that layout is on): segments of 64
+    # rows down to 1
+    for counts in ([64], [40, 1, 16, 0, 7]):
+        w = _fp8(T=64, k=1, E=32, n_group=4, topk_group=2, d=512, inter=256)
+        idx = np.repeat(np.arange(len(counts), dtype=np.int32), counts)
+        np.random.default_rng(8).shuffle(idx)
+        _experts_case(w, idx[:, None])
 
 
 # --------------------------------------------------- device-limited routing
