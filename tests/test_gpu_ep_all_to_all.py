@@ -89,6 +89,14 @@ def test_all_to_all_fp8_experts_group_routing():
     _check(base, 2, tol=TOL_FP8)
 
 
+def test_all_to_all_fp8_small_batch():
+    # 8 tokens per rank, top-4 of 64 experts over 2 ranks: each rank receives
+    # at most 64 rows, so its local e4m3 GEMMs run the small-batch stage layout
+    base = workloads.make_small("fp8", T=8, d=512, E=64, k=4, inter=256, shared_inter=256, n_group=8,
+                                topk_group=2)
+    _check(base, 2, tol=TOL_FP8)
+
+
 def test_all_to_all_fp8_chunked_driver_on_a_one_rank_nccl_group():
     import torch.distributed as dist
     base = to_device(workloads.make_small("fp8", T=300, d=512, E=64, k=6, inter=256, shared_inter=256, n_group=8,

@@ -498,13 +498,14 @@ def test_expert_utilisation_of_a_forward_pass():
 
 
 # ------------------------------------------------- expert parallelism (next row)
-@pytest.mark.parametrize("fp8,world", [(False, 2), (False, 4), (True, 2)])
-def test_forward_expert_parallel_shares_sum_to_the_layer(fp8, world):
+@pytest.mark.parametrize("fp8,world,T", [(False, 2, None), (False, 4, None), (True, 2, None), (True, 2, 48)])
+def test_forward_expert_parallel_shares_sum_to_the_layer(fp8, world, T):
     # every rank's share on this one GPU in turn (the all-reduce is the sum):
     # the sum matches the whole-layer launch up to fp32 summation order and
-    # the oracle within the layer's tolerance
+    # the oracle within the layer's tolerance (T=48: the FP8 small-batch
+    # stage layout on each rank's slice of the experts)
     from mixture_experts_ffn_17_b200 import expert_parallel as ep
-    w = _fp8() if fp8 else _medium(shared_inter=512)
+    w = (_fp8(T=T) if T else _fp8()) if fp8 else _medium(shared_inter=512)
     cfg = w.cfg
     y_full, idx, tw, counts, ws = run_forward(w)
     shape = B.shape_of(cfg)
